@@ -1,0 +1,160 @@
+"""Python access to the float64 CPU oracle (``pqk_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, the smoke check and the
+bench's CPU-baseline leg, never by the library. It shares no code with the
+CUDA path. Inputs are numpy arrays (bfloat16 as uint16 bit patterns, or
+float64); outputs are float64.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "pqk_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+ROPE_INTERLEAVED, ROPE_HALF = 0, 1
+NORM_RMS, NORM_LAYER, NORM_NONE = 0, 1, 2
+_IN_BF16, _IN_F64 = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (OpenMP, no fast-math)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-shared", "-fPIC",
+                               "-o", tmp, SRC, "-lm"])
+        os.replace(tmp, LIB)
+    return LIB
+
+
+def load(path: str):
+    """Load an oracle build from ``path`` and declare its signatures."""
+    L = C.CDLL(path)
+    vp, i32p, f32p, f64p = C.c_void_p, C.POINTER(C.c_int32), C.POINTER(C.c_float), C.POINTER(C.c_double)
+    L.oracle_qk_norm_rope.argtypes = [vp, C.c_int, C.c_int64, vp, C.c_int, i32p, C.c_int64, C.c_int,
+                                      C.c_int, C.c_double, C.c_double, C.c_int, i32p, C.c_int64, f64p]
+    L.oracle_varlen_attn.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
+                                     C.c_int, C.c_double, i32p, C.c_int64, f64p, f64p]
+    L.oracle_modulate_swiglu.argtypes = [vp, vp, C.c_int, f32p, f32p, f32p, i32p, C.c_int, C.c_int64,
+                                         C.c_int, C.c_int, C.c_double, vp, vp, C.c_int64, C.c_int, i32p,
+                                         C.c_int64, f64p, f64p, f64p]
+    for f in (L.oracle_qk_norm_rope, L.oracle_varlen_attn, L.oracle_modulate_swiglu):
+        f.restype = C.c_int
+    L.oracle_num_threads.restype = C.c_int
+    return L
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = load(LIB)
+    return _lib
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
+
+
+def _kind(a: np.ndarray) -> int:
+    if a.dtype == np.uint16:
+        return _IN_BF16
+    if a.dtype == np.float64:
+        return _IN_F64
+    raise TypeError(f"oracle inputs are bf16 bits (uint16) or float64, got {a.dtype}")
+
+
+def _ptr(a, ctype=None):
+    if a is None:
+        return None
+    if ctype is None:
+        return a.ctypes.data_as(C.c_void_p)
+    return a.ctypes.data_as(C.POINTER(ctype))
+
+
+def _rows(rows):
+    if rows is None:
+        return None, 0
+    r = np.ascontiguousarray(rows, dtype=np.int32)
+    return r, int(r.shape[0])
+
+
+def qk_norm_rope(x: np.ndarray, w: np.ndarray, pos: np.ndarray, eps: float, base: float,
+                 style: int = ROPE_INTERLEAVED, rows=None) -> np.ndarray:
+    """x: [T, H, D] (a strided view over a wider token row is allowed)."""
+    T, H, D = x.shape
+    stride_t = x.strides[0] // x.itemsize
+    assert x.strides[2] == x.itemsize and x.strides[1] == D * x.itemsize
+    # a strided token view is passed by its first element; stride_t covers
+    # the gap between tokens
+    w = np.ascontiguousarray(w)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    r, n = _rows(rows)
+    y = np.empty((n if r is not None else T, H, D), np.float64)
+    rc = lib().oracle_qk_norm_rope(_ptr(x), _kind(x), stride_t, _ptr(w), _kind(w), _ptr(pos, C.c_int32),
+                                   T, H, D, eps, base, style, _ptr(r, C.c_int32), n, _ptr(y, C.c_double))
+    if rc:
+        raise ValueError("oracle_qk_norm_rope: invalid arguments")
+    return y
+
+
+def varlen_attn(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float,
+                rows=None, want_lse: bool = True):
+    """q, k, v: [T, H, D] contiguous. Returns (o [nrows, H, D], lse [nrows, H])."""
+    T, H, D = q.shape
+    assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
+    q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    r, n = _rows(rows)
+    n = n if r is not None else T
+    o = np.empty((n, H, D), np.float64)
+    lse = np.empty((n, H), np.float64) if want_lse else None
+    rc = lib().oracle_varlen_attn(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32),
+                                  int(cu.shape[0]) - 1, T, H, D, scale, _ptr(r, C.c_int32), n if r is not None else 0,
+                                  _ptr(o, C.c_double), _ptr(lse, C.c_double))
+    if rc:
+        raise ValueError("oracle_varlen_attn: invalid arguments")
+    return o, lse
+
+
+def modulate_swiglu(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, gate_res: np.ndarray,
+                    cu_seqlens: np.ndarray, norm_type: int = NORM_RMS, eps: float = 1e-6,
+                    branch=None, gate=None, up=None, rows=None):
+    """Returns (x_out or None, h, act or None), float64."""
+    T, Cdim = x.shape
+    x = np.ascontiguousarray(x)
+    if branch is not None:
+        branch = np.ascontiguousarray(branch)
+        assert branch.dtype == x.dtype and branch.shape == x.shape
+    shift, scale, gate_res = (np.ascontiguousarray(a, dtype=np.float32) for a in (shift, scale, gate_res))
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    F, gu_stride = 0, 0
+    if gate is not None:
+        assert up is not None and gate.shape == up.shape and gate.dtype == x.dtype
+        F = gate.shape[1]
+        gate, up = np.ascontiguousarray(gate), np.ascontiguousarray(up)
+        gu_stride = F
+    r, n = _rows(rows)
+    n = n if r is not None else T
+    xo = np.empty((n, Cdim), np.float64) if branch is not None else None
+    h = np.empty((n, Cdim), np.float64)
+    act = np.empty((n, F), np.float64) if gate is not None else None
+    rc = lib().oracle_modulate_swiglu(_ptr(x), _ptr(branch), _kind(x), _ptr(shift, C.c_float),
+                                      _ptr(scale, C.c_float), _ptr(gate_res, C.c_float), _ptr(cu, C.c_int32),
+                                      int(cu.shape[0]) - 1, T, Cdim, norm_type, eps, _ptr(gate), _ptr(up),
+                                      gu_stride, F, _ptr(r, C.c_int32), n if r is not None else 0,
+                                      _ptr(xo, C.c_double), _ptr(h, C.c_double), _ptr(act, C.c_double))
+    if rc:
+        raise ValueError("oracle_modulate_swiglu: invalid arguments")
+    return xo, h, act

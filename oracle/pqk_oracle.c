@@ -1,0 +1,254 @@
+/*
+ * pqk_oracle.c -- plain float64 CPU oracle for the DiT-block hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the bench's
+ * CPU-baseline leg load this library. The CUDA library never links, includes
+ * or calls it, and it shares no code, header, table or constant with it.
+ *
+ * What it computes, and where the pages say so:
+ *   oracle_qk_norm_rope    -- Q/K normalisation merged with RoPE
+ *                             ("FastH3 在八卡 B300 上实现完整 MP4 生成快于播放时长",
+ *                             section "融合 DiT 算子"; "MiniMax H3 FastH3 real-time
+ *                             serving with vLLM-Omni", section "System-wide
+ *                             optimizations in vLLM-Omni", bullet "Fused DiT
+ *                             operators").
+ *   oracle_varlen_attn     -- softmax attention over one packed sequence per
+ *                             request, valid tokens only (first page, section
+ *                             "长序列注意力与通信优化"; second page, bullet
+ *                             "Long-sequence attention & communication").
+ *   oracle_modulate_swiglu -- modulation + normalisation + gated residual and
+ *                             SwiGLU in place of separate SiLU and multiply
+ *                             (first page "融合 DiT 算子"; second page bullet
+ *                             "Fused DiT operators").
+ *
+ * The pages state the operations, not their conventions; the readings taken
+ * where they are silent (norm per head over head_dim, norm before RoPE,
+ * theta_j = base^(-2j/D), pairing, adaLN as h = n*(1+scale)+shift with one
+ * vector set per request, x' = x + g*branch, SwiGLU = silu(gate)*up, the
+ * softmax scale passed by the caller, LSE in natural log) are listed with
+ * the pins that check each function in the repository's design notes. All
+ * three functions are pinned by closed forms, brute force and invariants in
+ * the CPU test suite.
+ *
+ * Every function is the plain definition: no blocking, fusion or
+ * reordering. Inputs are either bfloat16 bit patterns (widened exactly) or
+ * float64 values, selected per call.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_IN_BF16 0
+#define ORACLE_IN_F64 1
+
+#define ORACLE_ROPE_INTERLEAVED 0 /* pairs (2j, 2j+1) */
+#define ORACLE_ROPE_HALF 1        /* pairs (j, j + D/2) */
+
+#define ORACLE_NORM_RMS 0
+#define ORACLE_NORM_LAYER 1
+#define ORACLE_NORM_NONE 2
+
+/* Exact widening of a bfloat16 bit pattern: its bits are the top half of an
+ * IEEE binary32. */
+static double bf16_bits_to_double(uint16_t b) {
+  uint32_t u = ((uint32_t)b) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Element i of a buffer given as bf16 bits or as float64. */
+static double load(const void* p, int kind, int64_t i) {
+  if (kind == ORACLE_IN_BF16) return bf16_bits_to_double(((const uint16_t*)p)[i]);
+  return ((const double*)p)[i];
+}
+
+/* Segment s with cu[s] <= t < cu[s+1]; -1 if none. Linear scan: the plain
+ * definition of "the request that token t belongs to". */
+static int segment_of(const int32_t* cu, int B, int64_t t) {
+  for (int s = 0; s < B; ++s)
+    if (cu[s] <= t && t < cu[s + 1]) return s;
+  return -1;
+}
+
+static int check_cu(const int32_t* cu, int B, int64_t T) {
+  if (B < 0 || cu == NULL) return -1;
+  if (cu[0] != 0 || cu[B] != T) return -1;
+  for (int s = 0; s < B; ++s)
+    if (cu[s + 1] < cu[s]) return -1;
+  return 0;
+}
+
+/*
+ * RMSNorm over the D elements of one (token, head) row, weight w (shared by
+ * all heads), then RoPE with angle phi_j = pos[t] * base^(-2j/D), j < D/2:
+ *   (a, b) <- (a cos phi - b sin phi, a sin phi + b cos phi).
+ * x: [T, H, D] with stride_t elements between tokens (a fused QKV buffer
+ * has stride_t > H*D). rows: token indices to evaluate (NULL = all T).
+ * y: [nrows, H, D] float64 contiguous.
+ */
+int oracle_qk_norm_rope(const void* x, int x_kind, int64_t stride_t, const void* w, int w_kind,
+                        const int32_t* pos, int64_t T, int H, int D, double eps, double base,
+                        int style, const int32_t* rows, int64_t nrows, double* y) {
+  if (D <= 0 || D % 2 || H <= 0 || T < 0 || !(eps >= 0.0) || !(base > 0.0)) return -1;
+  if (style != ORACLE_ROPE_INTERLEAVED && style != ORACLE_ROPE_HALF) return -1;
+  if (rows == NULL) nrows = T;
+  int64_t bad = 0;
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int64_t t = rows ? rows[r] : r;
+    if (t < 0 || t >= T) { ++bad; continue; }
+    double* n = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int h = 0; h < H; ++h) {
+      const int64_t base_idx = t * stride_t + (int64_t)h * D;
+      double ms = 0.0;
+      for (int d = 0; d < D; ++d) {
+        double v = load(x, x_kind, base_idx + d);
+        ms += v * v;
+      }
+      ms /= (double)D;
+      const double inv = 1.0 / sqrt(ms + eps);
+      for (int d = 0; d < D; ++d) n[d] = load(x, x_kind, base_idx + d) * inv * load(w, w_kind, d);
+      double* out = y + (r * H + h) * (int64_t)D;
+      for (int j = 0; j < D / 2; ++j) {
+        const double theta = pow(base, -2.0 * (double)j / (double)D);
+        const double phi = (double)pos[t] * theta;
+        int ia, ib;
+        if (style == ORACLE_ROPE_INTERLEAVED) { ia = 2 * j; ib = 2 * j + 1; }
+        else { ia = j; ib = j + D / 2; }
+        const double a = n[ia], b = n[ib];
+        out[ia] = a * cos(phi) - b * sin(phi);
+        out[ib] = a * sin(phi) + b * cos(phi);
+      }
+    }
+    free(n);
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * Packed variable-length attention, bidirectional within each request and
+ * nothing across requests. For token t in request i = [cu[i], cu[i+1]) and
+ * head h:
+ *   s_j = scale * <q_t, k_j>, j in request i
+ *   m = max_j s_j, p_j = exp(s_j - m), l = sum_j p_j
+ *   o_t = sum_j p_j v_j / l,  lse_t = m + ln l.
+ * q, k, v: [T, H, D], stride_t elements between tokens. o: [nrows, H, D];
+ * lse: [nrows, H] or NULL.
+ */
+int oracle_varlen_attn(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
+                       const int32_t* cu, int B, int64_t T, int H, int D, double scale,
+                       const int32_t* rows, int64_t nrows, double* o, double* lse) {
+  if (check_cu(cu, B, T) || H <= 0 || D <= 0) return -1;
+  if (rows == NULL) nrows = T;
+  int64_t bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2) reduction(+ : bad)
+  for (int64_t r = 0; r < nrows; ++r) {
+    for (int h = 0; h < H; ++h) {
+      const int64_t t = rows ? rows[r] : r;
+      const int seg = (t >= 0 && t < T) ? segment_of(cu, B, t) : -1;
+      if (seg < 0) { ++bad; continue; }
+      const int64_t lo = cu[seg], L = (int64_t)cu[seg + 1] - cu[seg];
+      double* s = (double*)malloc(sizeof(double) * (size_t)L);
+      double* qt = (double*)malloc(sizeof(double) * (size_t)D);
+      for (int d = 0; d < D; ++d) qt[d] = load(q, in_kind, t * stride_t + (int64_t)h * D + d);
+      double m = -INFINITY;
+      for (int64_t j = 0; j < L; ++j) {
+        double acc = 0.0;
+        const int64_t kb = (lo + j) * stride_t + (int64_t)h * D;
+        for (int d = 0; d < D; ++d) acc += qt[d] * load(k, in_kind, kb + d);
+        s[j] = scale * acc;
+        if (s[j] > m) m = s[j];
+      }
+      double l = 0.0;
+      for (int64_t j = 0; j < L; ++j) { s[j] = exp(s[j] - m); l += s[j]; }
+      double* ot = o + (r * H + h) * (int64_t)D;
+      for (int d = 0; d < D; ++d) ot[d] = 0.0;
+      for (int64_t j = 0; j < L; ++j) {
+        const int64_t vb = (lo + j) * stride_t + (int64_t)h * D;
+        for (int d = 0; d < D; ++d) ot[d] += s[j] * load(v, in_kind, vb + d);
+      }
+      for (int d = 0; d < D; ++d) ot[d] /= l;
+      if (lse) lse[r * H + h] = m + log(l);
+      free(s);
+      free(qt);
+    }
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * Per token t of request s:
+ *   x'  = x + gate_res[s] * branch            (branch == NULL: x' = x)
+ *   n   = x' / sqrt(mean(x'^2) + eps)         (RMS, no affine)
+ *       = (x' - mu) / sqrt(var + eps)         (LAYER, biased variance)
+ *       = x'                                  (NONE)
+ *   h   = n * (1 + scale[s]) + shift[s]
+ *   act = gate / (1 + exp(-gate)) * up        (gate == NULL: skipped)
+ * x, branch: [T, C]; shift, scale, gate_res: [B, C] float32; gate, up:
+ * [T, F] with gu_stride elements between tokens. Outputs float64 with rows
+ * [nrows, C] / [nrows, F]; x_out may be NULL.
+ */
+int oracle_modulate_swiglu(const void* x, const void* branch, int in_kind, const float* shift,
+                           const float* scale, const float* gate_res, const int32_t* cu, int B,
+                           int64_t T, int C, int norm_type, double eps, const void* gate,
+                           const void* up, int64_t gu_stride, int F, const int32_t* rows,
+                           int64_t nrows, double* x_out, double* h_out, double* act_out) {
+  if (check_cu(cu, B, T) || C <= 0 || F < 0 || !(eps >= 0.0)) return -1;
+  if (norm_type != ORACLE_NORM_RMS && norm_type != ORACLE_NORM_LAYER && norm_type != ORACLE_NORM_NONE)
+    return -1;
+  if (rows == NULL) nrows = T;
+  int64_t bad = 0;
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t t = rows ? rows[r] : r;
+    const int seg = (t >= 0 && t < T) ? segment_of(cu, B, t) : -1;
+    if (seg < 0) { ++bad; continue; }
+    double* xp = (double*)malloc(sizeof(double) * (size_t)C);
+    for (int c = 0; c < C; ++c) {
+      double xv = load(x, in_kind, t * C + c);
+      if (branch) xv += (double)gate_res[(int64_t)seg * C + c] * load(branch, in_kind, t * C + c);
+      xp[c] = xv;
+      if (x_out) x_out[r * C + c] = xv;
+    }
+    double mu = 0.0, ms = 0.0, var = 0.0;
+    for (int c = 0; c < C; ++c) { mu += xp[c]; ms += xp[c] * xp[c]; }
+    mu /= (double)C;
+    ms /= (double)C;
+    for (int c = 0; c < C; ++c) var += (xp[c] - mu) * (xp[c] - mu);
+    var /= (double)C;
+    for (int c = 0; c < C; ++c) {
+      double n;
+      if (norm_type == ORACLE_NORM_RMS) n = xp[c] / sqrt(ms + eps);
+      else if (norm_type == ORACLE_NORM_LAYER) n = (xp[c] - mu) / sqrt(var + eps);
+      else n = xp[c];
+      h_out[r * C + c] = n * (1.0 + (double)scale[(int64_t)seg * C + c]) + (double)shift[(int64_t)seg * C + c];
+    }
+    if (gate && up && act_out) {
+      for (int f = 0; f < F; ++f) {
+        const double g = load(gate, in_kind, t * gu_stride + f);
+        const double u = load(up, in_kind, t * gu_stride + f);
+        act_out[r * (int64_t)F + f] = g / (1.0 + exp(-g)) * u;
+      }
+    }
+    free(xp);
+  }
+  return bad ? -1 : 0;
+}
+
+/* Number of OpenMP threads a parallel region of this library uses. */
+int oracle_num_threads(void) {
+  int n = 1;
+#ifdef _OPENMP
+#pragma omp parallel
+  {
+#pragma omp single
+    n = omp_get_num_threads();
+  }
+#endif
+  return n;
+}

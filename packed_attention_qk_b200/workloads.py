@@ -1,0 +1,277 @@
+"""Seeded synthetic workloads for the DiT-block hot path.
+
+This module only draws random numbers and lays out shapes. It holds none of
+the hot path's arithmetic, so both the float64 oracle (tests) and the CUDA
+path (library, bench) may take their inputs from it.
+
+Workload shapes follow the serving pages' description of the problem: one
+request is a joint text + audio + video token sequence of about 58k tokens
+packed without padding ("FastH3 在八卡 B300 上实现完整 MP4 生成快于播放时长",
+section "长序列注意力与通信优化"; "MiniMax H3 FastH3 real-time serving with
+vLLM-Omni", section "System-wide optimizations in vLLM-Omni"). The pages give
+no model dimensions; the head counts, widths and sequence mixes below are the
+five stated benchmark configurations.
+
+Recipe (every tensor has its own counter-independent stream, so a test can
+draw one tensor without drawing the others):
+  * stream for tensor ``name`` of config seed ``s``, chunk ``c`` =
+    ``numpy.random.Generator(PCG64(SeedSequence([s, TENSOR_ID[name], c])))``,
+    chunks of ``CHUNK`` elements in row-major order;
+  * activations Q, K, V, x, branch, gate, up ~ N(0, 1) drawn as float32, then
+    rounded once to bfloat16 (round to nearest even);
+  * RMSNorm weights w_q, w_k ~ U(0.5, 1.5), rounded to bfloat16;
+  * adaLN shift / scale / gated-residual gate ~ N(0, 0.1) kept in float32;
+  * outlier variant: an i.i.d. Bernoulli(0.001) mask over K's elements; masked
+    elements are multiplied by 20 in float32 before the bfloat16 rounding.
+bfloat16 tensors are returned as their uint16 bit patterns.
+"""
+
+from __future__ import annotations
+
+import concurrent.futures as _cf
+import os
+from dataclasses import dataclass, field
+
+import numpy as np
+
+CHUNK = 1 << 22
+
+TENSOR_ID = {
+    "q": 1, "k": 2, "v": 3, "x": 4, "branch": 5, "gate": 6, "up": 7,
+    "w_q": 8, "w_k": 9, "shift": 10, "scale": 11, "gate_res": 12,
+    "outlier": 13, "sample_rows": 14,
+}
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 (nearest even) and return the uint16 bits."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Exact widening of bfloat16 bits to float32."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    return bf16_bits_to_f32(b).astype(np.float64)
+
+
+def _chunk_rng(seed: int, name: str, chunk: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, TENSOR_ID[name], chunk])))
+
+
+def _draw(seed: int, name: str, n: int, kind: str, threads: int | None = None) -> np.ndarray:
+    """Draw ``n`` float32 values of distribution ``kind`` in chunks."""
+    out = np.empty(n, dtype=np.float32)
+    nchunks = (n + CHUNK - 1) // CHUNK
+
+    def fill(c: int) -> None:
+        lo, hi = c * CHUNK, min(n, (c + 1) * CHUNK)
+        g = _chunk_rng(seed, name, c)
+        if kind == "normal":
+            out[lo:hi] = g.standard_normal(hi - lo, dtype=np.float32)
+        elif kind == "normal01":
+            out[lo:hi] = g.standard_normal(hi - lo, dtype=np.float32) * np.float32(0.1)
+        elif kind == "uniform_w":
+            out[lo:hi] = g.uniform(0.5, 1.5, hi - lo).astype(np.float32)
+        elif kind == "bernoulli":
+            out[lo:hi] = (g.random(hi - lo, dtype=np.float32) < np.float32(0.001)).astype(np.float32)
+        else:
+            raise ValueError(kind)
+
+    if nchunks <= 1:
+        if nchunks:
+            fill(0)
+        return out
+    nt = threads or min(16, os.cpu_count() or 1)
+    with _cf.ThreadPoolExecutor(nt) as ex:
+        list(ex.map(fill, range(nchunks)))
+    return out
+
+
+def bf16_normal(seed: int, name: str, shape: tuple[int, ...]) -> np.ndarray:
+    n = int(np.prod(shape))
+    return f32_to_bf16_bits(_draw(seed, name, n, "normal")).reshape(shape)
+
+
+def bf16_weight(seed: int, name: str, d: int) -> np.ndarray:
+    return f32_to_bf16_bits(_draw(seed, name, d, "uniform_w"))
+
+
+def f32_modulation(seed: int, name: str, shape: tuple[int, ...]) -> np.ndarray:
+    n = int(np.prod(shape))
+    return _draw(seed, name, n, "normal01").reshape(shape)
+
+
+def bf16_k_with_outliers(seed: int, shape: tuple[int, ...]) -> np.ndarray:
+    """K for the outlier variant: 0.1% of entries multiplied by 20 before rounding."""
+    n = int(np.prod(shape))
+    k = _draw(seed, "k", n, "normal")
+    m = _draw(seed, "outlier", n, "bernoulli")
+    k = np.where(m > 0, k * np.float32(20.0), k)
+    return f32_to_bf16_bits(k).reshape(shape)
+
+
+# ----------------------------------------------------------------------------
+# Configurations
+# ----------------------------------------------------------------------------
+
+@dataclass
+class Workload:
+    name: str
+    seed: int
+    seg_lens: list[int]
+    H: int
+    D: int
+    C: int
+    F: int
+    # positions of each segment as a list of (modality, length) runs; ids
+    # restart at 0 for each run
+    pos_runs: list[list[int]] = field(default_factory=list)
+    rope_base: float = 10000.0
+    eps: float = 1e-6
+    attention: bool = True
+
+    @property
+    def T(self) -> int:
+        return int(sum(self.seg_lens))
+
+    @property
+    def B(self) -> int:
+        return len(self.seg_lens)
+
+    def cu_seqlens(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(self.seg_lens)]).astype(np.int32)
+
+    def positions(self) -> np.ndarray:
+        """Per-token RoPE ids; they restart at 0 for each modality run."""
+        parts = []
+        for runs in self.pos_runs:
+            for n in runs:
+                parts.append(np.arange(n, dtype=np.int32))
+        p = np.concatenate(parts) if parts else np.zeros(0, np.int32)
+        assert p.shape[0] == self.T
+        return p
+
+    def attn_flops(self) -> float:
+        """4*H*D per valid (query, key) pair within a request."""
+        return 4.0 * self.H * self.D * float(sum(int(L) * int(L) for L in self.seg_lens))
+
+    def prologue_bytes(self) -> int:
+        """qk_norm_rope: Q and K read + written (bf16) plus the int32 position."""
+        return self.T * (8 * self.H * self.D + 4)
+
+    def epilogue_bytes(self, with_branch: bool = False) -> int:
+        """modulate_swiglu: x (+branch, +x_out) in, h out; gate, up in; act out."""
+        per_tok = 2 * (2 * self.C + 3 * self.F) if not with_branch else 2 * (4 * self.C + 3 * self.F)
+        return self.T * per_tok
+
+
+def _c1() -> Workload:
+    return Workload("tiny packed attention block: 2 sequences 200+312 tokens, 4 heads, head_dim 64",
+                    0, [200, 312], H=4, D=64, C=256, F=512, pos_runs=[[200], [312]])
+
+
+def _c2() -> Workload:
+    return Workload("joint sequence of 4,096 tokens (text 256 + audio 512 + video 3,328), 16 heads, head_dim 128",
+                    1, [4096], H=16, D=128, C=2048, F=5632, pos_runs=[[256, 512, 3328]])
+
+
+def _c3() -> Workload:
+    # video tokens: 12 latent frames x 48 x 96; the flattened (t, h, w) id in
+    # token order is t*48*96 + h*96 + w, i.e. 0..55,295
+    return Workload("joint sequence of 58,048 tokens (text 512 + audio 2,240 + video 12x48x96), 24 heads, head_dim 128",
+                    2, [58048], H=24, D=128, C=3072, F=8192, pos_runs=[[512, 2240, 55296]])
+
+
+def _c4() -> Workload:
+    lens = [12345, 29024, 58048, 87072]
+    runs = [[12345], [29024], [512, 2240, 55296], [87072]]
+    return Workload("varlen batch of 4 requests 12,345/29,024/58,048/87,072 tokens, 24 heads, head_dim 128",
+                    3, lens, H=24, D=128, C=3072, F=8192, pos_runs=runs)
+
+
+def _c5(T: int) -> Workload:
+    return Workload(f"prologue/epilogue bandwidth sweep, {T} tokens, 40 heads x 128, hidden 5,120, ffn 13,824",
+                    4, [T], H=40, D=128, C=5120, F=13824, pos_runs=[[T]], attention=False)
+
+
+C5_TOKENS = (4096, 16384, 58048, 186489)
+
+
+def config(i: int, t5: int = 58048) -> Workload:
+    """The five benchmark configurations, 1-based like their numbering."""
+    if i == 1:
+        return _c1()
+    if i == 2:
+        return _c2()
+    if i == 3:
+        return _c3()
+    if i == 4:
+        return _c4()
+    if i == 5:
+        return _c5(t5)
+    raise ValueError(i)
+
+
+def custom(seg_lens: list[int], H: int, D: int, C: int | None = None, F: int | None = None,
+           seed: int = 100) -> Workload:
+    """Small ad-hoc shapes for edge-case tests; positions 0..L-1 per segment."""
+    C = C if C is not None else H * D
+    F = F if F is not None else 2 * C
+    return Workload(f"custom {seg_lens} H{H} D{D}", seed, list(seg_lens), H=H, D=D, C=C, F=F,
+                    pos_runs=[[L] for L in seg_lens])
+
+
+# ----------------------------------------------------------------------------
+# Tensor sets
+# ----------------------------------------------------------------------------
+
+def attention_inputs(w: Workload, outliers: bool = False) -> dict[str, np.ndarray]:
+    shp = (w.T, w.H, w.D)
+    k = bf16_k_with_outliers(w.seed, shp) if outliers else bf16_normal(w.seed, "k", shp)
+    return {"q": bf16_normal(w.seed, "q", shp), "k": k, "v": bf16_normal(w.seed, "v", shp),
+            "cu_seqlens": w.cu_seqlens()}
+
+
+def prologue_inputs(w: Workload) -> dict[str, np.ndarray]:
+    shp = (w.T, w.H, w.D)
+    return {"q": bf16_normal(w.seed, "q", shp), "k": bf16_normal(w.seed, "k", shp),
+            "w_q": bf16_weight(w.seed, "w_q", w.D), "w_k": bf16_weight(w.seed, "w_k", w.D),
+            "pos": w.positions()}
+
+
+def epilogue_inputs(w: Workload, with_branch: bool = False) -> dict[str, np.ndarray]:
+    d = {"x": bf16_normal(w.seed, "x", (w.T, w.C)),
+         "gate": bf16_normal(w.seed, "gate", (w.T, w.F)),
+         "up": bf16_normal(w.seed, "up", (w.T, w.F)),
+         "shift": f32_modulation(w.seed, "shift", (w.B, w.C)),
+         "scale": f32_modulation(w.seed, "scale", (w.B, w.C)),
+         "gate_res": f32_modulation(w.seed, "gate_res", (w.B, w.C)),
+         "cu_seqlens": w.cu_seqlens()}
+    if with_branch:
+        d["branch"] = bf16_normal(w.seed, "branch", (w.T, w.C))
+    return d
+
+
+def sample_rows(w: Workload, per_segment: int = 256) -> np.ndarray:
+    """Seeded query-row sample: per segment, its first and last row plus
+    ``per_segment - 2`` distinct rows drawn with seed (config seed + 1000)."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seed + 1000, TENSOR_ID["sample_rows"]])))
+    cu = w.cu_seqlens()
+    rows = []
+    for i in range(w.B):
+        lo, hi = int(cu[i]), int(cu[i + 1])
+        L = hi - lo
+        if L == 0:
+            continue
+        if L <= per_segment:
+            rows.append(np.arange(lo, hi))
+            continue
+        mid = g.choice(np.arange(lo + 1, hi - 1), size=per_segment - 2, replace=False)
+        rows.append(np.sort(np.concatenate([[lo], mid, [hi - 1]])))
+    return np.concatenate(rows).astype(np.int32) if rows else np.zeros(0, np.int32)

@@ -1,0 +1,54 @@
+"""Writes tests/golden/oracle_tiny_config.json: oracle outputs on the tiny
+packed-attention configuration (2 requests of 200 and 312 tokens, 4 heads,
+head_dim 64, hidden 256, ffn 512, seed 0). Calls only the oracle and the
+seeded input generators, so the stored numbers guard the oracle against
+unintended drift; they carry no authority of their own beyond that.
+
+Run from the repository root:  python tests/golden/make_golden.py
+"""
+
+import json
+import math
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+sys.path.insert(0, ROOT)
+
+from oracle import oracle  # noqa: E402
+from packed_attention_qk_b200 import workloads as wl  # noqa: E402
+
+ROWS = [0, 1, 199, 200, 311, 511]
+
+
+def summarise(a):
+    a = np.asarray(a, np.float64)
+    return {"sum": float(a.sum()), "abs_sum": float(np.abs(a).sum()), "sq_sum": float((a * a).sum())}
+
+
+def main():
+    w = wl.config(1)
+    p = wl.prologue_inputs(w)
+    a = wl.attention_inputs(w)
+    e = wl.epilogue_inputs(w, with_branch=True)
+    out = {"config": w.name, "rows": ROWS, "values_per_row": 8}
+    for style, tag in ((oracle.ROPE_INTERLEAVED, "interleaved"), (oracle.ROPE_HALF, "half")):
+        y = oracle.qk_norm_rope(p["q"], p["w_q"], p["pos"], w.eps, w.rope_base, style)
+        out[f"q_norm_rope_{tag}"] = {"summary": summarise(y), "head0": [y[r, 0, :8].tolist() for r in ROWS]}
+    o, lse = oracle.varlen_attn(a["q"], a["k"], a["v"], a["cu_seqlens"], 1.0 / math.sqrt(w.D))
+    out["attn_o"] = {"summary": summarise(o), "head0": [o[r, 0, :8].tolist() for r in ROWS]}
+    out["attn_lse"] = {"summary": summarise(lse), "rows": [lse[r].tolist() for r in ROWS]}
+    xo, h, act = oracle.modulate_swiglu(e["x"], e["shift"], e["scale"], e["gate_res"], e["cu_seqlens"],
+                                        branch=e["branch"], gate=e["gate"], up=e["up"], eps=w.eps)
+    for name, t in (("x_out", xo), ("h", h), ("act", act)):
+        out[name] = {"summary": summarise(t), "first": [t[r, :8].tolist() for r in ROWS]}
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "oracle_tiny_config.json")
+    with open(path, "w") as f:
+        json.dump(out, f, indent=1)
+    print("wrote", path)
+
+
+if __name__ == "__main__":
+    main()

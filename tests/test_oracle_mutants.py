@@ -1,0 +1,95 @@
+"""The oracle's pins must catch plausible mistakes (CPU only).
+
+Each case plants one mistake in a private copy of the oracle's C source (a
+dropped term, a wrong sign, index or exponent, swapped operands), builds it,
+points the oracle wrapper at that build and runs every pin of the three
+oracle test modules against it. A mutant that no pin rejects means the pins
+are too weak. Mistakes are planted only in the oracle, only on the CPU.
+"""
+
+import inspect
+import itertools
+import os
+import subprocess
+
+import pytest
+
+from oracle import oracle
+from tests import test_oracle_attention, test_oracle_modulate, test_oracle_norm_rope
+
+MUTANTS = {
+    "attn_drop_scale": ("s[j] = scale * acc;", "s[j] = acc;"),
+    "attn_value_row_of_query": ("const int64_t vb = (lo + j) * stride_t", "const int64_t vb = t * stride_t"),
+    "attn_lse_log2": ("lse[r * H + h] = m + log(l);", "lse[r * H + h] = m + log2(l);"),
+    "attn_drop_last_key": ("L = (int64_t)cu[seg + 1] - cu[seg];", "L = (int64_t)cu[seg + 1] - cu[seg] - 1;"),
+    "attn_no_normalise": ("ot[d] /= l;", "ot[d] /= 1.0;"),
+    "attn_key_from_other_head": ("const int64_t kb = (lo + j) * stride_t + (int64_t)h * D;",
+                                 "const int64_t kb = (lo + j) * stride_t;"),
+    "rope_sign": ("out[ia] = a * cos(phi) - b * sin(phi);", "out[ia] = a * cos(phi) + b * sin(phi);"),
+    "rope_exponent": ("pow(base, -2.0 * (double)j / (double)D)", "pow(base, -1.0 * (double)j / (double)D)"),
+    "rope_pairing_swapped": ("if (style == ORACLE_ROPE_INTERLEAVED) { ia = 2 * j;",
+                             "if (style != ORACLE_ROPE_INTERLEAVED) { ia = 2 * j;"),
+    "norm_eps_outside_sqrt": ("const double inv = 1.0 / sqrt(ms + eps);", "const double inv = 1.0 / (sqrt(ms) + eps);"),
+    "norm_sum_not_mean": ("ms /= (double)D;", "ms /= 1.0;"),
+    "norm_drop_weight": ("* inv * load(w, w_kind, d);", "* inv;"),
+    "mod_scale_not_offset": ("n * (1.0 + (double)scale[", "n * (0.0 + (double)scale["),
+    "mod_shift_of_first_request": ("+ (double)shift[(int64_t)seg * C + c];", "+ (double)shift[c];"),
+    "mod_residual_sign": ("if (branch) xv += ", "if (branch) xv -= "),
+    "mod_layer_unbiased": ("var /= (double)C;", "var /= (double)(C - 1);"),
+    "mod_rms_mean_subtracted": ("n = xp[c] / sqrt(ms + eps);", "n = (xp[c] - mu) / sqrt(ms + eps);"),
+    "silu_operands_swapped": ("act_out[r * (int64_t)F + f] = g / (1.0 + exp(-g)) * u;",
+                              "act_out[r * (int64_t)F + f] = u / (1.0 + exp(-u)) * g;"),
+    "silu_sign": ("g / (1.0 + exp(-g)) * u", "g / (1.0 + exp(g)) * u"),
+}
+
+
+def _pin_calls():
+    for mod in (test_oracle_attention, test_oracle_norm_rope, test_oracle_modulate):
+        for name, fn in inspect.getmembers(mod, inspect.isfunction):
+            if not name.startswith("test_") or fn.__module__ != mod.__name__:
+                continue
+            marks = [m for m in getattr(fn, "pytestmark", []) if m.name == "parametrize"]
+            if not marks:
+                yield f"{mod.__name__}.{name}", fn, {}
+                continue
+            names = [[n.strip() for n in m.args[0].split(",")] for m in marks]
+            for combo in itertools.product(*[m.args[1] for m in marks]):
+                kw = {}
+                for ns, vals in zip(names, combo):
+                    vals = vals if len(ns) > 1 else (vals,)
+                    kw.update(dict(zip(ns, vals)))
+                yield f"{mod.__name__}.{name}{kw}", fn, kw
+
+
+def _killed(lib_path):
+    saved = oracle._lib
+    oracle._lib = oracle.load(lib_path)
+    failures = []
+    try:
+        for label, fn, kw in _pin_calls():
+            try:
+                fn(**kw)
+            except (AssertionError, ValueError):
+                failures.append(label)
+    finally:
+        oracle._lib = saved
+    return failures
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_pins_reject_mutant(mutant, tmp_path):
+    old, new = MUTANTS[mutant]
+    src = open(oracle.SRC).read()
+    assert src.count(old) == 1, f"mutation site for {mutant} not found exactly once"
+    path = tmp_path / "m.c"
+    path.write_text(src.replace(old, new))
+    so = str(tmp_path / "libm.so")
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-shared", "-fPIC", "-o", so, str(path), "-lm"])
+    failures = _killed(so)
+    assert failures, f"no pin rejects mutant {mutant}"
+
+
+def test_unmutated_build_passes_every_pin(tmp_path):
+    so = str(tmp_path / "lib0.so")
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-shared", "-fPIC", "-o", so, oracle.SRC, "-lm"])
+    assert _killed(so) == []
