@@ -1,0 +1,381 @@
+"""Benchmark of one DiT-block hot-path step on B200.
+
+A step is one block call over one request of the 58,048-token joint
+text + audio + video sequence (24 heads x 128, hidden 3,072, FFN 8,192):
+  qk_norm_rope (Q, K)  ->  varlen_attn_fwd (Q, K, V)  ->
+  modulate_swiglu (x + gate_res * O as the gated residual, adaLN
+  modulation, SwiGLU on gate / up),
+all through the C ABI of libpqk. The dense projections between them are
+outside the hot path; seeded synthetic tensors stand in for their outputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). ``value`` is attention FLOPs of all ranks
+per second of device time of the whole step (max over ranks); the kernel
+figures and the roofline of the dominant kernel (the attention) are in the
+same line. With N > 1 (torchrun) every rank runs its own request: weak
+scaling, no collective on the data path.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "varlen attn TFLOP/s @58k tokens (% bf16 peak); fused DiT-op HBM GB/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_traffic.json")
+ATTN_SRC = os.path.join(ROOT, "packed_attention_qk_b200", "csrc", "varlen_attn_fwd.cu")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=3, help="workload number (3 = 58,048-token joint sequence)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        d = json.load(open(PEAKS_FILE))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def attn_traffic():
+    """Per-launch DRAM bytes of the attention kernel from a committed ncu
+    capture, or None when the kernel source changed since."""
+    try:
+        d = json.load(open(TRAFFIC_FILE))
+    except Exception:
+        return None
+    if d.get("source_sha256_16") != source_hash(ATTN_SRC):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index, enabled=True):
+        self.gpu, self.enabled, self.lines, self.proc = gpu_index, enabled, [], None
+
+    def __enter__(self):
+        if self.enabled:
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                              "-i", str(self.gpu), "-lms", "200"], stdout=subprocess.PIPE,
+                                             stderr=subprocess.DEVNULL, text=True)
+                self.t = threading.Thread(target=self._read, daemon=True)
+                self.t.start()
+            except Exception:
+                self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ inputs
+
+def make_inputs(w, device):
+    import torch
+    from packed_attention_qk_b200 import workloads as wl
+
+    def dev16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+    p = wl.prologue_inputs(w)
+    a = {"v": wl.bf16_normal(w.seed, "v", (w.T, w.H, w.D))}
+    e = wl.epilogue_inputs(w, with_branch=False)
+    d = {"q": dev16(p["q"]), "k": dev16(p["k"]), "v": dev16(a["v"]), "w_q": dev16(p["w_q"]),
+         "w_k": dev16(p["w_k"]), "pos": torch.from_numpy(p["pos"]).to(device),
+         "cu": torch.from_numpy(w.cu_seqlens()).to(device), "x": dev16(e["x"]), "gate": dev16(e["gate"]),
+         "up": dev16(e["up"]), "shift": torch.from_numpy(e["shift"]).to(device),
+         "scale": torch.from_numpy(e["scale"]).to(device), "gate_res": torch.from_numpy(e["gate_res"]).to(device)}
+    return d
+
+
+def alloc_outputs(w, d):
+    import torch
+    from packed_attention_qk_b200 import pqk
+    o = {"qn": torch.empty_like(d["q"]), "kn": torch.empty_like(d["k"]), "o": torch.empty_like(d["q"]),
+         "x_out": torch.empty_like(d["x"]), "h": torch.empty_like(d["x"]),
+         "act": torch.empty((w.T, w.F), dtype=torch.bfloat16, device=d["x"].device),
+         "ws": torch.empty(pqk.varlen_attn_workspace_size(w.B), dtype=torch.uint8, device=d["x"].device)}
+    return o
+
+
+def block_call(w, d, o, ev=None):
+    """One step: the three C-ABI calls on the current stream. ``ev`` (4
+    events) brackets the kernels for per-kernel device times."""
+    from packed_attention_qk_b200 import pqk
+    if ev:
+        ev[0].record()
+    pqk.qk_norm_rope(d["q"], d["k"], d["w_q"], d["w_k"], d["pos"], eps=w.eps, rope_base=w.rope_base,
+                     q_out=o["qn"], k_out=o["kn"])
+    if ev:
+        ev[1].record()
+    pqk.varlen_attn_fwd(o["qn"], o["kn"], d["v"], d["cu"], o=o["o"], workspace=o["ws"])
+    if ev:
+        ev[2].record()
+    pqk.modulate_swiglu(d["x"], d["shift"], d["scale"], d["cu"], gate_res=d["gate_res"],
+                        branch=o["o"].view(w.T, w.C), gate=d["gate"], up=d["up"], eps=w.eps, x_out=o["x_out"],
+                        h=o["h"], act=o["act"])
+    if ev:
+        ev[3].record()
+
+
+LAUNCHES_PER_STEP = 4  # qk_norm_rope, schedule builder, attention, modulate_swiglu
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def cpu_baseline_sample(w, rows_per_request, seed_rows=None):
+    """Times the oracle's attention on a seeded sample of query rows (all
+    heads, full keys). Returns (TFLOP/s, seconds, rows, threads)."""
+    from oracle import oracle
+    from packed_attention_qk_b200 import workloads as wl
+    x = wl.attention_inputs(w)
+    rows = wl.sample_rows(w, rows_per_request)
+    cu = w.cu_seqlens()
+    seg = np.searchsorted(cu, rows, side="right") - 1
+    flops = float(sum(4.0 * w.H * w.D * (cu[s + 1] - cu[s]) for s in seg))
+    t0 = time.perf_counter()
+    oracle.varlen_attn(x["q"], x["k"], x["v"], cu, 1.0 / math.sqrt(w.D), rows=rows)
+    dt = time.perf_counter() - t0
+    return flops / dt / 1e12, dt, int(len(rows)), oracle.num_threads()
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args, w):
+    """The oracle, as it stands, on host cores: each step is the attention
+    over a bounded seeded sample of query rows of the same workload."""
+    from oracle import oracle
+    from packed_attention_qk_b200 import workloads as wl
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    x = wl.attention_inputs(w)
+    cu = w.cu_seqlens()
+    rows = wl.sample_rows(w, 16)
+    seg = np.searchsorted(cu, rows, side="right") - 1
+    flops = float(sum(4.0 * w.H * w.D * (cu[s + 1] - cu[s]) for s in seg))
+    for _ in range(args.warmup):
+        oracle.varlen_attn(x["q"], x["k"], x["v"], cu, 1.0 / math.sqrt(w.D), rows=rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.varlen_attn(x["q"], x["k"], x["v"], cu, 1.0 / math.sqrt(w.D), rows=rows)
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    sample = f"{len(rows)} query rows x {w.H} heads x all {w.T} keys per step (float64 oracle)"
+    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": w.name, "tokens": w.T, "heads": w.H, "head_dim": w.D},
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    from packed_attention_qk_b200 import pqk
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    d = make_inputs(w, dev)
+    o = alloc_outputs(w, d)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        block_call(w, d, o)
+    torch.cuda.synchronize()
+    if pqk.get_device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local, enabled=not args.no_clocks) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        start.record()
+        for i in range(K):
+            block_call(w, d, o, evs[i])
+        stop.record()
+        torch.cuda.synchronize()
+        barrier()
+    total_ms = max_over_ranks(start.elapsed_time(stop))
+    if pqk.get_device_status() != 0:
+        raise RuntimeError("device status set during the timed steps")
+    pro = [e[0].elapsed_time(e[1]) for e in evs]
+    att = [e[1].elapsed_time(e[2]) for e in evs]
+    epi = [e[2].elapsed_time(e[3]) for e in evs]
+    ms_step = total_ms / K
+    flops = w.attn_flops()
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    att_ms = statistics.mean(att)
+    pk, pk_kind = peaks()
+    attn_tflops = flops / (att_ms * 1e-3) / 1e12
+    pro_gbs = w.prologue_bytes() / (statistics.mean(pro) * 1e-3) / 1e9
+    epi_bytes = w.epilogue_bytes(with_branch=True)
+    epi_gbs = epi_bytes / (statistics.mean(epi) * 1e-3) / 1e9
+
+    # e2e through host buffers: pinned H2D of every input, the three calls,
+    # D2H of the block outputs (x', h, act), all inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host_in = {k: d[k].cpu().pin_memory() for k in ("q", "k", "v", "x", "gate", "up", "w_q", "w_k", "pos", "cu",
+                                                          "shift", "scale", "gate_res")}
+        host_out = {k: torch.empty(o[k].shape, dtype=o[k].dtype, pin_memory=True) for k in ("x_out", "h", "act")}
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+        e2e_steps = max(2, min(K, 5))
+
+        def e2e_step():
+            for k, t in host_in.items():
+                d[k].copy_(t, non_blocking=True)
+            block_call(w, d, o)
+            for k, t in host_out.items():
+                t.copy_(o[k], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for _ in range(e2e_steps):
+            e2e_step()
+        t2.record()
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(s2.elapsed_time(t2)) / e2e_steps
+        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, secs, nrows, cores = cpu_baseline_sample(w, 96)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"attention of {nrows} seeded query rows x {w.H} heads over all keys of their request "
+                         f"(float64 oracle, {secs:.1f} s)"}
+
+    traffic = attn_traffic()
+    peak = pk["bf16_tflops_sustained"]
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "tokens_per_gpu": w.T, "requests_per_gpu": w.B, "heads": w.H,
+                   "head_dim": w.D, "hidden": w.C, "ffn": w.F,
+                   "l2": "inputs larger than L2 (Q, K, V 357 MB each; prologue 1.43 GB; epilogue 4.3 GB)"},
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": attn_tflops / peak, "traffic": traffic,
+                     "peak_kind": f"{pk_kind} bf16 sustained (kernel inside a long step)",
+                     "frac_of_nominal_2250": attn_tflops / 2250.0},
+        "kernels": {"qk_norm_rope_us": statistics.mean(pro) * 1e3, "qk_norm_rope_gbs": pro_gbs,
+                    "qk_norm_rope_frac_hbm": pro_gbs / pk["hbm_gbs"],
+                    "varlen_attn_ms": att_ms, "varlen_attn_tflops": attn_tflops,
+                    "modulate_swiglu_us": statistics.mean(epi) * 1e3, "modulate_swiglu_gbs": epi_gbs,
+                    "modulate_swiglu_frac_hbm": epi_gbs / pk["hbm_gbs"], "hbm_peak_gbs": pk["hbm_gbs"]},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    from packed_attention_qk_b200 import workloads as wl
+    w = wl.config(args.config)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,202 @@
+/*
+ * pqk.h -- C ABI of libpqk, the B200 (sm_100a) hot path of one block of a
+ * joint video + audio diffusion transformer: fused Q/K RMSNorm + RoPE,
+ * packed variable-length self-attention, and fused adaLN modulation +
+ * gated residual + SwiGLU.
+ *
+ * Source of the operations: "FastH3 在八卡 B300 上实现完整 MP4 生成快于播放时长"
+ * (sections "长序列注意力与通信优化" and "融合 DiT 算子") and "MiniMax H3 FastH3
+ * real-time serving with vLLM-Omni" (section "System-wide optimizations in
+ * vLLM-Omni", bullets "Long-sequence attention & communication" and "Fused
+ * DiT operators"). The pages describe what is fused and that packed
+ * sequences carry no padding; the conventions they leave open are fixed
+ * below and stated per call.
+ *
+ * General contract
+ *   - Every pointer argument named *device* is CUDA device memory owned by the
+ *     caller; the library allocates nothing and keeps no per-call state.
+ *   - bf16 means IEEE bfloat16 (2 bytes). Tensors are row-major as stated.
+ *   - Every device pointer must be 16-byte aligned; every row stride is in
+ *     elements and must be a multiple of 8 (16 bytes).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Every call is asynchronous on it: it validates its arguments
+ *     on the host, enqueues kernels and returns. Argument errors are
+ *     reported before anything is enqueued.
+ *   - Return value: PQK_OK (0) or a negative pqk_status. Conditions found by
+ *     the GPU while running (invalid cu_seqlens contents, a pipeline wait
+ *     that ran out) are written to a per-device status word; read it with
+ *     pqk_get_device_status after the work completes.
+ *   - All calls are deterministic: the same inputs give bit-identical
+ *     outputs on every run (no floating-point atomics, fixed reduction
+ *     order).
+ *   - Input and output buffers must not partially overlap. Exact in-place
+ *     use (output pointer == input pointer, same layout) is allowed where
+ *     stated.
+ */
+#ifndef PQK_H
+#define PQK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PQK_API __attribute__((visibility("default")))
+#else
+#define PQK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PQK_OK = 0,
+  PQK_ERR_INVALID_ARG = -1,  /* null pointer, bad size, bad enum value */
+  PQK_ERR_UNSUPPORTED = -2,  /* head_dim or device not supported */
+  PQK_ERR_MISALIGNED = -3,   /* pointer or stride not 16-byte aligned */
+  PQK_ERR_CUDA = -4,         /* a CUDA runtime call failed */
+  PQK_ERR_WORKSPACE = -5,    /* workspace missing or too small */
+  PQK_ERR_TIMEOUT = -6,      /* device: a bounded pipeline wait ran out */
+  PQK_ERR_BAD_SEQLENS = -7   /* device: cu_seqlens not 0 <= ... <= T, monotone */
+} pqk_status;
+
+/* RoPE pairing. INTERLEAVED rotates (x[2j], x[2j+1]); HALF rotates
+ * (x[j], x[j + D/2]). */
+typedef enum { PQK_ROPE_INTERLEAVED = 0, PQK_ROPE_HALF = 1 } pqk_rope_style;
+
+/* Normalisation of modulate_swiglu. RMS: x / sqrt(mean(x^2) + eps).
+ * LAYER: (x - mean) / sqrt(biased var + eps). NONE: x. No affine weight. */
+typedef enum { PQK_NORM_RMS = 0, PQK_NORM_LAYER = 1, PQK_NORM_NONE = 2 } pqk_norm_type;
+
+/*
+ * pqk_qk_norm_rope -- fused Q/K RMSNorm + RoPE ("Q/K normalisation merged
+ * with RoPE": first page, section "融合 DiT 算子"; second page, bullet "Fused
+ * DiT operators").
+ *
+ * For every token t < T, head h < H and X in {Q, K}, on the D elements x of
+ * row (t, h):
+ *   y_d  = x_d / sqrt(mean_d(x_d^2) + eps) * w_X[d]        (norm per head)
+ *   (a, b) <- (a cos phi - b sin phi, a sin phi + b cos phi) for every pair
+ *   of pqk_rope_style j < D/2, phi = pos[t] * rope_base^(-2j/D).
+ * Arithmetic in fp32 with the angle formed and reduced in fp64; outputs are
+ * rounded to bf16 (nearest even).
+ *
+ * q_in, k_in    device bf16 [T, H, D], q_stride_t / k_stride_t elements
+ *               between consecutive tokens (>= H*D; a fused QKV row works).
+ * q_out, k_out  device bf16, same layout and strides as the inputs; may
+ *               equal q_in / k_in (in place).
+ * q_weight, k_weight  device bf16 [D], shared by all heads.
+ * pos           device int32 [T], RoPE position id of every token.
+ * D             64 or 128. T >= 0 (T == 0 enqueues nothing). eps > 0.
+ */
+PQK_API int pqk_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                     int64_t q_stride_t, int64_t k_stride_t, const void* q_weight,
+                     const void* k_weight, const int32_t* pos, int64_t T, int H, int D,
+                     float eps, float rope_base, int rope_style, void* stream);
+
+/*
+ * pqk_varlen_attn_workspace_size -- bytes of device workspace that
+ * pqk_varlen_attn_fwd needs for B requests (its tile schedule).
+ */
+PQK_API size_t pqk_varlen_attn_workspace_size(int B);
+
+/*
+ * pqk_varlen_attn_fwd -- packed variable-length self-attention over one
+ * unpadded sequence per request, valid tokens only (first page, section
+ * "长序列注意力与通信优化"; second page, bullet "Long-sequence attention &
+ * communication").
+ *
+ * Request i covers tokens [cu_seqlens[i], cu_seqlens[i+1]). For every token
+ * t of request i and head h:
+ *   O[t, h] = sum_j softmax_j(softmax_scale * <Q[t, h], K[j, h]>) V[j, h],
+ *   j over request i only (bidirectional inside a request, nothing across),
+ *   lse[h, t] = ln sum_j exp(softmax_scale * <Q[t, h], K[j, h]>).
+ * bf16 tensor-core products with fp32 accumulation; probabilities are
+ * rounded to bf16 before the second product; O rounded to bf16.
+ *
+ * q, k, v       device bf16 [T, H, D], q_stride_t / k_stride_t / v_stride_t
+ *               elements between tokens (>= H*D).
+ * o             device bf16 [T, H, D], o_stride_t elements between tokens;
+ *               must not overlap q, k or v.
+ * lse           device fp32 [H, T] or NULL.
+ * cu_seqlens    device int32 [B+1], 0 = cu[0] <= cu[1] <= ... <= cu[B] = T;
+ *               empty requests are allowed. Checked on the device: a
+ *               violation sets PQK_ERR_BAD_SEQLENS in the status word and
+ *               the call writes no output.
+ * D             64 or 128. B >= 1, T >= 0.
+ * workspace     device memory of at least pqk_varlen_attn_workspace_size(B)
+ *               bytes, 16-byte aligned; it only holds this call's schedule
+ *               and may be reused once the call has completed on `stream`.
+ */
+PQK_API int pqk_varlen_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int64_t q_stride_t, int64_t k_stride_t, int64_t v_stride_t,
+                        int64_t o_stride_t, const int32_t* cu_seqlens, int B, int64_t T, int H,
+                        int D, float softmax_scale, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
+ * pqk_modulate_swiglu -- fused adaLN modulation + normalisation + gated
+ * residual, and SwiGLU in one pass (first page, section "融合 DiT 算子": the
+ * small DiT operators RMSNorm, SwiGLU and residual connections fused, SwiGLU
+ * in place of separate SiLU and multiply; second page, bullet "Fused DiT
+ * operators": modulation and normalization among them).
+ *
+ * For every token t of request s (cu_seqlens as in pqk_varlen_attn_fwd):
+ *   x'  = x[t] + gate_res[s] * branch[t]       (branch == NULL: x' = x[t])
+ *   h   = norm(x') * (1 + scale[s]) + shift[s] (pqk_norm_type over C)
+ *   act = silu(gate[t]) * up[t],  silu(g) = g / (1 + exp(-g))
+ * fp32 arithmetic on bf16 inputs, outputs rounded to bf16.
+ *
+ * x, branch     device bf16 [T, C] (branch may be NULL).
+ * x_out         device bf16 [T, C] receiving x', or NULL; may equal x.
+ * h             device bf16 [T, C]; may equal x.
+ * shift, scale  device fp32 [B, C]; gate_res device fp32 [B, C], may be
+ *               NULL when branch is NULL.
+ * cu_seqlens    device int32 [B+1] (must be valid; not re-checked here).
+ * gate, up      device bf16 [T, F] rows gu_stride_t elements apart (the two
+ *               halves of one [T, 2F] buffer work); both NULL skips SwiGLU.
+ * act           device bf16 [T, F] contiguous; may equal gate when
+ *               gu_stride_t == F.
+ * C, F          multiples of 8; C <= 16384. B >= 1, T >= 0, eps > 0.
+ */
+PQK_API int pqk_modulate_swiglu(const void* x, const void* branch, void* x_out, void* h,
+                        const float* shift, const float* scale, const float* gate_res,
+                        const int32_t* cu_seqlens, int B, int64_t T, int C, int norm_type,
+                        float eps, const void* gate, const void* up, int64_t gu_stride_t,
+                        void* act, int F, void* stream);
+
+/*
+ * pqk_get_device_status -- synchronises `stream`, then returns and clears
+ * the current device's status word: PQK_OK, PQK_ERR_TIMEOUT or
+ * PQK_ERR_BAD_SEQLENS (the first condition recorded since the last read),
+ * or PQK_ERR_CUDA if the synchronisation itself failed.
+ */
+PQK_API int pqk_get_device_status(void* stream);
+
+/*
+ * pqk_set_wait_timeout_ns -- upper bound, in nanoseconds, on every wait of
+ * the attention pipeline (default 1e9). A wait that runs out records
+ * PQK_ERR_TIMEOUT, its thread block stops issuing work, waits (again
+ * bounded) for its copies in flight, frees its tensor memory and exits.
+ * Values <= 0 restore the default. Affects calls enqueued afterwards.
+ */
+PQK_API void pqk_set_wait_timeout_ns(int64_t ns);
+
+/*
+ * pqk_selftest_wait_timeout -- diagnostic: enqueues one thread block that
+ * waits, with the bounded wait used by the attention pipeline, on a
+ * barrier that nothing completes. The wait runs out after timeout_ns and
+ * records PQK_ERR_TIMEOUT in the status word; the context stays usable.
+ */
+PQK_API int pqk_selftest_wait_timeout(int64_t timeout_ns, void* stream);
+
+/* Human-readable name of a pqk_status value. */
+PQK_API const char* pqk_status_string(int status);
+
+/* Library version, "major.minor.patch". */
+PQK_API const char* pqk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PQK_H */

@@ -1,0 +1,42 @@
+// pqk_internal.h -- launchers shared between the C-ABI front end
+// (pqk_api.cu) and the kernel translation units. Arguments are validated by
+// the front end before any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace pqk {
+
+int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride,
+                        int64_t k_stride, const void* wq, const void* wk, const int32_t* pos, int64_t T, int H,
+                        int D, float eps, float rope_base, int style, cudaStream_t stream, int num_sms);
+
+int launch_modulate_swiglu(const void* x, const void* branch, void* x_out, void* h, const float* shift,
+                           const float* scale, const float* gate_res, const int32_t* cu_seqlens, int B, int64_t T,
+                           int C, int norm_type, float eps, const void* gate, const void* up, int64_t gu_stride,
+                           void* act, int F, cudaStream_t stream, int num_sms);
+
+// Bytes of the attention tile schedule for B requests.
+size_t attn_schedule_bytes(int B);
+
+// Prepares and enqueues the attention kernel's TMA descriptors, the schedule
+// builder and the persistent attention kernel. Returns 0, or -1 when a CUDA
+// call failed, -2 when the tensor maps could not be encoded.
+int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, float* lse, int64_t q_stride,
+                       int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
+                       int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
+                       long long timeout_ns, cudaStream_t stream, int num_sms);
+
+int launch_wait_selftest(int* status, long long timeout_ns, cudaStream_t stream);
+
+// Status codes written by kernels into the device status word (same values
+// as the public pqk_status).
+constexpr int kStatusTimeout = -6;
+constexpr int kStatusBadSeqlens = -7;
+
+}  // namespace pqk

@@ -1,0 +1,196 @@
+// qk_norm_rope.cu -- fused Q/K RMSNorm + RoPE ("Q/K normalisation merged
+// with RoPE": "FastH3 在八卡 B300 上实现完整 MP4 生成快于播放时长", section
+// "融合 DiT 算子"; "MiniMax H3 FastH3 real-time serving with vLLM-Omni",
+// bullet "Fused DiT operators").
+//
+// HBM-bound: every bf16 element is read once and written once. One warp owns
+// one token at a time and walks its 2*H rows (Q heads, then K heads); each
+// row of D elements is split over D/8 lanes holding 8 elements (16 bytes)
+// apiece, so a warp step moves 2 (D=128) or 4 (D=64) full rows with fully
+// coalesced 16-byte accesses. The RMS reduction is a shuffle butterfly over
+// the row's lanes. A lane's RoPE angles only depend on the token and on its
+// fixed column slice, so cos/sin are formed once per token and reused for
+// all 2*H rows; the angle pos * base^(-2j/D) is formed and reduced modulo
+// 2*pi in fp64 (positions reach ~1.9e5, where an fp32 angle is off by
+// ~1e-2 rad) and only the reduced angle goes through the fp32 sine/cosine.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "pqk_internal.h"
+
+namespace pqk {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;  // warp steps whose loads are in flight together
+
+struct QkParams {
+  const __nv_bfloat16* q_in;
+  const __nv_bfloat16* k_in;
+  __nv_bfloat16* q_out;
+  __nv_bfloat16* k_out;
+  int64_t q_stride;
+  int64_t k_stride;
+  const __nv_bfloat16* wq;
+  const __nv_bfloat16* wk;
+  const int32_t* pos;
+  int64_t T;
+  int H;
+  float eps;
+  double log2_base;
+  int style;
+};
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  uint4 v;
+  v.x = pack_bf16x2(f[0], f[1]);
+  v.y = pack_bf16x2(f[2], f[3]);
+  v.z = pack_bf16x2(f[4], f[5]);
+  v.w = pack_bf16x2(f[6], f[7]);
+  return v;
+}
+
+// Angle phi = pos * theta reduced to [-pi, pi] in fp64, then the SFU sin/cos
+// in fp32 (accurate on that range).
+__device__ __forceinline__ void rope_sincos(int32_t pos, double theta, float& c, float& s) {
+  const double kTwoPi = 6.283185307179586476925286766559;
+  const double phi = static_cast<double>(pos) * theta;
+  const double k = rint(phi * (1.0 / kTwoPi));
+  const float r = static_cast<float>(fma(-k, kTwoPi, phi));
+  __sincosf(r, &s, &c);  // |r| <= pi: absolute error ~4e-7
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParams p) {
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerStep = 32 / kLanesPerRow;
+  constexpr int kHalfLanes = kLanesPerRow / 2;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanesPerRow;  // row within a warp step
+  const int chunk = lane % kLanesPerRow;  // 8-element column slice of the row
+  const bool interleaved = p.style == 0;
+
+  // theta_j = base^(-2j/D) for the D/2 pair indices, shared by the block.
+  // Interleaved: a lane's slice holds pairs j = 4*chunk .. 4*chunk+3. Half:
+  // it holds first-half elements j = 8*(chunk mod D/16) .. +7 or their
+  // second-half partners.
+  __shared__ double theta[D / 2];
+  for (int j = threadIdx.x; j < D / 2; j += kThreads)
+    theta[j] = exp2(-2.0 * static_cast<double>(j) / static_cast<double>(D) * p.log2_base);
+  __syncthreads();
+  const int j0 = interleaved ? 4 * chunk : 8 * (chunk % kHalfLanes);
+  const uint4 wq_raw = *reinterpret_cast<const uint4*>(p.wq + chunk * 8);
+  const uint4 wk_raw = *reinterpret_cast<const uint4*>(p.wk + chunk * 8);
+  const int rows = 2 * p.H;
+  const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + threadIdx.x / 32; t < p.T;
+       t += warps_total) {
+    const int32_t pos = p.pos[t];
+    float cs[8], sn[8];
+    if (interleaved) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) rope_sincos(pos, theta[j0 + i], cs[i], sn[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) rope_sincos(pos, theta[j0 + i], cs[i], sn[i]);
+    }
+    for (int r0 = 0; r0 < rows; r0 += kRowsPerStep * kUnroll) {
+      uint4 raw[kUnroll];
+      bool live[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int r = r0 + u * kRowsPerStep + sub;
+        live[u] = r < rows;
+        raw[u] = make_uint4(0, 0, 0, 0);
+        if (live[u]) {
+          const bool is_q = r < p.H;
+          const int h = is_q ? r : r - p.H;
+          const __nv_bfloat16* src = is_q ? p.q_in + t * p.q_stride : p.k_in + t * p.k_stride;
+          raw[u] = *reinterpret_cast<const uint4*>(src + h * D + chunk * 8);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int r = r0 + u * kRowsPerStep + sub;
+        const bool is_q = r < p.H;
+        float x[8];
+        unpack8(raw[u], x);
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+        for (int off = kHalfLanes; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float inv = rsqrtf(ss * (1.0f / D) + p.eps);
+        float wv[8], y[8];
+        unpack8(is_q ? wq_raw : wk_raw, wv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = x[i] * inv * wv[i];
+        float o[8];
+        if (interleaved) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float a = y[2 * i], b = y[2 * i + 1];
+            o[2 * i] = a * cs[i] - b * sn[i];
+            o[2 * i + 1] = a * sn[i] + b * cs[i];
+          }
+        } else {
+          const bool first_half = chunk < kHalfLanes;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float partner = __shfl_xor_sync(0xffffffffu, y[i], kHalfLanes);
+            o[i] = first_half ? (y[i] * cs[i] - partner * sn[i]) : (partner * sn[i] + y[i] * cs[i]);
+          }
+        }
+        if (live[u]) {
+          const int h = is_q ? r : r - p.H;
+          __nv_bfloat16* dst = is_q ? p.q_out + t * p.q_stride : p.k_out + t * p.k_stride;
+          *reinterpret_cast<uint4*>(dst + h * D + chunk * 8) = pack8(o);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride,
+                        int64_t k_stride, const void* wq, const void* wk, const int32_t* pos, int64_t T, int H,
+                        int D, float eps, float rope_base, int style, cudaStream_t stream, int num_sms) {
+  QkParams p;
+  p.q_in = static_cast<const __nv_bfloat16*>(q_in);
+  p.k_in = static_cast<const __nv_bfloat16*>(k_in);
+  p.q_out = static_cast<__nv_bfloat16*>(q_out);
+  p.k_out = static_cast<__nv_bfloat16*>(k_out);
+  p.q_stride = q_stride;
+  p.k_stride = k_stride;
+  p.wq = static_cast<const __nv_bfloat16*>(wq);
+  p.wk = static_cast<const __nv_bfloat16*>(wk);
+  p.pos = pos;
+  p.T = T;
+  p.H = H;
+  p.eps = eps;
+  p.log2_base = log2(static_cast<double>(rope_base));
+  p.style = style;
+  const int64_t warps_per_block = kThreads / 32;
+  const int64_t want = (T + warps_per_block - 1) / warps_per_block;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 3;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  if (D == 128)
+    qk_norm_rope_kernel<128><<<grid, kThreads, 0, stream>>>(p);
+  else
+    qk_norm_rope_kernel<64><<<grid, kThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace pqk

@@ -1,0 +1,623 @@
+// varlen_attn_fwd.cu -- packed variable-length bf16 self-attention on the
+// fifth-generation tensor cores (tcgen05 + tensor memory + TMA).
+//
+// The operation: every request's tokens attend to all tokens of the same
+// request and to nothing else; requests are packed back to back without
+// padding and only valid tokens are processed ("FastH3 在八卡 B300 上实现完整
+// MP4 生成快于播放时长", section "长序列注意力与通信优化"; "MiniMax H3 FastH3
+// real-time serving with vLLM-Omni", bullet "Long-sequence attention &
+// communication").
+//
+// Work unit ("work tile"): (request, head, block of 256 query rows) = two
+// 128-row query tiles Q0, Q1 that share every K/V tile. A one-block
+// schedule kernel turns cu_seqlens into a tile list (requests longest
+// first, then head, then query block, so that the CTAs running at the same
+// time read the same head's K/V from L2), and a persistent kernel with one
+// CTA per SM walks that list round-robin.
+//
+// CTA roles (320 threads):
+//   warps 0-3  softmax for Q0; thread r owns query row r (tensor-memory lane r)
+//   warps 4-7  softmax for Q1
+//   warp  8    TMA producer: Q tiles, then K_j, V_j into a ring of stages
+//   warp  9    tensor-memory allocator and single-thread MMA issuer
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   [0,128) S0 = Q0 K^T (fp32), [128,256) S1; P_i (bf16 pairs) overwrites the
+//   first 64 columns of S_i once the softmax has read S_i; [256,256+D) O0,
+//   [256+D,256+2D) O1 (fp32 accumulators).
+// MMA issue order per K/V tile j: O0 += P0 V_j, S0 = Q0 K_{j+1}^T,
+// O1 += P1 V_j, S1 = Q1 K_{j+1}^T, so each softmax group works on its S
+// while the tensor core runs the other group's two products. MMAs from one
+// thread execute in issue order, which makes the S_i write after P_i's read
+// safe; every other hand-off goes through an mbarrier:
+//   kv_full/kv_empty (TMA <-> MMA, per stage), q_full/q_empty,
+//   s_full[i] (MMA -> softmax i: S_i ready, and all earlier products of
+//   this thread complete), p_full[i] (softmax i -> MMA: P_i in tensor
+//   memory, O_i rescaled), o_done[i] (MMA -> softmax i: last product of
+//   the work tile complete).
+// Online softmax in the log2 domain with lazy rescaling: the running row
+// maximum is only raised (and O, l rescaled) when the tile maximum exceeds
+// it by more than 2^8, which keeps every probability <= 256 and makes
+// rescales rare after the first tiles.
+// Every wait is bounded (pqk::mbar_wait); a wait that runs out raises the
+// block's abort flag and the device status word, and the block drains its
+// copies and MMAs in flight (bounded again), frees tensor memory and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "pqk_internal.h"
+
+namespace pqk {
+namespace {
+
+constexpr int kBM = 128;          // query rows per Q tile
+constexpr int kBN = 128;          // keys per K/V tile
+constexpr int kRowsPerWork = 2 * kBM;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 8 score columns, this many take their exponential on the FMA pipe
+// (pqk::ex2_fma) and the rest on the SFU, balancing the two units.
+constexpr int kPolyPer8 = 0;
+constexpr int kSlabBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-byte swizzle width)
+
+template <int D>
+struct Layout {
+  static constexpr int kSlabs = D / 64;
+  static constexpr int kTileBytes = kSlabs * kSlabBytes;
+  static constexpr int kStages = D == 128 ? 5 : 10;
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  // barriers: kv_full[S], kv_empty[S], q_full, q_empty, s_full[2], p_full[2], o_done[2]
+  static constexpr int kNumBars = 2 * kStages + 8;
+  static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kAbortOff = kTmemSlotOff + 4;
+  static constexpr int kBytes = kAbortOff + 4;
+  static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
+  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256, kTmemO1 = 256 + D;
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+// Schedule in the workspace (int32): [0] number of work tiles, [1] number of
+// requests B, then for the requests in schedule order r = 0..B-1:
+// tile_start[B+1] (prefix of tiles), seg_start[B], seg_len[B].
+__host__ __device__ constexpr size_t sched_words(int B) { return 2 + (B + 1) + 2 * static_cast<size_t>(B); }
+
+struct AttnParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int64_t o_stride;
+  int64_t T;
+  int H;
+  float scale_log2;
+  const int32_t* sched;
+  int* status;
+  long long timeout_ns;
+};
+
+struct Work {
+  int seg_start;
+  int seg_len;
+  int head;
+  int q0;      // first query row of the work tile
+  int n_kv;    // number of K/V tiles
+};
+
+__device__ __forceinline__ Work decode_work(const int32_t* sched, int H, int w) {
+  const int B = sched[1];
+  const int32_t* tile_start = sched + 2;
+  const int32_t* seg_start = tile_start + B + 1;
+  const int32_t* seg_len = seg_start + B;
+  int lo = 0, hi = B - 1;  // last r with tile_start[r] <= w
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= w) lo = mid; else hi = mid - 1;
+  }
+  Work wk;
+  wk.seg_start = seg_start[lo];
+  wk.seg_len = seg_len[lo];
+  const int nqb = (wk.seg_len + kRowsPerWork - 1) / kRowsPerWork;
+  const int local = w - tile_start[lo];
+  wk.head = local / nqb;
+  wk.q0 = wk.seg_start + (local % nqb) * kRowsPerWork;
+  wk.n_kv = (wk.seg_len + kBN - 1) / kBN;
+  (void)H;
+  return wk;
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
+  *abort_flag = 1;
+  atomicCAS(status, 0, kStatusTimeout);
+}
+
+// ------------------------------------------------------------ schedule
+
+constexpr int kSchedThreads = 1024;
+constexpr int kSortLimit = 8192;  // requests ordered longest first up to this B
+
+__global__ void __launch_bounds__(kSchedThreads) build_schedule_kernel(const int32_t* cu, int B, int64_t T, int H,
+                                                                        int32_t* sched, int* status) {
+  __shared__ int bad;
+  __shared__ int32_t carry;
+  if (threadIdx.x == 0) {
+    bad = (cu[0] != 0 || static_cast<int64_t>(cu[B]) != T) ? 1 : 0;
+    carry = 0;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < B; i += kSchedThreads)
+    if (cu[i + 1] < cu[i]) bad = 1;
+  __syncthreads();
+  int32_t* tile_start = sched + 2;
+  int32_t* seg_start = tile_start + B + 1;
+  int32_t* seg_len = seg_start + B;
+  if (bad) {
+    if (threadIdx.x == 0) {
+      sched[0] = 0;
+      sched[1] = B;
+      atomicCAS(status, 0, kStatusBadSeqlens);
+    }
+    return;
+  }
+  // rank of request i: longer first, ties by index (identity order above kSortLimit)
+  for (int i = threadIdx.x; i < B; i += kSchedThreads) {
+    const int Li = cu[i + 1] - cu[i];
+    int rank = i;
+    if (B <= kSortLimit) {
+      rank = 0;
+      for (int j = 0; j < B; ++j) {
+        const int Lj = cu[j + 1] - cu[j];
+        rank += (Lj > Li) || (Lj == Li && j < i);
+      }
+    }
+    seg_start[rank] = cu[i];
+    seg_len[rank] = Li;
+  }
+  __syncthreads();
+  // exclusive prefix of tiles per request in schedule order, one chunk of
+  // kSchedThreads requests at a time (warp scans, then a scan of warp sums)
+  __shared__ int32_t warp_sums[kSchedThreads / 32];
+  for (int base = 0; base < B; base += kSchedThreads) {
+    const int i = base + threadIdx.x;
+    const int32_t n = i < B ? ((seg_len[i] + kRowsPerWork - 1) / kRowsPerWork) * H : 0;
+    int32_t incl = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+      if ((threadIdx.x & 31) >= off) incl += y;
+    }
+    if ((threadIdx.x & 31) == 31) warp_sums[threadIdx.x >> 5] = incl;
+    __syncthreads();
+    int32_t before = carry;
+    for (int w = 0; w < static_cast<int>(threadIdx.x >> 5); ++w) before += warp_sums[w];
+    if (i < B) tile_start[i] = before + incl - n;
+    __syncthreads();
+    if (threadIdx.x == kSchedThreads - 1) carry = before + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    tile_start[B] = carry;
+    sched[0] = carry;
+    sched[1] = B;
+  }
+}
+
+// ------------------------------------------------------------ attention
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t q_smem = base + L::kQOff;
+  const uint32_t kv_smem = base + L::kKVOff;
+  const uint32_t bar0 = base + L::kBarOff;
+  auto kv_full = [&](int s) { return bar0 + 8u * s; };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (L::kStages + s); };
+  const uint32_t q_full = bar0 + 8u * (2 * L::kStages);
+  const uint32_t q_empty = q_full + 8;
+  auto s_full = [&](int i) { return q_full + 16 + 8u * i; };
+  auto p_full = [&](int i) { return q_full + 32 + 8u * i; };
+  auto o_done = [&](int i) { return q_full + 48 + 8u * i; };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full(i), 1);
+      mbar_init(p_full(i), kBM);
+      mbar_init(o_done(i), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(base + L::kTmemSlotOff, 512);
+    tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    prefetch_tensor_map(&tm_q);
+    prefetch_tensor_map(&tm_k);
+    prefetch_tensor_map(&tm_v);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int n_work = p.sched[0];
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t load_idx = 0;
+      uint32_t q_loads = 0;
+      int wt = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
+        const Work wk = decode_work(p.sched, p.H, w);
+        if (wt > 0 && !(ok = mbar_wait(q_empty, (wt - 1) & 1, abort_flag, p.timeout_ns))) break;
+        mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+        ++q_loads;
+        for (int i = 0; i < 2; ++i)
+          for (int sl = 0; sl < L::kSlabs; ++sl)
+            tma_load_3d(q_smem + i * L::kTileBytes + sl * kSlabBytes, &tm_q, q_full, sl * 64, wk.head,
+                        wk.q0 + i * kBM);
+        for (int j = 0; j < wk.n_kv && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const int s = load_idx % L::kStages;
+            const uint32_t round = load_idx / L::kStages;
+            if (round > 0 && !(ok = mbar_wait(kv_empty(s), (round - 1) & 1, abort_flag, p.timeout_ns))) break;
+            mbar_arrive_expect_tx(kv_full(s), L::kTileBytes);
+            const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
+            for (int sl = 0; sl < L::kSlabs; ++sl)
+              tma_load_3d(kv_smem + s * L::kTileBytes + sl * kSlabBytes, tm, kv_full(s), sl * 64, wk.head,
+                          wk.seg_start + j * kBN);
+            ++load_idx;
+          }
+        }
+      }
+      if (!ok) {
+        raise_abort(abort_flag, p.status);
+        // drain: the last kStages loads and the last Q load may still be in flight
+        const uint32_t first = load_idx > static_cast<uint32_t>(L::kStages) ? load_idx - L::kStages : 0;
+        for (uint32_t idx = first; idx < load_idx; ++idx) {
+          const volatile int no_abort = 0;
+          mbar_wait(kv_full(idx % L::kStages), (idx / L::kStages) & 1, &no_abort, p.timeout_ns);
+        }
+        if (q_loads > 0) {
+          const volatile int no_abort = 0;
+          mbar_wait(q_full, (q_loads - 1) & 1, &no_abort, p.timeout_ns);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
+      uint32_t cons_idx = 0;
+      uint32_t p_phase = 0;
+      int wt = 0;
+      bool ok = true;
+      // S_i = Q_i K^T over D/16 K-steps of 16 (32 bytes inside the 128-byte row)
+      auto issue_qk = [&](int i, int stage) {
+        const uint32_t qa = q_smem + i * L::kTileBytes;
+        const uint32_t kb = kv_smem + stage * L::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k / 4) * kSlabBytes + (k % 4) * 32;
+          mma_bf16_ss(tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1), smem_desc_sw128(qa + off, 16, 1024),
+                      smem_desc_sw128(kb + off, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+        }
+      };
+      // O_i (+)= P_i V over kBN/16 K-steps; V is MN-major: 64-wide column
+      // slabs kSlabBytes apart, 8-row groups 1024 bytes apart
+      auto issue_pv = [&](int i, int stage, bool accumulate) {
+        const uint32_t vb = kv_smem + stage * L::kTileBytes;
+        const uint32_t p_col = tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1);
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k) {
+          mma_bf16_ts(tmem + (i == 0 ? L::kTmemO0 : L::kTmemO1), p_col + 8 * k,
+                      smem_desc_sw128(vb + k * 2048, kSlabBytes, 1024), kIdescPV,
+                      (accumulate || k > 0) ? 1u : 0u);
+        }
+      };
+      auto wait_stage = [&](uint32_t idx) {
+        return mbar_wait(kv_full(idx % L::kStages), (idx / L::kStages) & 1, abort_flag, p.timeout_ns);
+      };
+      for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
+        const Work wk = decode_work(p.sched, p.H, w);
+        if (!(ok = mbar_wait(q_full, wt & 1, abort_flag, p.timeout_ns))) break;
+        uint32_t k_stage_idx = cons_idx;
+        if (!(ok = wait_stage(k_stage_idx))) break;
+        tc_fence_after_sync();
+        issue_qk(0, k_stage_idx % L::kStages);
+        tc_commit(s_full(0));
+        issue_qk(1, k_stage_idx % L::kStages);
+        tc_commit(s_full(1));
+        tc_commit(kv_empty(k_stage_idx % L::kStages));
+        if (wk.n_kv == 1) tc_commit(q_empty);
+        ++cons_idx;
+        for (int j = 0; j < wk.n_kv; ++j) {
+          const uint32_t v_idx = cons_idx++;
+          const bool more = j + 1 < wk.n_kv;
+          if (!(ok = wait_stage(v_idx))) break;
+          if (!(ok = mbar_wait(p_full(0), p_phase, abort_flag, p.timeout_ns))) break;
+          tc_fence_after_sync();
+          issue_pv(0, v_idx % L::kStages, j > 0);
+          if (!more) tc_commit(o_done(0));
+          uint32_t nk_idx = 0;
+          if (more) {
+            nk_idx = cons_idx++;
+            if (!(ok = wait_stage(nk_idx))) break;
+            tc_fence_after_sync();
+            issue_qk(0, nk_idx % L::kStages);
+            tc_commit(s_full(0));
+          }
+          if (!(ok = mbar_wait(p_full(1), p_phase, abort_flag, p.timeout_ns))) break;
+          tc_fence_after_sync();
+          issue_pv(1, v_idx % L::kStages, j > 0);
+          if (!more) tc_commit(o_done(1));
+          tc_commit(kv_empty(v_idx % L::kStages));
+          if (more) {
+            issue_qk(1, nk_idx % L::kStages);
+            tc_commit(s_full(1));
+            tc_commit(kv_empty(nk_idx % L::kStages));
+            if (j + 2 == wk.n_kv) tc_commit(q_empty);
+          }
+          p_phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        raise_abort(abort_flag, p.status);
+        // every MMA issued by this thread must complete before the tensor
+        // memory is released: a fresh commit on o_done(0) completes its next
+        // phase (phase wt, or wt + 1 if this tile's commit was already made)
+        // once all of them are done
+        const volatile int no_abort = 0;
+        tc_commit(o_done(0));
+        mbar_wait(o_done(0), wt & 1, &no_abort, p.timeout_ns);
+        mbar_wait(o_done(0), (wt + 1) & 1, &no_abort, p.timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------ softmax groups
+    const int grp = warp >> 2;  // 0 -> Q0, 1 -> Q1
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + (grp == 0 ? L::kTmemS0 : L::kTmemS1);
+    const uint32_t t_o = tmem + lane_off + (grp == 0 ? L::kTmemO0 : L::kTmemO1);
+    uint32_t s_phase = 0;
+    int wt = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
+      const Work wk = decode_work(p.sched, p.H, w);
+      const int row = wk.q0 + grp * kBM + r;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < wk.n_kv; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full(grp), s_phase, abort_flag, p.timeout_ns));
+        if (!ok) break;
+        s_phase ^= 1u;
+        tc_fence_after_sync();
+        uint32_t sr[128];
+        tmem_ld_x128(t_s, sr);
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+        if (j == wk.n_kv - 1) {
+          const int valid = wk.seg_len - j * kBN;
+          if (valid < kBN) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c >= valid) s[c] = -INFINITY;
+          }
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+        if (j == 0) {
+          m = mx;
+        } else if (mx > m + kRescaleThreshold) {
+          // O_i holds the products of tiles 0..j-1, all complete (s_full
+          // for tile j completed after them); rescale it before P_j V_j
+          const float alpha = ex2_approx(m - mx);
+          l *= alpha;
+          m = mx;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld_x32(t_o + c0, ov);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+            tmem_st_x32(t_o + c0, ov);
+          }
+        }
+        const float neg_m = -m;
+        float l0 = 0.f, l1 = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float x0 = fmaf(s[c], p.scale_log2, neg_m);
+          const float x1 = fmaf(s[c + 1], p.scale_log2, neg_m);
+          const bool poly = (c & 7) >= 8 - kPolyPer8;
+          const float p0 = poly ? ex2_fma(x0) : ex2_approx(x0);
+          const float p1 = poly ? ex2_fma(x1) : ex2_approx(x1);
+          l0 += p0;
+          l1 += p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+        l += l0 + l1;
+        tmem_st_x64(t_s, pk);
+        tc_fence_before_sync();
+        mbar_arrive(p_full(grp));
+      }
+      if (!ok) break;
+      // epilogue: normalise O_i and write the valid rows
+      ok = __all_sync(0xffffffffu, mbar_wait(o_done(grp), wt & 1, abort_flag, p.timeout_ns));
+      if (!ok) break;
+      tc_fence_after_sync();
+      const float inv_l = 1.0f / l;
+      const bool valid_row = row < wk.seg_start + wk.seg_len;
+      __nv_bfloat16* dst = p.o + static_cast<int64_t>(row) * p.o_stride + wk.head * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t ov[32];
+        tmem_ld_x32(t_o + c0, ov);
+        if (valid_row) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(ov[c]) * inv_l, __uint_as_float(ov[c + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(ov[c + 2]) * inv_l, __uint_as_float(ov[c + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(ov[c + 4]) * inv_l, __uint_as_float(ov[c + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(ov[c + 6]) * inv_l, __uint_as_float(ov[c + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(dst + c0 + c) = v;
+          }
+        }
+      }
+      if (valid_row && p.lse != nullptr)
+        p.lse[static_cast<int64_t>(wk.head) * p.T + row] = (m + __log2f(l)) * 0.69314718055994530942f;
+      tc_fence_before_sync();
+    }
+    if (!ok) raise_abort(abort_flag, p.status);
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------ self-test
+
+__global__ void wait_selftest_kernel(int* status, long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives on `bar`: the bounded wait must give up
+    if (!mbar_wait(b, 0, &abort_flag, timeout_ns)) atomicCAS(status, 0, kStatusTimeout);
+  }
+}
+
+// ------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [T, H, D] bf16 with `stride` elements between tokens, read as boxes of
+// 64 columns x 1 head x 128 tokens, 128-byte swizzled; rows past T read as 0.
+bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t T, int H, int D, int64_t stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(stride) * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kBM)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+bool set_smem_attr() {
+  static int done[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<D>::kAlloc) !=
+        cudaSuccess)
+      return false;
+    done[dev] = 1;
+  }
+  return true;
+}
+
+}  // namespace
+
+size_t attn_schedule_bytes(int B) { return ((sched_words(B) * sizeof(int32_t)) + 255) & ~static_cast<size_t>(255); }
+
+int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, float* lse, int64_t q_stride,
+                       int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
+                       int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
+                       long long timeout_ns, cudaStream_t stream, int num_sms) {
+  CUtensorMap tq, tk, tv;
+  if (!make_qkv_map(&tq, q, T, H, D, q_stride) || !make_qkv_map(&tk, k, T, H, D, k_stride) ||
+      !make_qkv_map(&tv, v, T, H, D, v_stride))
+    return -2;
+  int32_t* sched = static_cast<int32_t*>(workspace);
+  build_schedule_kernel<<<1, kSchedThreads, 0, stream>>>(cu_seqlens, B, T, H, sched, status);
+  if (cudaGetLastError() != cudaSuccess) return -1;
+  AttnParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.o_stride = o_stride;
+  p.T = T;
+  p.H = H;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.sched = sched;
+  p.status = status;
+  p.timeout_ns = timeout_ns;
+  // upper bound of work tiles: every request adds at most one partial block
+  const int64_t max_work = static_cast<int64_t>(H) * ((T + kRowsPerWork - 1) / kRowsPerWork + B);
+  const int grid = static_cast<int>(max_work < num_sms ? max_work : num_sms);
+  if (D == 128) {
+    if (!set_smem_attr<128>()) return -1;
+    attn_fwd_kernel<128><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+  } else {
+    if (!set_smem_attr<64>()) return -1;
+    attn_fwd_kernel<64><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_wait_selftest(int* status, long long timeout_ns, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(status, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace pqk

@@ -1,0 +1,182 @@
+"""Thin Python binding of libpqk's C ABI (include/pqk.h).
+
+Argument marshalling only: every step of the hot path runs in the CUDA
+kernels behind the C ABI. PyTorch supplies device memory (``data_ptr``) and
+the current CUDA stream. There is no fallback: if ``libpqk.so`` has not been
+built, loading fails with an error.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libpqk.so")
+
+PQK_OK = 0
+STATUS = {0: "PQK_OK", -1: "PQK_ERR_INVALID_ARG", -2: "PQK_ERR_UNSUPPORTED", -3: "PQK_ERR_MISALIGNED",
+          -4: "PQK_ERR_CUDA", -5: "PQK_ERR_WORKSPACE", -6: "PQK_ERR_TIMEOUT", -7: "PQK_ERR_BAD_SEQLENS"}
+ROPE_INTERLEAVED, ROPE_HALF = 0, 1
+NORM_RMS, NORM_LAYER, NORM_NONE = 0, 1, 2
+
+# every symbol include/pqk.h declares
+EXPORTS = ("pqk_qk_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd", "pqk_modulate_swiglu",
+           "pqk_get_device_status", "pqk_set_wait_timeout_ns", "pqk_selftest_wait_timeout", "pqk_status_string",
+           "pqk_version")
+
+
+class PqkError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {code} ({STATUS.get(code, 'unknown')}: {status_string(code)})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib(path: str | None = None) -> C.CDLL:
+    """Load libpqk.so (built by packed_attention_qk_b200.build) and declare
+    its signatures."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"libpqk.so not found at {p}: build it with `python -m packed_attention_qk_b200.build`")
+    L = C.CDLL(p)
+    vp, i64, i32, f32, sz = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
+    L.pqk_qk_norm_rope.argtypes = [vp, vp, vp, vp, i64, i64, vp, vp, vp, i64, i32, i32, f32, f32, i32, vp]
+    L.pqk_qk_norm_rope.restype = i32
+    L.pqk_varlen_attn_workspace_size.argtypes = [i32]
+    L.pqk_varlen_attn_workspace_size.restype = sz
+    L.pqk_varlen_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32, vp, sz,
+                                      vp]
+    L.pqk_varlen_attn_fwd.restype = i32
+    L.pqk_modulate_swiglu.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, f32, vp, vp, i64, vp,
+                                      i32, vp]
+    L.pqk_modulate_swiglu.restype = i32
+    L.pqk_get_device_status.argtypes = [vp]
+    L.pqk_get_device_status.restype = i32
+    L.pqk_set_wait_timeout_ns.argtypes = [i64]
+    L.pqk_set_wait_timeout_ns.restype = None
+    L.pqk_selftest_wait_timeout.argtypes = [i64, vp]
+    L.pqk_selftest_wait_timeout.restype = i32
+    L.pqk_status_string.argtypes = [i32]
+    L.pqk_status_string.restype = C.c_char_p
+    L.pqk_version.argtypes = []
+    L.pqk_version.restype = C.c_char_p
+    if path is None:
+        _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().pqk_status_string(code).decode()
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != PQK_OK:
+        raise PqkError(fn, rc)
+
+
+def _stream(stream) -> int | None:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _token_stride(t, ndim: int) -> int:
+    assert t.dim() == ndim, f"expected a {ndim}-d tensor, got {tuple(t.shape)}"
+    for d in range(1, ndim):
+        want = 1
+        for e in range(d + 1, ndim):
+            want *= t.shape[e]
+        assert t.stride(d) == want, "only the token (first) dimension may be strided"
+    return t.stride(0)
+
+
+# ---------------------------------------------------------------- calls
+
+def qk_norm_rope(q, k, w_q, w_k, pos, *, eps: float = 1e-6, rope_base: float = 10000.0,
+                 style: int = ROPE_INTERLEAVED, q_out=None, k_out=None, stream=None):
+    """Fused Q/K RMSNorm + RoPE. q, k: bf16 [T, H, D] (token dim may be
+    strided); outputs default to in place."""
+    q_out = q if q_out is None else q_out
+    k_out = k if k_out is None else k_out
+    T, H, D = q.shape
+    qs, ks = _token_stride(q, 3), _token_stride(k, 3)
+    assert _token_stride(q_out, 3) == qs and _token_stride(k_out, 3) == ks
+    _check("pqk_qk_norm_rope", lib().pqk_qk_norm_rope(
+        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), qs, ks, _ptr(w_q), _ptr(w_k), _ptr(pos), T, H, D, eps,
+        rope_base, style, _stream(stream)))
+    return q_out, k_out
+
+
+def varlen_attn_workspace_size(B: int) -> int:
+    return int(lib().pqk_varlen_attn_workspace_size(B))
+
+
+def varlen_attn_fwd(q, k, v, cu_seqlens, *, softmax_scale: float | None = None, o=None, lse=None,
+                    workspace=None, want_lse: bool = False, stream=None):
+    """Packed varlen attention. q, k, v: bf16 [T, H, D]; cu_seqlens: int32
+    [B+1] on the device. Returns (o, lse or None)."""
+    import torch
+    T, H, D = q.shape
+    B = cu_seqlens.shape[0] - 1
+    scale = softmax_scale if softmax_scale is not None else D ** -0.5
+    if o is None:
+        o = torch.empty((T, H, D), dtype=q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((H, T), dtype=torch.float32, device=q.device)
+    ws_bytes = varlen_attn_workspace_size(B)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check("pqk_varlen_attn_fwd", lib().pqk_varlen_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _token_stride(q, 3), _token_stride(k, 3),
+        _token_stride(v, 3), _token_stride(o, 3), _ptr(cu_seqlens), B, T, H, D, scale, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+def modulate_swiglu(x, shift, scale, cu_seqlens, *, gate_res=None, branch=None, gate=None, up=None,
+                    norm_type: int = NORM_RMS, eps: float = 1e-6, x_out=None, h=None, act=None, stream=None):
+    """Fused gated residual + norm + adaLN modulation, and SwiGLU.
+    Returns (x_out or None, h, act or None)."""
+    import torch
+    T, Cdim = x.shape
+    B = cu_seqlens.shape[0] - 1
+    if h is None:
+        h = torch.empty_like(x)
+    F, gu_stride = 0, 0
+    if gate is not None:
+        F = gate.shape[1]
+        gu_stride = _token_stride(gate, 2)
+        assert _token_stride(up, 2) == gu_stride
+        if act is None:
+            act = torch.empty((T, F), dtype=x.dtype, device=x.device)
+    _check("pqk_modulate_swiglu", lib().pqk_modulate_swiglu(
+        _ptr(x), _ptr(branch), _ptr(x_out), _ptr(h), _ptr(shift), _ptr(scale), _ptr(gate_res), _ptr(cu_seqlens),
+        B, T, Cdim, norm_type, eps, _ptr(gate), _ptr(up), gu_stride, _ptr(act), F, _stream(stream)))
+    return x_out, h, act
+
+
+def get_device_status(stream=None) -> int:
+    return int(lib().pqk_get_device_status(_stream(stream)))
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    lib().pqk_set_wait_timeout_ns(int(ns))
+
+
+def selftest_wait_timeout(timeout_ns: int, stream=None) -> None:
+    _check("pqk_selftest_wait_timeout", lib().pqk_selftest_wait_timeout(int(timeout_ns), _stream(stream)))
+
+
+def version() -> str:
+    return lib().pqk_version().decode()

@@ -64,24 +64,35 @@ def _chunk_rng(seed: int, name: str, chunk: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, TENSOR_ID[name], chunk])))
 
 
-def _draw(seed: int, name: str, n: int, kind: str, threads: int | None = None) -> np.ndarray:
-    """Draw ``n`` float32 values of distribution ``kind`` in chunks."""
-    out = np.empty(n, dtype=np.float32)
+def _chunk_values(seed: int, name: str, c: int, m: int, kind: str) -> np.ndarray:
+    g = _chunk_rng(seed, name, c)
+    if kind == "normal":
+        return g.standard_normal(m, dtype=np.float32)
+    if kind == "normal01":
+        return g.standard_normal(m, dtype=np.float32) * np.float32(0.1)
+    if kind == "uniform_w":
+        return g.uniform(0.5, 1.5, m).astype(np.float32)
+    if kind == "bernoulli":
+        return (g.random(m, dtype=np.float32) < np.float32(0.001)).astype(np.float32)
+    raise ValueError(kind)
+
+
+def _draw(seed: int, name: str, n: int, kind: str, threads: int | None = None, to_bf16: bool = False,
+          outlier_name: str | None = None) -> np.ndarray:
+    """Draw ``n`` values of distribution ``kind`` chunk by chunk: float32, or
+    bf16 bits rounded per chunk (``to_bf16``) so that no full-size float32
+    temporary exists. With ``outlier_name``, elements whose Bernoulli(0.001)
+    mask (stream ``outlier_name``) is set are multiplied by 20 first."""
+    out = np.empty(n, dtype=np.uint16 if to_bf16 else np.float32)
     nchunks = (n + CHUNK - 1) // CHUNK
 
     def fill(c: int) -> None:
         lo, hi = c * CHUNK, min(n, (c + 1) * CHUNK)
-        g = _chunk_rng(seed, name, c)
-        if kind == "normal":
-            out[lo:hi] = g.standard_normal(hi - lo, dtype=np.float32)
-        elif kind == "normal01":
-            out[lo:hi] = g.standard_normal(hi - lo, dtype=np.float32) * np.float32(0.1)
-        elif kind == "uniform_w":
-            out[lo:hi] = g.uniform(0.5, 1.5, hi - lo).astype(np.float32)
-        elif kind == "bernoulli":
-            out[lo:hi] = (g.random(hi - lo, dtype=np.float32) < np.float32(0.001)).astype(np.float32)
-        else:
-            raise ValueError(kind)
+        vals = _chunk_values(seed, name, c, hi - lo, kind)
+        if outlier_name is not None:
+            m = _chunk_values(seed, outlier_name, c, hi - lo, "bernoulli")
+            vals = np.where(m > 0, vals * np.float32(20.0), vals)
+        out[lo:hi] = f32_to_bf16_bits(vals) if to_bf16 else vals
 
     if nchunks <= 1:
         if nchunks:
@@ -95,7 +106,7 @@ def _draw(seed: int, name: str, n: int, kind: str, threads: int | None = None) -
 
 def bf16_normal(seed: int, name: str, shape: tuple[int, ...]) -> np.ndarray:
     n = int(np.prod(shape))
-    return f32_to_bf16_bits(_draw(seed, name, n, "normal")).reshape(shape)
+    return _draw(seed, name, n, "normal", to_bf16=True).reshape(shape)
 
 
 def bf16_weight(seed: int, name: str, d: int) -> np.ndarray:
@@ -110,10 +121,7 @@ def f32_modulation(seed: int, name: str, shape: tuple[int, ...]) -> np.ndarray:
 def bf16_k_with_outliers(seed: int, shape: tuple[int, ...]) -> np.ndarray:
     """K for the outlier variant: 0.1% of entries multiplied by 20 before rounding."""
     n = int(np.prod(shape))
-    k = _draw(seed, "k", n, "normal")
-    m = _draw(seed, "outlier", n, "bernoulli")
-    k = np.where(m > 0, k * np.float32(20.0), k)
-    return f32_to_bf16_bits(k).reshape(shape)
+    return _draw(seed, "k", n, "normal", to_bf16=True, outlier_name="outlier").reshape(shape)
 
 
 # ----------------------------------------------------------------------------

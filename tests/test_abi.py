@@ -1,0 +1,152 @@
+"""The C-ABI library loads, exports every entry point include/pqk.h declares,
+and rejects bad arguments on the host before touching a GPU (CPU only: no
+compute call is made; every case below returns before any CUDA call)."""
+
+import os
+import re
+import subprocess
+
+import pytest
+
+from packed_attention_qk_b200 import build as pqk_build
+from packed_attention_qk_b200 import pqk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pqk.h")
+
+ERR_INVALID, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_WORKSPACE = -1, -2, -3, -5
+A = 0x10000  # a 16-byte aligned fake device address; never dereferenced on the host
+U = 0x10004  # misaligned
+
+
+@pytest.fixture(scope="module")
+def L():
+    pqk_build.build()
+    return pqk.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"PQK_API\s+[\w\s\*]+?\b(pqk_\w+)\s*\(", text)))
+
+
+def test_header_declarations_match_binding_list():
+    assert declared_functions() == sorted(pqk.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", pqk.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+    # nothing but the C ABI is exported
+    assert {n for n in exported if n.startswith("pqk_")} == set(declared_functions())
+
+
+def test_library_has_no_libcuda_or_oracle_dependency(L):
+    out = subprocess.run(["ldd", pqk.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "oracle" not in out
+
+
+def test_status_strings_and_version(L):
+    assert pqk.status_string(0) == "ok"
+    for code in range(-1, -8, -1):
+        assert pqk.status_string(code) != "unknown status"
+    assert pqk.status_string(-99) == "unknown status"
+    assert re.fullmatch(r"\d+\.\d+\.\d+", pqk.version())
+
+
+def test_workspace_size(L):
+    assert L.pqk_varlen_attn_workspace_size(0) == 0
+    a, b = L.pqk_varlen_attn_workspace_size(1), L.pqk_varlen_attn_workspace_size(4096)
+    assert a > 0 and b > a and a % 256 == 0 and b % 256 == 0
+    assert b >= 4 * (2 + 4097 + 2 * 4096)
+
+
+def qk(L, **kw):
+    a = dict(q_in=A, k_in=A, q_out=A, k_out=A, qs=1024, ks=1024, wq=A, wk=A, pos=A, T=16, H=8, D=128, eps=1e-6,
+             base=10000.0, style=0)
+    a.update(kw)
+    return L.pqk_qk_norm_rope(a["q_in"], a["k_in"], a["q_out"], a["k_out"], a["qs"], a["ks"], a["wq"], a["wk"],
+                              a["pos"], a["T"], a["H"], a["D"], a["eps"], a["base"], a["style"], None)
+
+
+def test_qk_norm_rope_host_errors(L):
+    assert qk(L, D=96) == ERR_UNSUPPORTED
+    assert qk(L, D=256) == ERR_UNSUPPORTED
+    assert qk(L, H=0) == ERR_INVALID
+    assert qk(L, T=-1) == ERR_INVALID
+    assert qk(L, eps=0.0) == ERR_INVALID
+    assert qk(L, base=-1.0) == ERR_INVALID
+    assert qk(L, style=2) == ERR_INVALID
+    assert qk(L, qs=1000) == ERR_INVALID           # < H*D
+    assert qk(L, q_in=None) == ERR_INVALID
+    assert qk(L, pos=None) == ERR_INVALID
+    assert qk(L, k_out=U) == ERR_MISALIGNED
+    assert qk(L, wq=U) == ERR_MISALIGNED
+    assert qk(L, qs=1028) == ERR_MISALIGNED        # not a multiple of 8 elements
+    assert qk(L, T=0, q_in=None) == 0              # empty: nothing to do
+
+
+def attn(L, **kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=None, qs=1024, ks=1024, vs=1024, os_=1024, cu=A, B=2, T=512, H=8, D=128,
+             scale=0.088, ws=A, wsb=4096)
+    a.update(kw)
+    return L.pqk_varlen_attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["qs"], a["ks"], a["vs"], a["os_"],
+                                 a["cu"], a["B"], a["T"], a["H"], a["D"], a["scale"], a["ws"], a["wsb"], None)
+
+
+def test_varlen_attn_host_errors(L):
+    assert attn(L, D=96) == ERR_UNSUPPORTED
+    assert attn(L, B=0) == ERR_INVALID
+    assert attn(L, H=0) == ERR_INVALID
+    assert attn(L, scale=0.0) == ERR_INVALID
+    assert attn(L, scale=float("inf")) == ERR_INVALID
+    assert attn(L, vs=512) == ERR_INVALID
+    assert attn(L, cu=None) == ERR_INVALID
+    assert attn(L, o=None) == ERR_INVALID
+    assert attn(L, v=U) == ERR_MISALIGNED
+    assert attn(L, lse=U) == ERR_MISALIGNED
+    assert attn(L, os_=1032 + 4) == ERR_MISALIGNED
+    assert attn(L, ws=None) == ERR_WORKSPACE
+    assert attn(L, wsb=8) == ERR_WORKSPACE
+    assert attn(L, ws=U) == ERR_MISALIGNED
+    assert attn(L, T=0, q=None) == 0
+
+
+def mod(L, **kw):
+    a = dict(x=A, br=None, xo=None, h=A, shift=A, scale=A, gr=None, cu=A, B=1, T=8, C=256, nt=0, eps=1e-6,
+             gate=A, up=A, gus=512, act=A, F=512)
+    a.update(kw)
+    return L.pqk_modulate_swiglu(a["x"], a["br"], a["xo"], a["h"], a["shift"], a["scale"], a["gr"], a["cu"], a["B"],
+                                 a["T"], a["C"], a["nt"], a["eps"], a["gate"], a["up"], a["gus"], a["act"], a["F"],
+                                 None)
+
+
+def test_modulate_swiglu_host_errors(L):
+    assert mod(L, C=250) == ERR_INVALID
+    assert mod(L, C=16392) == ERR_INVALID
+    assert mod(L, nt=3) == ERR_INVALID
+    assert mod(L, eps=0.0) == ERR_INVALID
+    assert mod(L, B=0) == ERR_INVALID
+    assert mod(L, br=A, gr=None) == ERR_INVALID     # branch needs its gate
+    assert mod(L, up=None) == ERR_INVALID           # gate without up
+    assert mod(L, F=500, gus=500) == ERR_INVALID
+    assert mod(L, gus=256) == ERR_INVALID           # stride < F
+    assert mod(L, act=None) == ERR_INVALID
+    assert mod(L, x=U) == ERR_MISALIGNED
+    assert mod(L, gate=U) == ERR_MISALIGNED
+    assert mod(L, gus=1028) == ERR_MISALIGNED
+    assert mod(L, T=0, x=None) == 0
+
+
+def test_selftest_rejects_bad_timeout(L):
+    assert L.pqk_selftest_wait_timeout(0, None) == ERR_INVALID
+    assert L.pqk_selftest_wait_timeout(20_000_000_000, None) == ERR_INVALID
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="libpqk.so not found"):
+        pqk.lib(str(tmp_path / "libpqk.so"))
