@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=3, help="workload number (3 = 58,048-token joint sequence)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="one request of this many tokens with the shape of --config (a smaller case for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -237,6 +239,34 @@ def run_reference(args, w):
     print(json.dumps(out), flush=True)
 
 
+class Ranks:
+    """Process-group plumbing of a multi-rank run: a barrier and the maximum
+    of a value over ranks (the device time of the slowest rank). With one
+    rank both are no-ops. The same calls in the same order on every rank."""
+
+    def __init__(self, world: int, device):
+        self.world, self.device = world, device
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, v: float) -> float:
+        if self.world == 1:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def throughput(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -250,17 +280,8 @@ def run_ours(args, w):
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(world, dev)
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     d = make_inputs(w, dev)
     o = alloc_outputs(w, d)
@@ -291,7 +312,7 @@ def run_ours(args, w):
     epi = [e[2].elapsed_time(e[3]) for e in evs]
     ms_step = total_ms / K
     flops = w.attn_flops()
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = throughput(flops, world, ms_step)
     att_ms = statistics.mean(att)
     pk, pk_kind = peaks()
     attn_tflops = flops / (att_ms * 1e-3) / 1e12
@@ -328,7 +349,7 @@ def run_ours(args, w):
         torch.cuda.synchronize()
         barrier()
         e2e_ms = max_over_ranks(s2.elapsed_time(t2)) / e2e_steps
-        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": throughput(flops, world, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
 
     cpu = None
@@ -371,6 +392,9 @@ def main():
     args = parse()
     from packed_attention_qk_b200 import workloads as wl
     w = wl.config(args.config)
+    if args.tokens:
+        w = wl.Workload(f"one request of {args.tokens} tokens, {w.H} heads x {w.D}, hidden {w.C}, ffn {w.F}", w.seed,
+                        [args.tokens], H=w.H, D=w.D, C=w.C, F=w.F, pos_runs=[[args.tokens]])
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -5,14 +5,13 @@
 // real-time serving with vLLM-Omni", bullet "Fused DiT operators":
 // modulation and normalization among the fused operators).
 //
-// HBM-bound. A 256-thread block owns one token at a time (grid-stride over
-// tokens). Part 1 keeps the token's C-wide row in registers (8 elements of
-// 16 bytes per slot, up to kMaxSlots slots per thread), forms the gated
-// residual, reduces sum / sum of squares across the block (warp shuffles,
-// then one shared-memory exchange), and writes h = norm * (1 + scale) +
-// shift with the request's modulation vectors (read through the read-only
-// cache, shared by every token of the request). Part 2 streams the token's
-// gate / up rows in 16-byte chunks, kUnroll chunks in flight per thread.
+// HBM-bound. One warp owns one token at a time (grid-stride over tokens,
+// eight warps per block, no block barriers): it streams the token's C-wide
+// row in 16-byte chunks, forms the gated residual and its sum / sum of
+// squares (shuffle reduction), reads the row again from cache to write
+// h = norm * (1 + scale) + shift with the request's modulation vectors
+// (read-only cache, shared by every token of the request), then streams
+// the token's gate / up rows, kUnroll chunks in flight per lane.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -82,107 +81,88 @@ __device__ __forceinline__ int find_segment(const int32_t* cu, int B, int64_t t)
   return lo;
 }
 
-// Block-wide sum of two values; every thread gets the result.
-__device__ __forceinline__ float2 block_sum2(float a, float b, float2* scratch) {
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-    a += __shfl_xor_sync(0xffffffffu, a, off);
-    b += __shfl_xor_sync(0xffffffffu, b, off);
-  }
-  const int warp = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) scratch[warp] = make_float2(a, b);
-  __syncthreads();
-  float2 r = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) {
-    r.x += scratch[w].x;
-    r.y += scratch[w].y;
-  }
-  __syncthreads();
-  return r;
-}
-
 __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-template <int kMaxSlots>
-__global__ void __launch_bounds__(kThreads) modulate_swiglu_kernel(const ModParams p) {
-  __shared__ float2 scratch[kThreads / 32];
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// x' chunk c of token t: x + gate_res[s] * branch (or x alone).
+__device__ __forceinline__ void residual_chunk(const ModParams& p, int64_t t, int64_t mod_row, int c, float (&xv)[8]) {
+  unpack8(*reinterpret_cast<const uint4*>(p.x + t * p.C + c * 8), xv);
+  if (p.branch != nullptr) {
+    float br[8], g[8];
+    unpack8(*reinterpret_cast<const uint4*>(p.branch + t * p.C + c * 8), br);
+    load8f(p.gate_res + mod_row + c * 8, g);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) xv[i] = fmaf(g[i], br[i], xv[i]);
+  }
+}
+
+// One warp per token (grid-stride over tokens). Pass 1 streams the token's
+// C-wide row, forms x' (written out when requested) and its sum and sum of
+// squares; a shuffle reduction gives the statistics to every lane. Pass 2
+// reads the row again (now in L1/L2), re-forms x' bit-identically and
+// writes h. Then the lanes stream the token's gate / up rows. No block
+// barriers: each warp moves at its own pace.
+__global__ void __launch_bounds__(kThreads, 3) modulate_swiglu_kernel(const ModParams p) {
+  const int lane = threadIdx.x & 31;
   const int nchunks = p.C / 8;
   const int fchunks = p.F / 8;
   const float inv_c = 1.0f / static_cast<float>(p.C);
-  for (int64_t t = blockIdx.x; t < p.T; t += gridDim.x) {
+  const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); t < p.T;
+       t += warps_total) {
     const int seg = find_segment(p.cu, p.B, t);
     const int64_t mod_row = static_cast<int64_t>(seg) * p.C;
-    // ---- part 1: gated residual, norm, modulation
-    float xv[kMaxSlots][8];
     float s1 = 0.f, s2 = 0.f;
+    for (int c = lane; c < nchunks; c += 32) {
+      float xv[8];
+      residual_chunk(p, t, mod_row, c, xv);
+      if (p.x_out != nullptr) *reinterpret_cast<uint4*>(p.x_out + t * p.C + c * 8) = pack8(xv);
 #pragma unroll
-    for (int k = 0; k < kMaxSlots; ++k) {
-      const int c = threadIdx.x + k * kThreads;
-      if (c < nchunks) {
-        unpack8(*reinterpret_cast<const uint4*>(p.x + t * p.C + c * 8), xv[k]);
-        if (p.branch != nullptr) {
-          float br[8], g[8];
-          unpack8(*reinterpret_cast<const uint4*>(p.branch + t * p.C + c * 8), br);
-          load8f(p.gate_res + mod_row + c * 8, g);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) xv[k][i] = fmaf(g[i], br[i], xv[k][i]);
-        }
-        if (p.x_out != nullptr) *reinterpret_cast<uint4*>(p.x_out + t * p.C + c * 8) = pack8(xv[k]);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          s1 += xv[k][i];
-          s2 = fmaf(xv[k][i], xv[k][i], s2);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) xv[k][i] = 0.f;
+      for (int i = 0; i < 8; ++i) {
+        s1 += xv[i];
+        s2 = fmaf(xv[i], xv[i], s2);
       }
     }
     float mu = 0.f, inv = 1.f;
     if (p.norm_type == 0) {
-      const float2 r = block_sum2(s1, s2, scratch);
-      inv = rsqrtf(r.y * inv_c + p.eps);
+      inv = rsqrtf(warp_sum(s2) * inv_c + p.eps);
     } else if (p.norm_type == 1) {
-      // two passes over the registers: mean, then the centred second moment
-      const float2 r = block_sum2(s1, 0.f, scratch);
-      mu = r.x * inv_c;
+      mu = warp_sum(s1) * inv_c;
+      // centred second moment from a second read of the row
       float d2 = 0.f;
+      for (int c = lane; c < nchunks; c += 32) {
+        float xv[8];
+        residual_chunk(p, t, mod_row, c, xv);
 #pragma unroll
-      for (int k = 0; k < kMaxSlots; ++k) {
-        const int c = threadIdx.x + k * kThreads;
-        if (c < nchunks) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) d2 = fmaf(xv[k][i] - mu, xv[k][i] - mu, d2);
-        }
+        for (int i = 0; i < 8; ++i) d2 = fmaf(xv[i] - mu, xv[i] - mu, d2);
       }
-      const float2 r2 = block_sum2(d2, 0.f, scratch);
-      inv = rsqrtf(r2.x * inv_c + p.eps);
+      inv = rsqrtf(warp_sum(d2) * inv_c + p.eps);
     }
+    for (int c = lane; c < nchunks; c += 32) {
+      float xv[8], sc[8], sh[8], hv[8];
+      residual_chunk(p, t, mod_row, c, xv);
+      load8f(p.scale + mod_row + c * 8, sc);
+      load8f(p.shift + mod_row + c * 8, sh);
 #pragma unroll
-    for (int k = 0; k < kMaxSlots; ++k) {
-      const int c = threadIdx.x + k * kThreads;
-      if (c < nchunks) {
-        float sc[8], sh[8], hv[8];
-        load8f(p.scale + mod_row + c * 8, sc);
-        load8f(p.shift + mod_row + c * 8, sh);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) hv[i] = fmaf((xv[k][i] - mu) * inv, 1.0f + sc[i], sh[i]);
-        *reinterpret_cast<uint4*>(p.h + t * p.C + c * 8) = pack8(hv);
-      }
+      for (int i = 0; i < 8; ++i) hv[i] = fmaf((xv[i] - mu) * inv, 1.0f + sc[i], sh[i]);
+      *reinterpret_cast<uint4*>(p.h + t * p.C + c * 8) = pack8(hv);
     }
-    // ---- part 2: SwiGLU
     if (p.gate != nullptr) {
       const __nv_bfloat16* grow = p.gate + t * p.gu_stride;
       const __nv_bfloat16* urow = p.up + t * p.gu_stride;
       __nv_bfloat16* arow = p.act + t * static_cast<int64_t>(p.F);
-      for (int c0 = threadIdx.x; c0 < fchunks; c0 += kThreads * kUnroll) {
+      for (int c0 = lane; c0 < fchunks; c0 += 32 * kUnroll) {
         uint4 gr[kUnroll], ur[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-          const int c = c0 + u * kThreads;
+          const int c = c0 + u * 32;
           if (c < fchunks) {
             gr[u] = *reinterpret_cast<const uint4*>(grow + c * 8);
             ur[u] = *reinterpret_cast<const uint4*>(urow + c * 8);
@@ -190,7 +170,7 @@ __global__ void __launch_bounds__(kThreads) modulate_swiglu_kernel(const ModPara
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-          const int c = c0 + u * kThreads;
+          const int c = c0 + u * 32;
           if (c < fchunks) {
             float g[8], uu[8], a[8];
             unpack8(gr[u], g);
@@ -230,17 +210,11 @@ int launch_modulate_swiglu(const void* x, const void* branch, void* x_out, void*
   p.gu_stride = gu_stride;
   p.act = static_cast<__nv_bfloat16*>(act);
   p.F = gate != nullptr ? F : 0;
-  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
-  const int grid = static_cast<int>(T < cap ? T : cap);
-  const int slots = (C / 8 + kThreads - 1) / kThreads;
-  if (slots <= 1)
-    modulate_swiglu_kernel<1><<<grid, kThreads, 0, stream>>>(p);
-  else if (slots <= 2)
-    modulate_swiglu_kernel<2><<<grid, kThreads, 0, stream>>>(p);
-  else if (slots <= 4)
-    modulate_swiglu_kernel<4><<<grid, kThreads, 0, stream>>>(p);
-  else
-    modulate_swiglu_kernel<8><<<grid, kThreads, 0, stream>>>(p);
+  const int64_t warps_per_block = kThreads / 32;
+  const int64_t want = (T + warps_per_block - 1) / warps_per_block;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 3;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  modulate_swiglu_kernel<<<grid, kThreads, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

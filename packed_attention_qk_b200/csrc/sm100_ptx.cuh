@@ -258,25 +258,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 64 (used for part of the softmax so the
-// SFU is not the only unit computing exponentials). Range reduction by the
-// nearest integer with additions only: adding 1.5 * 2^23 leaves n = round(x)
-// in the low mantissa bits of t, t - 1.5 * 2^23 is n as a float, and 2^n
-// scales by an integer add of n << 23 to the exponent bits. 2^f on
-// [-1/2, 1/2] is 1 + f (c1 + f (c2 + f c3)), a minimax fit of relative error
-// 1.0e-4 (coefficients from csrc/fit_exp2_poly.py). Inputs below -126
-// (including -inf) are clamped to -126, giving ~1e-38 instead of 0.
-__device__ __forceinline__ float ex2_fma(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = __fadd_rn(x, 12582912.0f);
-  const float n = __fadd_rn(t, -12582912.0f);
-  const float f = __fadd_rn(x, -n);
-  float p = fmaf(f, 0.055009059607982635f, 0.2422109693288803f);
-  p = fmaf(p, f, 0.6932829022407532f);
-  p = fmaf(p, f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` in bits 0-15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -60,10 +60,12 @@ constexpr int kRowsPerWork = 2 * kBM;
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Of every 8 score columns, this many take their exponential on the FMA pipe
-// (pqk::ex2_fma) and the rest on the SFU, balancing the two units.
-constexpr int kPolyPer8 = 0;
+// The running row maximum only moves when a tile's maximum exceeds it by
+// more than this (log2 units), so probabilities stay <= 2^threshold.
+#ifndef PQK_ATTN_RESCALE_LOG2
+#define PQK_ATTN_RESCALE_LOG2 8.0f
+#endif
+constexpr float kRescaleThreshold = PQK_ATTN_RESCALE_LOG2;
 constexpr int kSlabBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-byte swizzle width)
 
 template <int D>
@@ -208,6 +210,53 @@ __global__ void __launch_bounds__(kSchedThreads) build_schedule_kernel(const int
 }
 
 // ------------------------------------------------------------ attention
+
+// The 128 fp32 scores of this thread's row from tensor memory; columns at
+// or past `valid` become -inf.
+__device__ __forceinline__ void load_scores(uint32_t taddr, int valid, float (&s)[128]) {
+  uint32_t r[128];
+  tmem_ld_x128(taddr, r);
+#pragma unroll
+  for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(r[c]);
+  if (valid < kBN) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (c >= valid) s[c] = -INFINITY;
+  }
+}
+
+__device__ __forceinline__ float row_max(const float (&s)[128]) {
+  float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+#pragma unroll
+  for (int c = 4; c < 128; c += 4) {
+    m0 = fmaxf(m0, s[c]);
+    m1 = fmaxf(m1, s[c + 1]);
+    m2 = fmaxf(m2, s[c + 2]);
+    m3 = fmaxf(m3, s[c + 3]);
+  }
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+// p_c = 2^(s_c * scale_log2 - m) for the 128 columns, packed to bf16 pairs,
+// and their fp32 sum.
+__device__ __forceinline__ void exp_tile(const float (&s)[128], float scale_log2, float neg_m, uint32_t (&pk)[64],
+                                         float& sum) {
+  float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 128; c += 4) {
+    const float e0 = ex2_approx(fmaf(s[c], scale_log2, neg_m));
+    const float e1 = ex2_approx(fmaf(s[c + 1], scale_log2, neg_m));
+    const float e2 = ex2_approx(fmaf(s[c + 2], scale_log2, neg_m));
+    const float e3 = ex2_approx(fmaf(s[c + 3], scale_log2, neg_m));
+    l0 += e0;
+    l1 += e1;
+    l2 += e2;
+    l3 += e3;
+    pk[c / 2] = pack_bf16x2(e0, e1);
+    pk[c / 2 + 1] = pack_bf16x2(e2, e3);
+  }
+  sum = (l0 + l1) + (l2 + l3);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -417,36 +466,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         s_phase ^= 1u;
         tc_fence_after_sync();
-        uint32_t sr[128];
-        tmem_ld_x128(t_s, sr);
+        // keys at or past the request end (last tile only) are masked
+        const int valid = j == wk.n_kv - 1 ? wk.seg_len - j * kBN : kBN;
         float s[128];
-#pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-        if (j == wk.n_kv - 1) {
-          const int valid = wk.seg_len - j * kBN;
-          if (valid < kBN) {
-#pragma unroll
-            for (int c = 0; c < 128; ++c)
-              if (c >= valid) s[c] = -INFINITY;
-          }
-        }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
-        }
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+        load_scores(t_s, valid, s);
+        const float mx = row_max(s) * p.scale_log2;
+        const bool need_rescale = j > 0 && mx > m + kRescaleThreshold;
+        float alpha = 1.0f;
         if (j == 0) {
           m = mx;
-        } else if (mx > m + kRescaleThreshold) {
-          // O_i holds the products of tiles 0..j-1, all complete (s_full
-          // for tile j completed after them); rescale it before P_j V_j
-          const float alpha = ex2_approx(m - mx);
+        } else if (need_rescale) {
+          alpha = ex2_approx(m - mx);
           l *= alpha;
           m = mx;
+        }
+        // O_i holds the products of tiles 0..j-1, all complete (s_full for
+        // tile j completed after them): rescale it before P_j V_j. Tensor-
+        // memory loads and stores are warp-collective (.sync.aligned), so
+        // the whole warp takes this path when any of its rows needs it, the
+        // other rows with alpha = 1.
+        if (__any_sync(0xffffffffu, need_rescale)) {
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t ov[32];
@@ -456,21 +495,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_x32(t_o + c0, ov);
           }
         }
-        const float neg_m = -m;
-        float l0 = 0.f, l1 = 0.f;
         uint32_t pk[64];
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float x0 = fmaf(s[c], p.scale_log2, neg_m);
-          const float x1 = fmaf(s[c + 1], p.scale_log2, neg_m);
-          const bool poly = (c & 7) >= 8 - kPolyPer8;
-          const float p0 = poly ? ex2_fma(x0) : ex2_approx(x0);
-          const float p1 = poly ? ex2_fma(x1) : ex2_approx(x1);
-          l0 += p0;
-          l1 += p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-        }
-        l += l0 + l1;
+        float l_tile;
+        exp_tile(s, p.scale_log2, -m, pk, l_tile);
+        l += l_tile;
         tmem_st_x64(t_s, pk);
         tc_fence_before_sync();
         mbar_arrive(p_full(grp));
