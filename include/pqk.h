@@ -135,6 +135,30 @@ PQK_API int pqk_varlen_attn_fwd(const void* q, const void* k, const void* v, voi
                         void* stream);
 
 /*
+ * pqk_varlen_attn_fwd_noalloc -- pqk_varlen_attn_fwd for callers that cannot
+ * allocate device memory. The pages have no counterpart: this entry point
+ * exists for callers such as plugins or embedded runtimes that are handed
+ * only their input and output buffers by a host framework that owns the
+ * whole device heap, and so have no way to obtain the schedule workspace.
+ * The schedule lives instead in a fixed array inside the library's own
+ * device memory (about 48 KB on every GPU that loads the library, held
+ * until the process exits).
+ *
+ * Arguments and results are those of pqk_varlen_attn_fwd without the
+ * workspace. B may be at most 4096; a larger B returns PQK_ERR_WORKSPACE.
+ * The first call on a device looks up the array's device address (a CUDA
+ * runtime query, no allocation); make that first call before capturing a
+ * stream. Every call uses the same array, so calls whose work overlaps on
+ * the GPU (e.g. on different streams) race and must be serialised by the
+ * caller; each call rewrites the whole schedule it reads, so nothing needs
+ * to be cleared between calls.
+ */
+PQK_API int pqk_varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int64_t q_stride_t, int64_t k_stride_t, int64_t v_stride_t,
+                                int64_t o_stride_t, const int32_t* cu_seqlens, int B, int64_t T,
+                                int H, int D, float softmax_scale, void* stream);
+
+/*
  * pqk_modulate_swiglu -- fused adaLN modulation + normalisation + gated
  * residual, and SwiGLU in one pass (first page, section "融合 DiT 算子": the
  * small DiT operators RMSNorm, SwiGLU and residual connections fused, SwiGLU

@@ -21,7 +21,8 @@ ROPE_INTERLEAVED, ROPE_HALF = 0, 1
 NORM_RMS, NORM_LAYER, NORM_NONE = 0, 1, 2
 
 # every symbol include/pqk.h declares
-EXPORTS = ("pqk_qk_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd", "pqk_modulate_swiglu",
+EXPORTS = ("pqk_qk_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd",
+           "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu",
            "pqk_get_device_status", "pqk_set_wait_timeout_ns", "pqk_selftest_wait_timeout", "pqk_status_string",
            "pqk_version")
 
@@ -53,6 +54,9 @@ def lib(path: str | None = None) -> C.CDLL:
     L.pqk_varlen_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32, vp, sz,
                                       vp]
     L.pqk_varlen_attn_fwd.restype = i32
+    L.pqk_varlen_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32,
+                                              vp]
+    L.pqk_varlen_attn_fwd_noalloc.restype = i32
     L.pqk_modulate_swiglu.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, f32, vp, vp, i64, vp,
                                       i32, vp]
     L.pqk_modulate_swiglu.restype = i32
@@ -141,6 +145,26 @@ def varlen_attn_fwd(q, k, v, cu_seqlens, *, softmax_scale: float | None = None, 
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _token_stride(q, 3), _token_stride(k, 3),
         _token_stride(v, 3), _token_stride(o, 3), _ptr(cu_seqlens), B, T, H, D, scale, _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+def varlen_attn_fwd_noalloc(q, k, v, cu_seqlens, *, softmax_scale: float | None = None, o=None, lse=None,
+                            want_lse: bool = False, stream=None):
+    """Packed varlen attention for callers that cannot allocate device
+    memory: the tile schedule lives in the library's own fixed device array
+    (at most 4096 requests; calls must not overlap on the GPU). The outputs
+    are allocated here only when not passed in."""
+    import torch
+    T, H, D = q.shape
+    B = cu_seqlens.shape[0] - 1
+    scale = softmax_scale if softmax_scale is not None else D ** -0.5
+    if o is None:
+        o = torch.empty((T, H, D), dtype=q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((H, T), dtype=torch.float32, device=q.device)
+    _check("pqk_varlen_attn_fwd_noalloc", lib().pqk_varlen_attn_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _token_stride(q, 3), _token_stride(k, 3),
+        _token_stride(v, 3), _token_stride(o, 3), _ptr(cu_seqlens), B, T, H, D, scale, _stream(stream)))
     return o, lse
 
 
