@@ -66,6 +66,25 @@ constexpr int kMmaWarp = 9;
 #define PQK_ATTN_RESCALE_LOG2 8.0f
 #endif
 constexpr float kRescaleThreshold = PQK_ATTN_RESCALE_LOG2;
+// Softmax arithmetic on packed fp32 pairs (fma/add .f32x2) and three-input
+// max, halving the non-SFU instructions per score.
+#ifndef PQK_ATTN_PACKED
+#define PQK_ATTN_PACKED 1
+#endif
+constexpr bool kPacked = PQK_ATTN_PACKED != 0;
+// P written to tensor memory in 32-column chunks as it is computed (one
+// wait at the end) instead of all 64 packed registers at once.
+#ifndef PQK_ATTN_CHUNKED
+#define PQK_ATTN_CHUNKED 0
+#endif
+constexpr bool kChunked = PQK_ATTN_CHUNKED != 0;
+// Of every 8 columns, this many take their exponential on the FMA pipe
+// (packed polynomial) instead of the SFU.
+#ifndef PQK_ATTN_POLY_PER8
+#define PQK_ATTN_POLY_PER8 0
+#endif
+constexpr int kPolyPer8 = PQK_ATTN_POLY_PER8;
+static_assert(kPolyPer8 % 2 == 0 && kPolyPer8 >= 0 && kPolyPer8 <= 8, "pairs of columns per 8");
 constexpr int kSlabBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-byte swizzle width)
 
 template <int D>
@@ -226,36 +245,92 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, int valid, float (&s
 }
 
 __device__ __forceinline__ float row_max(const float (&s)[128]) {
-  float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+  if constexpr (kPacked) {
+    // four chains of three-input maxima over 2 new columns each
+    float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-  for (int c = 4; c < 128; c += 4) {
-    m0 = fmaxf(m0, s[c]);
-    m1 = fmaxf(m1, s[c + 1]);
-    m2 = fmaxf(m2, s[c + 2]);
-    m3 = fmaxf(m3, s[c + 3]);
+    for (int c = 4; c < 128; c += 8) {
+      m0 = max3(m0, s[c], s[c + 1]);
+      m1 = max3(m1, s[c + 2], s[c + 3]);
+      m2 = max3(m2, s[c + 4], s[c + 5]);
+      m3 = max3(m3, s[c + 6], s[c + 7]);
+    }
+    return max3(m0, m1, fmaxf(m2, m3));
+  } else {
+    float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+#pragma unroll
+    for (int c = 4; c < 128; c += 4) {
+      m0 = fmaxf(m0, s[c]);
+      m1 = fmaxf(m1, s[c + 1]);
+      m2 = fmaxf(m2, s[c + 2]);
+      m3 = fmaxf(m3, s[c + 3]);
+    }
+    return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
   }
-  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-// p_c = 2^(s_c * scale_log2 - m) for the 128 columns, packed to bf16 pairs,
-// and their fp32 sum.
-__device__ __forceinline__ void exp_tile(const float (&s)[128], float scale_log2, float neg_m, uint32_t (&pk)[64],
-                                         float& sum) {
-  float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-#pragma unroll
-  for (int c = 0; c < 128; c += 4) {
-    const float e0 = ex2_approx(fmaf(s[c], scale_log2, neg_m));
-    const float e1 = ex2_approx(fmaf(s[c + 1], scale_log2, neg_m));
-    const float e2 = ex2_approx(fmaf(s[c + 2], scale_log2, neg_m));
-    const float e3 = ex2_approx(fmaf(s[c + 3], scale_log2, neg_m));
-    l0 += e0;
-    l1 += e1;
-    l2 += e2;
-    l3 += e3;
-    pk[c / 2] = pack_bf16x2(e0, e1);
-    pk[c / 2 + 1] = pack_bf16x2(e2, e3);
+// Exponentials of 4 consecutive columns starting at c (a multiple of 4).
+__device__ __forceinline__ void exp4(const float (&s)[128], int c, float scale_log2, float neg_m, float (&e)[4]) {
+  float x0, x1, x2, x3;
+  if constexpr (kPacked) {
+    fma2_bcast(s[c], s[c + 1], scale_log2, neg_m, x0, x1);
+    fma2_bcast(s[c + 2], s[c + 3], scale_log2, neg_m, x2, x3);
+  } else {
+    x0 = fmaf(s[c], scale_log2, neg_m);
+    x1 = fmaf(s[c + 1], scale_log2, neg_m);
+    x2 = fmaf(s[c + 2], scale_log2, neg_m);
+    x3 = fmaf(s[c + 3], scale_log2, neg_m);
   }
-  sum = (l0 + l1) + (l2 + l3);
+  // columns (c & 7) in [8 - kPolyPer8, 8) use the FMA-pipe polynomial
+  if ((c & 7) >= 8 - kPolyPer8) ex2_poly2(x0, x1, e[0], e[1]);
+  else { e[0] = ex2_approx(x0); e[1] = ex2_approx(x1); }
+  if (((c + 2) & 7) >= 8 - kPolyPer8) ex2_poly2(x2, x3, e[2], e[3]);
+  else { e[2] = ex2_approx(x2); e[3] = ex2_approx(x3); }
+}
+
+// p_c = 2^(s_c * scale_log2 - m) for the 128 columns, rounded to bf16 pairs
+// and written over the first 64 columns of S at `t_p` (tensor memory); returns
+// their fp32 sum. Waits for its tensor-memory stores before returning.
+__device__ __forceinline__ float exp_tile_store(const float (&s)[128], float scale_log2, float neg_m, uint32_t t_p) {
+  float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+  if constexpr (kChunked) {
+#pragma unroll
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int c = c0; c < c0 + 32; c += 4) {
+        float e[4];
+        exp4(s, c, scale_log2, neg_m, e);
+        if constexpr (kPacked) {
+          add2_acc(l0, l1, e[0], e[1]);
+          add2_acc(l2, l3, e[2], e[3]);
+        } else {
+          l0 += e[0]; l1 += e[1]; l2 += e[2]; l3 += e[3];
+        }
+        pk[(c - c0) / 2] = pack_bf16x2(e[0], e[1]);
+        pk[(c - c0) / 2 + 1] = pack_bf16x2(e[2], e[3]);
+      }
+      tmem_st_x16_nowait(t_p + c0 / 2, pk);
+    }
+    tmem_st_wait();
+  } else {
+    uint32_t pk[64];
+#pragma unroll
+    for (int c = 0; c < 128; c += 4) {
+      float e[4];
+      exp4(s, c, scale_log2, neg_m, e);
+      if constexpr (kPacked) {
+        add2_acc(l0, l1, e[0], e[1]);
+        add2_acc(l2, l3, e[2], e[3]);
+      } else {
+        l0 += e[0]; l1 += e[1]; l2 += e[2]; l3 += e[3];
+      }
+      pk[c / 2] = pack_bf16x2(e[0], e[1]);
+      pk[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
+    }
+    tmem_st_x64(t_p, pk);
+  }
+  return (l0 + l1) + (l2 + l3);
 }
 
 template <int D>
@@ -495,11 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_x32(t_o + c0, ov);
           }
         }
-        uint32_t pk[64];
-        float l_tile;
-        exp_tile(s, p.scale_log2, -m, pk, l_tile);
-        l += l_tile;
-        tmem_st_x64(t_s, pk);
+        l += exp_tile_store(s, p.scale_log2, -m, t_s);
         tc_fence_before_sync();
         mbar_arrive(p_full(grp));
       }
