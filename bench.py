@@ -320,6 +320,32 @@ def run_ours(args, w):
     epi_bytes = w.epilogue_bytes(with_branch=True)
     epi_gbs = epi_bytes / (statistics.mean(epi) * 1e-3) / 1e9
 
+    # the three-axis RoPE variant on the same Q, K: (t, h, w) ids for the video
+    # latent grid, one-axis ids repeated for text and audio
+    pos3 = torch.from_numpy(w.positions3()).to(dev)
+    sections = (w.D // 8, 3 * w.D // 16, 3 * w.D // 16)
+    ev3 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for _ in range(2):
+        pqk.qk_norm_rope_3axis(d["q"], d["k"], d["w_q"], d["w_k"], pos3, sections, eps=w.eps,
+                               rope_base=w.rope_base, q_out=o["qn"], k_out=o["kn"])
+    ev3[0].record()
+    reps3 = 10
+    for _ in range(reps3):
+        pqk.qk_norm_rope_3axis(d["q"], d["k"], d["w_q"], d["w_k"], pos3, sections, eps=w.eps,
+                               rope_base=w.rope_base, q_out=o["qn"], k_out=o["kn"])
+    ev3[1].record()
+    torch.cuda.synchronize()
+    rope3_us = ev3[0].elapsed_time(ev3[1]) / reps3 * 1e3
+    rope3_gbs = w.prologue_bytes(three_axis=True) / (rope3_us * 1e-6) / 1e9
+    # the one-axis kernel timed the same way (back to back), for comparison
+    ev3[0].record()
+    for _ in range(reps3):
+        pqk.qk_norm_rope(d["q"], d["k"], d["w_q"], d["w_k"], d["pos"], eps=w.eps, rope_base=w.rope_base,
+                         q_out=o["qn"], k_out=o["kn"])
+    ev3[1].record()
+    torch.cuda.synchronize()
+    rope1_b2b_us = ev3[0].elapsed_time(ev3[1]) / reps3 * 1e3
+
     # e2e through host buffers: pinned H2D of every input, the three calls,
     # D2H of the block outputs (x', h, act), all inside the timed region
     e2e = None
@@ -376,7 +402,11 @@ def run_ours(args, w):
                     "qk_norm_rope_frac_hbm": pro_gbs / pk["hbm_gbs"],
                     "varlen_attn_ms": att_ms, "varlen_attn_tflops": attn_tflops,
                     "modulate_swiglu_us": statistics.mean(epi) * 1e3, "modulate_swiglu_gbs": epi_gbs,
-                    "modulate_swiglu_frac_hbm": epi_gbs / pk["hbm_gbs"], "hbm_peak_gbs": pk["hbm_gbs"]},
+                    "modulate_swiglu_frac_hbm": epi_gbs / pk["hbm_gbs"], "hbm_peak_gbs": pk["hbm_gbs"],
+                    "qk_norm_rope_3axis_us": rope3_us, "qk_norm_rope_3axis_gbs": rope3_gbs,
+                    "qk_norm_rope_3axis_frac_hbm": rope3_gbs / pk["hbm_gbs"],
+                    "qk_norm_rope_3axis_sections": list(sections),
+                    "qk_norm_rope_back_to_back_us": rope1_b2b_us},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * K,

@@ -95,6 +95,28 @@ PQK_API int pqk_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, vo
                      float eps, float rope_base, int rope_style, void* stream);
 
 /*
+ * pqk_qk_norm_rope_3axis -- pqk_qk_norm_rope with a (t, h, w) position per
+ * token for video latents. The pages give no RoPE variant; the reading
+ * taken: every pair j keeps theta_j = rope_base^(-2j/D) and takes its angle
+ * from one axis, the D/2 pair indices being split into consecutive sections
+ * of sec_t, sec_h, sec_w pairs (sec_t + sec_h + sec_w == D/2):
+ *   phi_j = pos3[t][0] * theta_j for j < sec_t,
+ *           pos3[t][1] * theta_j for sec_t <= j < sec_t + sec_h,
+ *           pos3[t][2] * theta_j otherwise.
+ * Tokens whose three ids are equal (text, audio) get exactly the one-axis
+ * rotation of pqk_qk_norm_rope.
+ *
+ * pos3          device int32 [T, 3]. Other arguments and errors as in
+ *               pqk_qk_norm_rope; sections that are negative or do not sum
+ *               to D/2 return PQK_ERR_INVALID_ARG.
+ */
+PQK_API int pqk_qk_norm_rope_3axis(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                           int64_t q_stride_t, int64_t k_stride_t, const void* q_weight,
+                           const void* k_weight, const int32_t* pos3, int sec_t, int sec_h,
+                           int sec_w, int64_t T, int H, int D, float eps, float rope_base,
+                           int rope_style, void* stream);
+
+/*
  * pqk_varlen_attn_workspace_size -- bytes of device workspace that
  * pqk_varlen_attn_fwd needs for B requests (its tile schedule).
  */

@@ -48,7 +48,12 @@ def load(path: str):
     L.oracle_modulate_swiglu.argtypes = [vp, vp, C.c_int, f32p, f32p, f32p, i32p, C.c_int, C.c_int64,
                                          C.c_int, C.c_int, C.c_double, vp, vp, C.c_int64, C.c_int, i32p,
                                          C.c_int64, f64p, f64p, f64p]
-    for f in (L.oracle_qk_norm_rope, L.oracle_varlen_attn, L.oracle_modulate_swiglu):
+    L.oracle_qk_norm_rope_3axis.argtypes = [vp, C.c_int, C.c_int64, vp, C.c_int, i32p, i32p, C.c_int64, C.c_int,
+                                            C.c_int, C.c_double, C.c_double, C.c_int, i32p, C.c_int64, f64p]
+    L.oracle_qk_fullc_norm_rope.argtypes = [vp, C.c_int, C.c_int64, vp, C.c_int, i32p, C.c_int64, C.c_int, C.c_int,
+                                            C.c_double, C.c_double, C.c_int, i32p, C.c_int64, f64p]
+    for f in (L.oracle_qk_norm_rope, L.oracle_qk_norm_rope_3axis, L.oracle_qk_fullc_norm_rope, L.oracle_varlen_attn,
+              L.oracle_modulate_swiglu):
         f.restype = C.c_int
     L.oracle_num_threads.restype = C.c_int
     return L
@@ -106,6 +111,44 @@ def qk_norm_rope(x: np.ndarray, w: np.ndarray, pos: np.ndarray, eps: float, base
                                    T, H, D, eps, base, style, _ptr(r, C.c_int32), n, _ptr(y, C.c_double))
     if rc:
         raise ValueError("oracle_qk_norm_rope: invalid arguments")
+    return y
+
+
+def qk_norm_rope_3axis(x: np.ndarray, w: np.ndarray, pos3: np.ndarray, sections, eps: float, base: float,
+                       style: int = ROPE_INTERLEAVED, rows=None) -> np.ndarray:
+    """x: [T, H, D]; pos3: [T, 3] (t, h, w) ids; sections: pairs per axis."""
+    T, H, D = x.shape
+    stride_t = x.strides[0] // x.itemsize
+    assert x.strides[2] == x.itemsize and x.strides[1] == D * x.itemsize
+    w = np.ascontiguousarray(w)
+    pos3 = np.ascontiguousarray(pos3, dtype=np.int32)
+    assert pos3.shape == (T, 3)
+    sec = np.ascontiguousarray(sections, dtype=np.int32)
+    r, n = _rows(rows)
+    y = np.empty((n if r is not None else T, H, D), np.float64)
+    rc = lib().oracle_qk_norm_rope_3axis(_ptr(x), _kind(x), stride_t, _ptr(w), _kind(w), _ptr(pos3, C.c_int32),
+                                         _ptr(sec, C.c_int32), T, H, D, eps, base, style, _ptr(r, C.c_int32), n,
+                                         _ptr(y, C.c_double))
+    if rc:
+        raise ValueError("oracle_qk_norm_rope_3axis: invalid arguments")
+    return y
+
+
+def qk_fullc_norm_rope(x: np.ndarray, w: np.ndarray, pos: np.ndarray, eps: float, base: float,
+                       style: int = ROPE_INTERLEAVED, rows=None) -> np.ndarray:
+    """x: [T, H, D]; w: [H*D]; RMS over all H*D elements of a token."""
+    T, H, D = x.shape
+    stride_t = x.strides[0] // x.itemsize
+    assert x.strides[2] == x.itemsize and x.strides[1] == D * x.itemsize
+    w = np.ascontiguousarray(w).reshape(-1)
+    assert w.shape[0] == H * D
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    r, n = _rows(rows)
+    y = np.empty((n if r is not None else T, H, D), np.float64)
+    rc = lib().oracle_qk_fullc_norm_rope(_ptr(x), _kind(x), stride_t, _ptr(w), _kind(w), _ptr(pos, C.c_int32), T, H,
+                                         D, eps, base, style, _ptr(r, C.c_int32), n, _ptr(y, C.c_double))
+    if rc:
+        raise ValueError("oracle_qk_fullc_norm_rope: invalid arguments")
     return y
 
 

@@ -12,6 +12,12 @@
  *                             serving with vLLM-Omni", section "System-wide
  *                             optimizations in vLLM-Omni", bullet "Fused DiT
  *                             operators").
+ *   oracle_qk_norm_rope_3axis -- the same with a (t, h, w) position per
+ *                             token for video latents (a reading: the pages
+ *                             give no RoPE variant; see the function).
+ *   oracle_qk_fullc_norm_rope -- the same with the norm over all heads of
+ *                             a token (weight of H*D entries), a reading of
+ *                             "Q/K normalisation" the pages leave open.
  *   oracle_varlen_attn     -- softmax attention over one packed sequence per
  *                             request, valid tokens only (first page, section
  *                             "长序列注意力与通信优化"; second page, bullet
@@ -83,6 +89,36 @@ static int check_cu(const int32_t* cu, int B, int64_t T) {
   return 0;
 }
 
+/* RMSNorm of the D elements of one (token, head) row, times the weight:
+ * n_d = x_d / sqrt(mean(x^2) + eps) * w_d. */
+static void rms_times_weight(const void* x, int x_kind, int64_t row, const void* w, int w_kind, int D,
+                             double eps, double* n) {
+  double ms = 0.0;
+  for (int d = 0; d < D; ++d) {
+    double v = load(x, x_kind, row + d);
+    ms += v * v;
+  }
+  ms /= (double)D;
+  const double inv = 1.0 / sqrt(ms + eps);
+  for (int d = 0; d < D; ++d) n[d] = load(x, x_kind, row + d) * inv * load(w, w_kind, d);
+}
+
+/* Element indices of RoPE pair j. */
+static void pair_of(int style, int j, int D, int* ia, int* ib) {
+  if (style == ORACLE_ROPE_INTERLEAVED) { *ia = 2 * j; *ib = 2 * j + 1; }
+  else { *ia = j; *ib = j + D / 2; }
+}
+
+/* theta_j = base^(-2j/D). */
+static double rope_theta(double base, int j, int D) { return pow(base, -2.0 * (double)j / (double)D); }
+
+/* (a, b) <- (a cos phi - b sin phi, a sin phi + b cos phi). */
+static void rotate_pair(const double* n, double* out, int ia, int ib, double phi) {
+  const double a = n[ia], b = n[ib];
+  out[ia] = a * cos(phi) - b * sin(phi);
+  out[ib] = a * sin(phi) + b * cos(phi);
+}
+
 /*
  * RMSNorm over the D elements of one (token, head) row, weight w (shared by
  * all heads), then RoPE with angle phi_j = pos[t] * base^(-2j/D), j < D/2:
@@ -104,25 +140,89 @@ int oracle_qk_norm_rope(const void* x, int x_kind, int64_t stride_t, const void*
     if (t < 0 || t >= T) { ++bad; continue; }
     double* n = (double*)malloc(sizeof(double) * (size_t)D);
     for (int h = 0; h < H; ++h) {
-      const int64_t base_idx = t * stride_t + (int64_t)h * D;
-      double ms = 0.0;
-      for (int d = 0; d < D; ++d) {
-        double v = load(x, x_kind, base_idx + d);
-        ms += v * v;
-      }
-      ms /= (double)D;
-      const double inv = 1.0 / sqrt(ms + eps);
-      for (int d = 0; d < D; ++d) n[d] = load(x, x_kind, base_idx + d) * inv * load(w, w_kind, d);
+      rms_times_weight(x, x_kind, t * stride_t + (int64_t)h * D, w, w_kind, D, eps, n);
       double* out = y + (r * H + h) * (int64_t)D;
       for (int j = 0; j < D / 2; ++j) {
-        const double theta = pow(base, -2.0 * (double)j / (double)D);
-        const double phi = (double)pos[t] * theta;
         int ia, ib;
-        if (style == ORACLE_ROPE_INTERLEAVED) { ia = 2 * j; ib = 2 * j + 1; }
-        else { ia = j; ib = j + D / 2; }
-        const double a = n[ia], b = n[ib];
-        out[ia] = a * cos(phi) - b * sin(phi);
-        out[ib] = a * sin(phi) + b * cos(phi);
+        pair_of(style, j, D, &ia, &ib);
+        rotate_pair(n, out, ia, ib, (double)pos[t] * rope_theta(base, j, D));
+      }
+    }
+    free(n);
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * RMSNorm as in oracle_qk_norm_rope, then RoPE with three position axes:
+ * pair j < D/2 keeps the frequency theta_j = base^(-2j/D) but takes its
+ * position from axis a(j) of pos3[t] = (t-id, h-id, w-id), where the pair
+ * indices are split into consecutive sections of sec[0], sec[1], sec[2]
+ * pairs (sec[0] + sec[1] + sec[2] = D/2): a(j) = 0 for j < sec[0], 1 for
+ * j < sec[0] + sec[1], else 2. pos3: [T, 3] int32.
+ */
+int oracle_qk_norm_rope_3axis(const void* x, int x_kind, int64_t stride_t, const void* w, int w_kind,
+                              const int32_t* pos3, const int32_t* sec, int64_t T, int H, int D, double eps,
+                              double base, int style, const int32_t* rows, int64_t nrows, double* y) {
+  if (D <= 0 || D % 2 || H <= 0 || T < 0 || !(eps >= 0.0) || !(base > 0.0)) return -1;
+  if (style != ORACLE_ROPE_INTERLEAVED && style != ORACLE_ROPE_HALF) return -1;
+  if (sec[0] < 0 || sec[1] < 0 || sec[2] < 0 || sec[0] + sec[1] + sec[2] != D / 2) return -1;
+  if (rows == NULL) nrows = T;
+  int64_t bad = 0;
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int64_t t = rows ? rows[r] : r;
+    if (t < 0 || t >= T) { ++bad; continue; }
+    double* n = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int h = 0; h < H; ++h) {
+      rms_times_weight(x, x_kind, t * stride_t + (int64_t)h * D, w, w_kind, D, eps, n);
+      double* out = y + (r * H + h) * (int64_t)D;
+      for (int j = 0; j < D / 2; ++j) {
+        const int axis = j < sec[0] ? 0 : (j < sec[0] + sec[1] ? 1 : 2);
+        int ia, ib;
+        pair_of(style, j, D, &ia, &ib);
+        rotate_pair(n, out, ia, ib, (double)pos3[t * 3 + axis] * rope_theta(base, j, D));
+      }
+    }
+    free(n);
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * Full-width variant: the RMS is taken over all H*D elements of the token's
+ * row of X (every head together), the weight w has H*D entries, then every
+ * head is rotated as in oracle_qk_norm_rope:
+ *   y_{h,d} = x_{h,d} / sqrt(mean_{h',d'}(x^2) + eps) * w[h*D + d].
+ */
+int oracle_qk_fullc_norm_rope(const void* x, int x_kind, int64_t stride_t, const void* w, int w_kind,
+                              const int32_t* pos, int64_t T, int H, int D, double eps, double base, int style,
+                              const int32_t* rows, int64_t nrows, double* y) {
+  if (D <= 0 || D % 2 || H <= 0 || T < 0 || !(eps >= 0.0) || !(base > 0.0)) return -1;
+  if (style != ORACLE_ROPE_INTERLEAVED && style != ORACLE_ROPE_HALF) return -1;
+  if (rows == NULL) nrows = T;
+  int64_t bad = 0;
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int64_t t = rows ? rows[r] : r;
+    if (t < 0 || t >= T) { ++bad; continue; }
+    const int64_t width = (int64_t)H * D;
+    double ms = 0.0;
+    for (int64_t e = 0; e < width; ++e) {
+      const double v = load(x, x_kind, t * stride_t + e);
+      ms += v * v;
+    }
+    ms /= (double)width;
+    const double inv = 1.0 / sqrt(ms + eps);
+    double* n = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int h = 0; h < H; ++h) {
+      for (int d = 0; d < D; ++d)
+        n[d] = load(x, x_kind, t * stride_t + (int64_t)h * D + d) * inv * load(w, w_kind, (int64_t)h * D + d);
+      double* out = y + (r * H + h) * (int64_t)D;
+      for (int j = 0; j < D / 2; ++j) {
+        int ia, ib;
+        pair_of(style, j, D, &ia, &ib);
+        rotate_pair(n, out, ia, ib, (double)pos[t] * rope_theta(base, j, D));
       }
     }
     free(n);

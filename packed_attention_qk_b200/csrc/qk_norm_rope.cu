@@ -13,6 +13,8 @@
 // all 2*H rows; the angle pos * base^(-2j/D) is formed and reduced modulo
 // 2*pi in fp64 (positions reach ~1.9e5, where an fp32 angle is off by
 // ~1e-2 rad) and only the reduced angle goes through the fp32 sine/cosine.
+// The three-axis variant (video latents with (t, h, w) ids) keeps the same
+// frequencies and takes each pair's position from the axis of its section.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -35,7 +37,8 @@ struct QkParams {
   int64_t k_stride;
   const __nv_bfloat16* wq;
   const __nv_bfloat16* wk;
-  const int32_t* pos;
+  const int32_t* pos;  // [T] ids, or [T, 3] (t, h, w) ids for the three-axis variant
+  int sec0, sec1;      // three-axis: pairs j < sec0 use t, j < sec0 + sec1 use h, the rest w
   int64_t T;
   int H;
   float eps;
@@ -71,7 +74,7 @@ __device__ __forceinline__ void rope_sincos(int32_t pos, double theta, float& c,
   __sincosf(r, &s, &c);  // |r| <= pi: absolute error ~4e-7
 }
 
-template <int D>
+template <int D, bool kThreeAxis>
 __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParams p) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerStep = 32 / kLanesPerRow;
@@ -90,20 +93,36 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
     theta[j] = exp2(-2.0 * static_cast<double>(j) / static_cast<double>(D) * p.log2_base);
   __syncthreads();
   const int j0 = interleaved ? 4 * chunk : 8 * (chunk % kHalfLanes);
+  // three-axis: which of (t, h, w) each of this lane's pair slots reads
+  int axis[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int j = j0 + i;
+    axis[i] = kThreeAxis ? (j < p.sec0 ? 0 : (j < p.sec0 + p.sec1 ? 1 : 2)) : 0;
+  }
   const uint4 wq_raw = *reinterpret_cast<const uint4*>(p.wq + chunk * 8);
   const uint4 wk_raw = *reinterpret_cast<const uint4*>(p.wk + chunk * 8);
   const int rows = 2 * p.H;
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + threadIdx.x / 32; t < p.T;
        t += warps_total) {
-    const int32_t pos = p.pos[t];
+    int32_t pos3[3];
+    if constexpr (kThreeAxis) {
+      pos3[0] = p.pos[3 * t];
+      pos3[1] = p.pos[3 * t + 1];
+      pos3[2] = p.pos[3 * t + 2];
+    } else {
+      pos3[0] = p.pos[t];
+    }
     float cs[8], sn[8];
     if (interleaved) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) rope_sincos(pos, theta[j0 + i], cs[i], sn[i]);
+      for (int i = 0; i < 4; ++i)
+        rope_sincos(kThreeAxis ? pos3[axis[i]] : pos3[0], theta[j0 + i], cs[i], sn[i]);
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) rope_sincos(pos, theta[j0 + i], cs[i], sn[i]);
+      for (int i = 0; i < 8; ++i)
+        rope_sincos(kThreeAxis ? pos3[axis[i]] : pos3[0], theta[j0 + i], cs[i], sn[i]);
     }
     for (int r0 = 0; r0 < rows; r0 += kRowsPerStep * kUnroll) {
       uint4 raw[kUnroll];
@@ -165,8 +184,9 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
 }  // namespace
 
 int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride,
-                        int64_t k_stride, const void* wq, const void* wk, const int32_t* pos, int64_t T, int H,
-                        int D, float eps, float rope_base, int style, cudaStream_t stream, int num_sms) {
+                        int64_t k_stride, const void* wq, const void* wk, const int32_t* pos, const int* sections,
+                        int64_t T, int H, int D, float eps, float rope_base, int style, cudaStream_t stream,
+                        int num_sms) {
   QkParams p;
   p.q_in = static_cast<const __nv_bfloat16*>(q_in);
   p.k_in = static_cast<const __nv_bfloat16*>(k_in);
@@ -177,6 +197,8 @@ int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k
   p.wq = static_cast<const __nv_bfloat16*>(wq);
   p.wk = static_cast<const __nv_bfloat16*>(wk);
   p.pos = pos;
+  p.sec0 = sections ? sections[0] : 0;
+  p.sec1 = sections ? sections[1] : 0;
   p.T = T;
   p.H = H;
   p.eps = eps;
@@ -186,10 +208,15 @@ int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k
   const int64_t want = (T + warps_per_block - 1) / warps_per_block;
   const int64_t cap = static_cast<int64_t>(num_sms) * 3;
   const int grid = static_cast<int>(want < cap ? want : cap);
-  if (D == 128)
-    qk_norm_rope_kernel<128><<<grid, kThreads, 0, stream>>>(p);
+  const bool three = sections != nullptr;
+  if (D == 128 && !three)
+    qk_norm_rope_kernel<128, false><<<grid, kThreads, 0, stream>>>(p);
+  else if (D == 128)
+    qk_norm_rope_kernel<128, true><<<grid, kThreads, 0, stream>>>(p);
+  else if (!three)
+    qk_norm_rope_kernel<64, false><<<grid, kThreads, 0, stream>>>(p);
   else
-    qk_norm_rope_kernel<64><<<grid, kThreads, 0, stream>>>(p);
+    qk_norm_rope_kernel<64, true><<<grid, kThreads, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

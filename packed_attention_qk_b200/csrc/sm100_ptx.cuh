@@ -249,57 +249,7 @@ __device__ __forceinline__ void tmem_st_x64(uint32_t taddr, const uint32_t (&r)[
       : "memory");
 }
 
-// Stores 16 columns without waiting (source registers are read at issue);
-// pair with tmem_st_wait() before the stores must be visible.
-__device__ __forceinline__ void tmem_st_x16_nowait(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n"
-      :
-      : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
 // ---------------------------------------------------------------- math
-
-// 2^x on the FMA pipe for two values at once (packed fp32 pairs), x >= -126
-// after the clamp. Range reduction by the nearest integer with additions
-// only (adding 1.5 * 2^23 leaves n = round(x) in the low mantissa bits of t;
-// t - 1.5 * 2^23 is n as a float), 2^f on [-1/2, 1/2] by the polynomial
-// 1 + f (c1 + f (c2 + f c3)) whose coefficients were fitted here (minimax
-// relative error 1.0e-4 with the constant term fixed at 1, a linear program
-// over a dense grid, rounded to fp32), and the scaling by 2^n as an integer
-// add of n << 23 to the exponent bits. Masked (-inf) inputs give ~1e-38.
-__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
-  x0 = fmaxf(x0, -126.0f);
-  x1 = fmaxf(x1, -126.0f);
-  uint32_t t0, t1, p0, p1;
-  asm("{\n"
-      ".reg .b64 rx, rt, rn, rf, rp, rk, rm;\n"
-      "mov.b64 rx, {%4, %5};\n"
-      "mov.b64 rk, {%6, %6};\n"           // 1.5 * 2^23
-      "add.rn.f32x2 rt, rx, rk;\n"
-      "sub.rn.f32x2 rn, rt, rk;\n"
-      "sub.rn.f32x2 rf, rx, rn;\n"
-      "mov.b64 rm, {%8, %8};\n"           // c2
-      "mov.b64 rk, {%7, %7};\n"           // c3
-      "fma.rn.f32x2 rp, rf, rk, rm;\n"
-      "mov.b64 rm, {%9, %9};\n"           // c1
-      "fma.rn.f32x2 rp, rp, rf, rm;\n"
-      "mov.b64 rm, {%10, %10};\n"         // 1
-      "fma.rn.f32x2 rp, rp, rf, rm;\n"
-      "mov.b64 {%0, %1}, rt;\n"
-      "mov.b64 {%2, %3}, rp;\n"
-      "}\n"
-      : "=r"(t0), "=r"(t1), "=r"(p0), "=r"(p1)
-      : "f"(x0), "f"(x1), "f"(12582912.0f), "f"(0.055009059607982635f), "f"(0.2422109693288803f),
-        "f"(0.6932829022407532f), "f"(1.0f));
-  y0 = __uint_as_float(p0 + (t0 << 23));
-  y1 = __uint_as_float(p1 + (t1 << 23));
-}
-
 
 // 2^x on the SFU (approximate, flushes denormals; 2^-inf = 0).
 __device__ __forceinline__ float ex2_approx(float x) {

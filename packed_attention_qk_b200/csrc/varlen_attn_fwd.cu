@@ -72,19 +72,6 @@ constexpr float kRescaleThreshold = PQK_ATTN_RESCALE_LOG2;
 #define PQK_ATTN_PACKED 1
 #endif
 constexpr bool kPacked = PQK_ATTN_PACKED != 0;
-// P written to tensor memory in 32-column chunks as it is computed (one
-// wait at the end) instead of all 64 packed registers at once.
-#ifndef PQK_ATTN_CHUNKED
-#define PQK_ATTN_CHUNKED 0
-#endif
-constexpr bool kChunked = PQK_ATTN_CHUNKED != 0;
-// Of every 8 columns, this many take their exponential on the FMA pipe
-// (packed polynomial) instead of the SFU.
-#ifndef PQK_ATTN_POLY_PER8
-#define PQK_ATTN_POLY_PER8 0
-#endif
-constexpr int kPolyPer8 = PQK_ATTN_POLY_PER8;
-static_assert(kPolyPer8 % 2 == 0 && kPolyPer8 >= 0 && kPolyPer8 <= 8, "pairs of columns per 8");
 constexpr int kSlabBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-byte swizzle width)
 
 template <int D>
@@ -281,11 +268,10 @@ __device__ __forceinline__ void exp4(const float (&s)[128], int c, float scale_l
     x2 = fmaf(s[c + 2], scale_log2, neg_m);
     x3 = fmaf(s[c + 3], scale_log2, neg_m);
   }
-  // columns (c & 7) in [8 - kPolyPer8, 8) use the FMA-pipe polynomial
-  if ((c & 7) >= 8 - kPolyPer8) ex2_poly2(x0, x1, e[0], e[1]);
-  else { e[0] = ex2_approx(x0); e[1] = ex2_approx(x1); }
-  if (((c + 2) & 7) >= 8 - kPolyPer8) ex2_poly2(x2, x3, e[2], e[3]);
-  else { e[2] = ex2_approx(x2); e[3] = ex2_approx(x3); }
+  e[0] = ex2_approx(x0);
+  e[1] = ex2_approx(x1);
+  e[2] = ex2_approx(x2);
+  e[3] = ex2_approx(x3);
 }
 
 // p_c = 2^(s_c * scale_log2 - m) for the 128 columns, rounded to bf16 pairs
@@ -293,43 +279,24 @@ __device__ __forceinline__ void exp4(const float (&s)[128], int c, float scale_l
 // their fp32 sum. Waits for its tensor-memory stores before returning.
 __device__ __forceinline__ float exp_tile_store(const float (&s)[128], float scale_log2, float neg_m, uint32_t t_p) {
   float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-  if constexpr (kChunked) {
+  uint32_t pk[64];
 #pragma unroll
-    for (int c0 = 0; c0 < 128; c0 += 32) {
-      uint32_t pk[16];
-#pragma unroll
-      for (int c = c0; c < c0 + 32; c += 4) {
-        float e[4];
-        exp4(s, c, scale_log2, neg_m, e);
-        if constexpr (kPacked) {
-          add2_acc(l0, l1, e[0], e[1]);
-          add2_acc(l2, l3, e[2], e[3]);
-        } else {
-          l0 += e[0]; l1 += e[1]; l2 += e[2]; l3 += e[3];
-        }
-        pk[(c - c0) / 2] = pack_bf16x2(e[0], e[1]);
-        pk[(c - c0) / 2 + 1] = pack_bf16x2(e[2], e[3]);
-      }
-      tmem_st_x16_nowait(t_p + c0 / 2, pk);
+  for (int c = 0; c < 128; c += 4) {
+    float e[4];
+    exp4(s, c, scale_log2, neg_m, e);
+    if constexpr (kPacked) {
+      add2_acc(l0, l1, e[0], e[1]);
+      add2_acc(l2, l3, e[2], e[3]);
+    } else {
+      l0 += e[0];
+      l1 += e[1];
+      l2 += e[2];
+      l3 += e[3];
     }
-    tmem_st_wait();
-  } else {
-    uint32_t pk[64];
-#pragma unroll
-    for (int c = 0; c < 128; c += 4) {
-      float e[4];
-      exp4(s, c, scale_log2, neg_m, e);
-      if constexpr (kPacked) {
-        add2_acc(l0, l1, e[0], e[1]);
-        add2_acc(l2, l3, e[2], e[3]);
-      } else {
-        l0 += e[0]; l1 += e[1]; l2 += e[2]; l3 += e[3];
-      }
-      pk[c / 2] = pack_bf16x2(e[0], e[1]);
-      pk[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
-    }
-    tmem_st_x64(t_p, pk);
+    pk[c / 2] = pack_bf16x2(e[0], e[1]);
+    pk[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
   }
+  tmem_st_x64(t_p, pk);
   return (l0 + l1) + (l2 + l3);
 }
 

@@ -165,13 +165,33 @@ class Workload:
         assert p.shape[0] == self.T
         return p
 
+    def positions3(self, video_grid: tuple[int, int, int] = (12, 48, 96)) -> np.ndarray:
+        """[T, 3] (t, h, w) ids for the three-axis RoPE variant: a modality
+        run whose length equals the video latent grid gets the grid's
+        (t, h, w) coordinates in token order (t-major); every other run gets
+        its one-axis ids repeated on the three axes."""
+        nt, nh, nw = video_grid
+        parts = []
+        for runs in self.pos_runs:
+            for n in runs:
+                if n == nt * nh * nw:
+                    t, h, w = np.meshgrid(np.arange(nt), np.arange(nh), np.arange(nw), indexing="ij")
+                    parts.append(np.stack([t.ravel(), h.ravel(), w.ravel()], 1))
+                else:
+                    a = np.arange(n)
+                    parts.append(np.stack([a, a, a], 1))
+        p = np.concatenate(parts).astype(np.int32) if parts else np.zeros((0, 3), np.int32)
+        assert p.shape[0] == self.T
+        return np.ascontiguousarray(p)
+
     def attn_flops(self) -> float:
         """4*H*D per valid (query, key) pair within a request."""
         return 4.0 * self.H * self.D * float(sum(int(L) * int(L) for L in self.seg_lens))
 
-    def prologue_bytes(self) -> int:
-        """qk_norm_rope: Q and K read + written (bf16) plus the int32 position."""
-        return self.T * (8 * self.H * self.D + 4)
+    def prologue_bytes(self, three_axis: bool = False) -> int:
+        """qk_norm_rope: Q and K read + written (bf16) plus the int32
+        position (three of them for the (t, h, w) variant)."""
+        return self.T * (8 * self.H * self.D + (12 if three_axis else 4))
 
     def epilogue_bytes(self, with_branch: bool = False) -> int:
         """modulate_swiglu: x (+branch, +x_out) in, h out; gate, up in; act out."""

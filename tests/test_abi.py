@@ -90,6 +90,25 @@ def test_qk_norm_rope_host_errors(L):
     assert qk(L, T=0, q_in=None) == 0              # empty: nothing to do
 
 
+def qk3(L, **kw):
+    a = dict(q_in=A, k_in=A, q_out=A, k_out=A, qs=1024, ks=1024, wq=A, wk=A, pos=A, st=16, sh=24, sw=24, T=16, H=8,
+             D=128, eps=1e-6, base=10000.0, style=0)
+    a.update(kw)
+    return L.pqk_qk_norm_rope_3axis(a["q_in"], a["k_in"], a["q_out"], a["k_out"], a["qs"], a["ks"], a["wq"],
+                                    a["wk"], a["pos"], a["st"], a["sh"], a["sw"], a["T"], a["H"], a["D"], a["eps"],
+                                    a["base"], a["style"], None)
+
+
+def test_qk_norm_rope_3axis_host_errors(L):
+    assert qk3(L, sw=23) == ERR_INVALID            # sections must cover D/2 pairs
+    assert qk3(L, st=-1, sh=41) == ERR_INVALID
+    assert qk3(L, D=64) == ERR_INVALID             # 16 + 24 + 24 != 32
+    assert qk3(L, D=96, st=16, sh=16, sw=16) == ERR_UNSUPPORTED
+    assert qk3(L, pos=None) == ERR_INVALID
+    assert qk3(L, q_out=U) == ERR_MISALIGNED
+    assert qk3(L, T=0, q_in=None) == 0
+
+
 def attn(L, **kw):
     a = dict(q=A, k=A, v=A, o=A, lse=None, qs=1024, ks=1024, vs=1024, os_=1024, cu=A, B=2, T=512, H=8, D=128,
              scale=0.088, ws=A, wsb=4096)

@@ -92,6 +92,59 @@ def test_qk_norm_rope_deterministic():
         assert torch.equal(k.view(torch.int16), outs[0][1].view(torch.int16))
 
 
+# ---------------------------------------------------------------- three-axis RoPE
+
+SECTIONS = {128: (16, 24, 24), 64: (8, 12, 12)}
+
+
+def prologue3_case(w, style, grid, rows=None):
+    torch = torch_cuda()
+    x = wl.prologue_inputs(w)
+    pos3 = w.positions3(grid)
+    q, k = to_dev_bf16(x["q"]), to_dev_bf16(x["k"])
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    sec = SECTIONS[w.D]
+    pqk.qk_norm_rope_3axis(q, k, to_dev_bf16(x["w_q"]), to_dev_bf16(x["w_k"]), to_dev(pos3), sec, eps=w.eps,
+                           rope_base=w.rope_base, style=style, q_out=qo, k_out=ko)
+    torch.cuda.synchronize()
+    sel = (lambda t: t) if rows is None else (lambda t: t[torch.from_numpy(rows).long().cuda()])
+    for name, out, wname in (("q", qo, "w_q"), ("k", ko, "w_k")):
+        ref = oracle.qk_norm_rope_3axis(x[name], x[wname], pos3, sec, w.eps, w.rope_base, style, rows=rows)
+        assert_elementwise(bf16_to_f64(sel(out)), ref, f"{w.name} {name} three-axis style {style}")
+
+
+@pytest.mark.parametrize("style", [pqk.ROPE_INTERLEAVED, pqk.ROPE_HALF])
+def test_qk_norm_rope_3axis_small_video_grids(style):
+    # a joint sequence whose video run is a 3 x 5 x 7 latent grid (D 128), and
+    # a D 64 one with a 2 x 4 x 6 grid
+    w = wl.Workload("text 9 + audio 4 + video 3x5x7", 60, [9 + 4 + 105], H=3, D=128, C=384, F=64,
+                    pos_runs=[[9, 4, 105]])
+    prologue3_case(w, style, (3, 5, 7))
+    w = wl.Workload("text 5 + video 2x4x6", 61, [5 + 48], H=2, D=64, C=128, F=64, pos_runs=[[5, 48]])
+    prologue3_case(w, style, (2, 4, 6))
+
+
+def test_qk_norm_rope_3axis_58048_tokens_sampled():
+    w = wl.config(3)
+    prologue3_case(w, pqk.ROPE_INTERLEAVED, (12, 48, 96), rows=wl.sample_rows(w, 1024))
+
+
+def test_qk_norm_rope_3axis_with_equal_ids_is_bitwise_the_one_axis_kernel():
+    torch = torch_cuda()
+    w = wl.config(2)
+    x = wl.prologue_inputs(w)
+    pos = x["pos"]
+    pos3 = np.ascontiguousarray(np.stack([pos, pos, pos], 1))
+    a = [to_dev_bf16(x["q"]), to_dev_bf16(x["k"])]
+    b = [to_dev_bf16(x["q"]), to_dev_bf16(x["k"])]
+    wq, wk = to_dev_bf16(x["w_q"]), to_dev_bf16(x["w_k"])
+    pqk.qk_norm_rope(a[0], a[1], wq, wk, to_dev(pos))
+    pqk.qk_norm_rope_3axis(b[0], b[1], wq, wk, to_dev(pos3), SECTIONS[w.D])
+    torch.cuda.synchronize()
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+    assert torch.equal(a[1].view(torch.int16), b[1].view(torch.int16))
+
+
 # ---------------------------------------------------------------- modulate_swiglu
 
 def epilogue_case(w, norm_type=pqk.NORM_RMS, with_branch=False, rows=None, fused_gate_up=False, swiglu=True):

@@ -15,7 +15,8 @@ import subprocess
 import pytest
 
 from oracle import oracle
-from tests import test_oracle_attention, test_oracle_modulate, test_oracle_norm_rope
+from tests import (test_oracle_attention, test_oracle_fullc, test_oracle_modulate, test_oracle_norm_rope,
+                   test_oracle_rope3)
 
 MUTANTS = {
     "attn_drop_scale": ("s[j] = scale * acc;", "s[j] = acc;"),
@@ -27,11 +28,15 @@ MUTANTS = {
                                  "const int64_t kb = (lo + j) * stride_t;"),
     "rope_sign": ("out[ia] = a * cos(phi) - b * sin(phi);", "out[ia] = a * cos(phi) + b * sin(phi);"),
     "rope_exponent": ("pow(base, -2.0 * (double)j / (double)D)", "pow(base, -1.0 * (double)j / (double)D)"),
-    "rope_pairing_swapped": ("if (style == ORACLE_ROPE_INTERLEAVED) { ia = 2 * j;",
-                             "if (style != ORACLE_ROPE_INTERLEAVED) { ia = 2 * j;"),
-    "norm_eps_outside_sqrt": ("const double inv = 1.0 / sqrt(ms + eps);", "const double inv = 1.0 / (sqrt(ms) + eps);"),
+    "rope_pairing_swapped": ("if (style == ORACLE_ROPE_INTERLEAVED) { *ia = 2 * j;",
+                             "if (style != ORACLE_ROPE_INTERLEAVED) { *ia = 2 * j;"),
+    "norm_eps_outside_sqrt": ("ms /= (double)D;\n  const double inv = 1.0 / sqrt(ms + eps);",
+                              "ms /= (double)D;\n  const double inv = 1.0 / (sqrt(ms) + eps);"),
+    "fullc_eps_outside_sqrt": ("ms /= (double)width;\n    const double inv = 1.0 / sqrt(ms + eps);",
+                               "ms /= (double)width;\n    const double inv = 1.0 / (sqrt(ms) + eps);"),
     "norm_sum_not_mean": ("ms /= (double)D;", "ms /= 1.0;"),
-    "norm_drop_weight": ("* inv * load(w, w_kind, d);", "* inv;"),
+    "norm_drop_weight": ("n[d] = load(x, x_kind, row + d) * inv * load(w, w_kind, d);",
+                         "n[d] = load(x, x_kind, row + d) * inv;"),
     "mod_scale_not_offset": ("n * (1.0 + (double)scale[", "n * (0.0 + (double)scale["),
     "mod_shift_of_first_request": ("+ (double)shift[(int64_t)seg * C + c];", "+ (double)shift[c];"),
     "mod_residual_sign": ("if (branch) xv += ", "if (branch) xv -= "),
@@ -40,11 +45,17 @@ MUTANTS = {
     "silu_operands_swapped": ("act_out[r * (int64_t)F + f] = g / (1.0 + exp(-g)) * u;",
                               "act_out[r * (int64_t)F + f] = u / (1.0 + exp(-u)) * g;"),
     "silu_sign": ("g / (1.0 + exp(-g)) * u", "g / (1.0 + exp(g)) * u"),
+    "rope3_axis_boundary": ("const int axis = j < sec[0] ? 0 :", "const int axis = j <= sec[0] ? 0 :"),
+    "rope3_axes_swapped": ("(j < sec[0] + sec[1] ? 1 : 2)", "(j < sec[0] + sec[1] ? 2 : 1)"),
+    "rope3_ids_of_first_token": ("(double)pos3[t * 3 + axis]", "(double)pos3[axis]"),
+    "fullc_mean_over_one_head": ("ms /= (double)width;", "ms /= (double)D;"),
+    "fullc_weight_of_first_head": ("* inv * load(w, w_kind, (int64_t)h * D + d);", "* inv * load(w, w_kind, d);"),
 }
 
 
 def _pin_calls():
-    for mod in (test_oracle_attention, test_oracle_norm_rope, test_oracle_modulate):
+    for mod in (test_oracle_attention, test_oracle_norm_rope, test_oracle_modulate, test_oracle_rope3,
+                test_oracle_fullc):
         for name, fn in inspect.getmembers(mod, inspect.isfunction):
             if not name.startswith("test_") or fn.__module__ != mod.__name__:
                 continue
