@@ -345,6 +345,21 @@ def run_ours(args, w):
     ev3[1].record()
     torch.cuda.synchronize()
     rope1_b2b_us = ev3[0].elapsed_time(ev3[1]) / reps3 * 1e3
+    # the full-width Q/K norm variant (weights of H*D entries), same way
+    from packed_attention_qk_b200 import workloads as wl
+    fw = wl.fullc_weights(w)
+    fwq = torch.from_numpy(fw["w_q"].view(np.int16)).view(torch.bfloat16).to(dev)
+    fwk = torch.from_numpy(fw["w_k"].view(np.int16)).view(torch.bfloat16).to(dev)
+    pqk.qk_fullc_norm_rope(d["q"], d["k"], fwq, fwk, d["pos"], eps=w.eps, rope_base=w.rope_base, q_out=o["qn"],
+                           k_out=o["kn"])
+    ev3[0].record()
+    for _ in range(reps3):
+        pqk.qk_fullc_norm_rope(d["q"], d["k"], fwq, fwk, d["pos"], eps=w.eps, rope_base=w.rope_base,
+                               q_out=o["qn"], k_out=o["kn"])
+    ev3[1].record()
+    torch.cuda.synchronize()
+    fullc_us = ev3[0].elapsed_time(ev3[1]) / reps3 * 1e3
+    fullc_gbs = (w.prologue_bytes() + 2 * w.H * w.D * 2) / (fullc_us * 1e-6) / 1e9
 
     # e2e through host buffers: pinned H2D of every input, the three calls,
     # D2H of the block outputs (x', h, act), all inside the timed region
@@ -406,7 +421,9 @@ def run_ours(args, w):
                     "qk_norm_rope_3axis_us": rope3_us, "qk_norm_rope_3axis_gbs": rope3_gbs,
                     "qk_norm_rope_3axis_frac_hbm": rope3_gbs / pk["hbm_gbs"],
                     "qk_norm_rope_3axis_sections": list(sections),
-                    "qk_norm_rope_back_to_back_us": rope1_b2b_us},
+                    "qk_norm_rope_back_to_back_us": rope1_b2b_us,
+                    "qk_fullc_norm_rope_us": fullc_us, "qk_fullc_norm_rope_gbs": fullc_gbs,
+                    "qk_fullc_norm_rope_frac_hbm": fullc_gbs / pk["hbm_gbs"]},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * K,

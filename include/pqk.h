@@ -117,6 +117,24 @@ PQK_API int pqk_qk_norm_rope_3axis(const void* q_in, const void* k_in, void* q_o
                            int rope_style, void* stream);
 
 /*
+ * pqk_qk_fullc_norm_rope -- pqk_qk_norm_rope with the RMS taken over all H*D
+ * elements of a token's Q (and, separately, K) row instead of per head, and
+ * one weight per element; then every head is rotated as in
+ * pqk_qk_norm_rope. A reading of "Q/K normalisation merged with RoPE" (first
+ * page, section "融合 DiT 算子") that the pages leave open, next to the
+ * per-head default:
+ *   y_{h,d} = x_{h,d} / sqrt(mean over the token's H*D elements of x^2 + eps)
+ *             * w_X[h*D + d].
+ *
+ * q_weight, k_weight  device bf16 [H*D]. Other arguments, layouts and errors
+ * as in pqk_qk_norm_rope.
+ */
+PQK_API int pqk_qk_fullc_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                           int64_t q_stride_t, int64_t k_stride_t, const void* q_weight,
+                           const void* k_weight, const int32_t* pos, int64_t T, int H, int D,
+                           float eps, float rope_base, int rope_style, void* stream);
+
+/*
  * pqk_varlen_attn_workspace_size -- bytes of device workspace that
  * pqk_varlen_attn_fwd needs for B requests (its tile schedule).
  */

@@ -15,6 +15,10 @@
 // ~1e-2 rad) and only the reduced angle goes through the fp32 sine/cosine.
 // The three-axis variant (video latents with (t, h, w) ids) keeps the same
 // frequencies and takes each pair's position from the axis of its section.
+// The full-width variant normalises over all H*D elements of a token's Q (or
+// K) with one weight per element: a first pass of the warp over the token's
+// rows sums the squares (full-warp reduction), the second pass re-reads the
+// rows (now in cache), normalises, rotates and stores.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -74,7 +78,7 @@ __device__ __forceinline__ void rope_sincos(int32_t pos, double theta, float& c,
   __sincosf(r, &s, &c);  // |r| <= pi: absolute error ~4e-7
 }
 
-template <int D, bool kThreeAxis>
+template <int D, bool kThreeAxis, bool kFullWidth>
 __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParams p) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerStep = 32 / kLanesPerRow;
@@ -100,8 +104,9 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
     const int j = j0 + i;
     axis[i] = kThreeAxis ? (j < p.sec0 ? 0 : (j < p.sec0 + p.sec1 ? 1 : 2)) : 0;
   }
-  const uint4 wq_raw = *reinterpret_cast<const uint4*>(p.wq + chunk * 8);
-  const uint4 wk_raw = *reinterpret_cast<const uint4*>(p.wk + chunk * 8);
+  // per-head weights ([D], shared by all heads) stay in registers
+  const uint4 wq_raw = kFullWidth ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(p.wq + chunk * 8);
+  const uint4 wk_raw = kFullWidth ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(p.wk + chunk * 8);
   const int rows = 2 * p.H;
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + threadIdx.x / 32; t < p.T;
@@ -124,6 +129,43 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
       for (int i = 0; i < 8; ++i)
         rope_sincos(kThreeAxis ? pos3[axis[i]] : pos3[0], theta[j0 + i], cs[i], sn[i]);
     }
+    // full width: the RMS of every Q (and K) element of the token, from a
+    // first pass over its rows and a reduction over the whole warp
+    float inv_q = 0.f, inv_k = 0.f;
+    if constexpr (kFullWidth) {
+      float ssq_q = 0.f, ssq_k = 0.f;
+      for (int r0 = 0; r0 < rows; r0 += kRowsPerStep * kUnroll) {
+        uint4 raw[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int r = r0 + u * kRowsPerStep + sub;
+          raw[u] = make_uint4(0, 0, 0, 0);
+          if (r < rows) {
+            const bool is_q = r < p.H;
+            const __nv_bfloat16* src = is_q ? p.q_in + t * p.q_stride : p.k_in + t * p.k_stride;
+            raw[u] = *reinterpret_cast<const uint4*>(src + (is_q ? r : r - p.H) * D + chunk * 8);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int r = r0 + u * kRowsPerStep + sub;
+          float x[8];
+          unpack8(raw[u], x);
+          float ss = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+          if (r < p.H) ssq_q += ss; else ssq_k += ss;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        ssq_q += __shfl_xor_sync(0xffffffffu, ssq_q, off);
+        ssq_k += __shfl_xor_sync(0xffffffffu, ssq_k, off);
+      }
+      const float inv_width = 1.0f / static_cast<float>(p.H * D);
+      inv_q = rsqrtf(ssq_q * inv_width + p.eps);
+      inv_k = rsqrtf(ssq_k * inv_width + p.eps);
+    }
     for (int r0 = 0; r0 < rows; r0 += kRowsPerStep * kUnroll) {
       uint4 raw[kUnroll];
       bool live[kUnroll];
@@ -145,14 +187,24 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
         const bool is_q = r < p.H;
         float x[8];
         unpack8(raw[u], x);
-        float ss = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
-#pragma unroll
-        for (int off = kHalfLanes; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float inv = rsqrtf(ss * (1.0f / D) + p.eps);
+        float inv;
         float wv[8], y[8];
-        unpack8(is_q ? wq_raw : wk_raw, wv);
+        if constexpr (kFullWidth) {
+          inv = is_q ? inv_q : inv_k;
+          // one weight per element of the token's H*D row
+          const int h = is_q ? r : r - p.H;
+          uint4 wraw = make_uint4(0, 0, 0, 0);
+          if (live[u]) wraw = __ldg(reinterpret_cast<const uint4*>((is_q ? p.wq : p.wk) + h * D + chunk * 8));
+          unpack8(wraw, wv);
+        } else {
+          float ss = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+          for (int off = kHalfLanes; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          inv = rsqrtf(ss * (1.0f / D) + p.eps);
+          unpack8(is_q ? wq_raw : wk_raw, wv);
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = x[i] * inv * wv[i];
         float o[8];
@@ -185,8 +237,8 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
 
 int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride,
                         int64_t k_stride, const void* wq, const void* wk, const int32_t* pos, const int* sections,
-                        int64_t T, int H, int D, float eps, float rope_base, int style, cudaStream_t stream,
-                        int num_sms) {
+                        bool full_width, int64_t T, int H, int D, float eps, float rope_base, int style,
+                        cudaStream_t stream, int num_sms) {
   QkParams p;
   p.q_in = static_cast<const __nv_bfloat16*>(q_in);
   p.k_in = static_cast<const __nv_bfloat16*>(k_in);
@@ -209,14 +261,21 @@ int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k
   const int64_t cap = static_cast<int64_t>(num_sms) * 3;
   const int grid = static_cast<int>(want < cap ? want : cap);
   const bool three = sections != nullptr;
-  if (D == 128 && !three)
-    qk_norm_rope_kernel<128, false><<<grid, kThreads, 0, stream>>>(p);
-  else if (D == 128)
-    qk_norm_rope_kernel<128, true><<<grid, kThreads, 0, stream>>>(p);
-  else if (!three)
-    qk_norm_rope_kernel<64, false><<<grid, kThreads, 0, stream>>>(p);
-  else
-    qk_norm_rope_kernel<64, true><<<grid, kThreads, 0, stream>>>(p);
+  if (D == 128) {
+    if (full_width)
+      qk_norm_rope_kernel<128, false, true><<<grid, kThreads, 0, stream>>>(p);
+    else if (three)
+      qk_norm_rope_kernel<128, true, false><<<grid, kThreads, 0, stream>>>(p);
+    else
+      qk_norm_rope_kernel<128, false, false><<<grid, kThreads, 0, stream>>>(p);
+  } else {
+    if (full_width)
+      qk_norm_rope_kernel<64, false, true><<<grid, kThreads, 0, stream>>>(p);
+    else if (three)
+      qk_norm_rope_kernel<64, true, false><<<grid, kThreads, 0, stream>>>(p);
+    else
+      qk_norm_rope_kernel<64, false, false><<<grid, kThreads, 0, stream>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -21,7 +21,7 @@ ROPE_INTERLEAVED, ROPE_HALF = 0, 1
 NORM_RMS, NORM_LAYER, NORM_NONE = 0, 1, 2
 
 # every symbol include/pqk.h declares
-EXPORTS = ("pqk_qk_norm_rope", "pqk_qk_norm_rope_3axis", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd",
+EXPORTS = ("pqk_qk_norm_rope", "pqk_qk_norm_rope_3axis", "pqk_qk_fullc_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd",
            "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu",
            "pqk_get_device_status", "pqk_set_wait_timeout_ns", "pqk_selftest_wait_timeout", "pqk_status_string",
            "pqk_version")
@@ -52,6 +52,8 @@ def lib(path: str | None = None) -> C.CDLL:
     L.pqk_qk_norm_rope_3axis.argtypes = [vp, vp, vp, vp, i64, i64, vp, vp, vp, i32, i32, i32, i64, i32, i32, f32, f32,
                                          i32, vp]
     L.pqk_qk_norm_rope_3axis.restype = i32
+    L.pqk_qk_fullc_norm_rope.argtypes = [vp, vp, vp, vp, i64, i64, vp, vp, vp, i64, i32, i32, f32, f32, i32, vp]
+    L.pqk_qk_fullc_norm_rope.restype = i32
     L.pqk_varlen_attn_workspace_size.argtypes = [i32]
     L.pqk_varlen_attn_workspace_size.restype = sz
     L.pqk_varlen_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32, vp, sz,
@@ -138,6 +140,21 @@ def qk_norm_rope_3axis(q, k, w_q, w_k, pos3, sections, *, eps: float = 1e-6, rop
     _check("pqk_qk_norm_rope_3axis", lib().pqk_qk_norm_rope_3axis(
         _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), qs, ks, _ptr(w_q), _ptr(w_k), _ptr(pos3), st, sh, sw, T, H, D,
         eps, rope_base, style, _stream(stream)))
+    return q_out, k_out
+
+
+def qk_fullc_norm_rope(q, k, w_q, w_k, pos, *, eps: float = 1e-6, rope_base: float = 10000.0,
+                       style: int = ROPE_INTERLEAVED, q_out=None, k_out=None, stream=None):
+    """Fused Q/K RMSNorm over all H*D elements of a token (weights [H*D]) +
+    RoPE per head."""
+    q_out = q if q_out is None else q_out
+    k_out = k if k_out is None else k_out
+    T, H, D = q.shape
+    qs, ks = _token_stride(q, 3), _token_stride(k, 3)
+    assert _token_stride(q_out, 3) == qs and _token_stride(k_out, 3) == ks
+    _check("pqk_qk_fullc_norm_rope", lib().pqk_qk_fullc_norm_rope(
+        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), qs, ks, _ptr(w_q), _ptr(w_k), _ptr(pos), T, H, D, eps,
+        rope_base, style, _stream(stream)))
     return q_out, k_out
 
 

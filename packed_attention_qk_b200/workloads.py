@@ -39,7 +39,7 @@ CHUNK = 1 << 22
 TENSOR_ID = {
     "q": 1, "k": 2, "v": 3, "x": 4, "branch": 5, "gate": 6, "up": 7,
     "w_q": 8, "w_k": 9, "shift": 10, "scale": 11, "gate_res": 12,
-    "outlier": 13, "sample_rows": 14,
+    "outlier": 13, "sample_rows": 14, "w_q_full": 15, "w_k_full": 16,
 }
 
 
@@ -271,6 +271,11 @@ def prologue_inputs(w: Workload) -> dict[str, np.ndarray]:
     return {"q": bf16_normal(w.seed, "q", shp), "k": bf16_normal(w.seed, "k", shp),
             "w_q": bf16_weight(w.seed, "w_q", w.D), "w_k": bf16_weight(w.seed, "w_k", w.D),
             "pos": w.positions()}
+
+
+def fullc_weights(w: Workload) -> dict[str, np.ndarray]:
+    """Weights of the full-width Q/K norm: one per element of the H*D row."""
+    return {"w_q": bf16_weight(w.seed, "w_q_full", w.H * w.D), "w_k": bf16_weight(w.seed, "w_k_full", w.H * w.D)}
 
 
 def epilogue_inputs(w: Workload, with_branch: bool = False) -> dict[str, np.ndarray]:

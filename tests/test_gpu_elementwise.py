@@ -145,6 +145,49 @@ def test_qk_norm_rope_3axis_with_equal_ids_is_bitwise_the_one_axis_kernel():
     assert torch.equal(a[1].view(torch.int16), b[1].view(torch.int16))
 
 
+# ---------------------------------------------------------------- full-width Q/K norm
+
+def fullc_case(w, style, rows=None):
+    torch = torch_cuda()
+    x = wl.prologue_inputs(w)
+    fw = wl.fullc_weights(w)
+    q, k = to_dev_bf16(x["q"]), to_dev_bf16(x["k"])
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    pqk.qk_fullc_norm_rope(q, k, to_dev_bf16(fw["w_q"]), to_dev_bf16(fw["w_k"]), to_dev(x["pos"]), eps=w.eps,
+                           rope_base=w.rope_base, style=style, q_out=qo, k_out=ko)
+    torch.cuda.synchronize()
+    sel = (lambda t: t) if rows is None else (lambda t: t[torch.from_numpy(rows).long().cuda()])
+    for name, out, wname in (("q", qo, "w_q"), ("k", ko, "w_k")):
+        ref = oracle.qk_fullc_norm_rope(x[name], fw[wname], x["pos"], w.eps, w.rope_base, style, rows=rows)
+        assert_elementwise(bf16_to_f64(sel(out)), ref, f"{w.name} {name} full width style {style}")
+
+
+@pytest.mark.parametrize("style", [pqk.ROPE_INTERLEAVED, pqk.ROPE_HALF])
+def test_qk_fullc_norm_rope_small(style):
+    fullc_case(wl.config(1), style)
+    fullc_case(wl.custom([37, 0, 90], H=5, D=128, seed=62), style)
+    fullc_case(wl.custom([50], H=3, D=64, seed=63), style)
+
+
+def test_qk_fullc_norm_rope_58048_tokens_sampled():
+    w = wl.config(3)
+    fullc_case(w, pqk.ROPE_INTERLEAVED, rows=wl.sample_rows(w, 512))
+
+
+def test_qk_fullc_norm_rope_one_head_is_bitwise_the_per_head_kernel():
+    torch = torch_cuda()
+    w = wl.custom([300], H=1, D=128, seed=64)
+    x = wl.prologue_inputs(w)
+    a = [to_dev_bf16(x["q"]), to_dev_bf16(x["k"])]
+    b = [to_dev_bf16(x["q"]), to_dev_bf16(x["k"])]
+    wq, wk, pos = to_dev_bf16(x["w_q"]), to_dev_bf16(x["w_k"]), to_dev(x["pos"])
+    pqk.qk_norm_rope(a[0], a[1], wq, wk, pos)
+    pqk.qk_fullc_norm_rope(b[0], b[1], wq, wk, pos)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+    assert torch.equal(a[1].view(torch.int16), b[1].view(torch.int16))
+
+
 # ---------------------------------------------------------------- modulate_swiglu
 
 def epilogue_case(w, norm_type=pqk.NORM_RMS, with_branch=False, rows=None, fused_gate_up=False, swiglu=True):
