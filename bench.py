@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--config", type=int, default=3, help="workload number (3 = 58,048-token joint sequence)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="one request of this many tokens with the shape of --config (a smaller case for profiling)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="prologue/epilogue bandwidth sweep (40 heads x 128; hidden 5,120, FFN 13,824) instead "
+                         "of the step; one JSON line per kernel and token count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -361,37 +364,73 @@ def run_ours(args, w):
     fullc_us = ev3[0].elapsed_time(ev3[1]) / reps3 * 1e3
     fullc_gbs = (w.prologue_bytes() + 2 * w.H * w.D * 2) / (fullc_us * 1e-6) / 1e9
 
-    # e2e through host buffers: pinned H2D of every input, the three calls,
-    # D2H of the block outputs (x', h, act), all inside the timed region
+    # e2e through host buffers: every step copies all of its inputs from
+    # pinned host memory to the device (H2D stream), runs the three C-ABI
+    # calls (compute stream) and copies its outputs x', h, act back to pinned
+    # host memory (D2H stream), all inside the timed region. Two device buffer
+    # sets let step i+1's uploads and step i-1's downloads overlap step i's
+    # kernels, as a serving loop would; events order each buffer set's reuse.
     e2e = None
     if not args.no_e2e:
-        host_in = {k: d[k].cpu().pin_memory() for k in ("q", "k", "v", "x", "gate", "up", "w_q", "w_k", "pos", "cu",
-                                                          "shift", "scale", "gate_res")}
-        host_out = {k: torch.empty(o[k].shape, dtype=o[k].dtype, pin_memory=True) for k in ("x_out", "h", "act")}
+        in_keys = ("q", "k", "v", "x", "gate", "up", "w_q", "w_k", "pos", "cu", "shift", "scale", "gate_res")
+        out_keys = ("x_out", "h", "act")
+        host_in = {k: d[k].cpu().pin_memory() for k in in_keys}
+        host_out = [{k: torch.empty(o[k].shape, dtype=o[k].dtype, pin_memory=True) for k in out_keys}
+                    for _ in range(2)]
+        sets = [(d, o), ({k: torch.empty_like(d[k]) for k in in_keys}, alloc_outputs(w, d))]
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-        e2e_steps = max(2, min(K, 5))
+        d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
+        s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        e2e_steps = max(4, min(K, 8))
 
-        def e2e_step():
-            for k, t in host_in.items():
-                d[k].copy_(t, non_blocking=True)
-            block_call(w, d, o)
-            for k, t in host_out.items():
-                t.copy_(o[k], non_blocking=True)
+        def run_e2e(n):
+            ev_in = [None, None]     # inputs of set b uploaded
+            ev_done = [None, None]   # kernels of set b finished
+            ev_out = [None, None]    # outputs of set b downloaded
+            for i in range(n):
+                b = i % 2
+                dd, oo = sets[b]
+                with torch.cuda.stream(s_in):
+                    if ev_done[b] is not None:
+                        s_in.wait_event(ev_done[b])      # set b's previous kernels have read their inputs
+                    for k in in_keys:
+                        dd[k].copy_(host_in[k], non_blocking=True)
+                    ev_in[b] = torch.cuda.Event()
+                    ev_in[b].record(s_in)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(ev_in[b])
+                    if ev_out[b] is not None:
+                        s_cmp.wait_event(ev_out[b])      # set b's previous outputs are on the host
+                    block_call(w, dd, oo)
+                    ev_done[b] = torch.cuda.Event()
+                    ev_done[b].record(s_cmp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_done[b])
+                    for k in out_keys:
+                        host_out[b][k].copy_(oo[k], non_blocking=True)
+                    ev_out[b] = torch.cuda.Event()
+                    ev_out[b].record(s_out)
 
-        e2e_step()
+        run_e2e(2)
         torch.cuda.synchronize()
         barrier()
         s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s2.record()
-        for _ in range(e2e_steps):
-            e2e_step()
-        t2.record()
+        s2.record(torch.cuda.current_stream())
+        for st in (s_in, s_cmp, s_out):
+            st.wait_stream(torch.cuda.current_stream())
+        run_e2e(e2e_steps)
+        for st in (s_in, s_cmp, s_out):
+            torch.cuda.current_stream().wait_stream(st)
+        t2.record(torch.cuda.current_stream())
         torch.cuda.synchronize()
         barrier()
+        if pqk.get_device_status() != 0:
+            raise RuntimeError("device status set during the end-to-end steps")
         e2e_ms = max_over_ranks(s2.elapsed_time(t2)) / e2e_steps
         e2e = {"value": throughput(flops, world, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "overlap": "two buffer sets: uploads and downloads overlap neighbouring steps' kernels"}
+        del sets
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -435,9 +474,66 @@ def run_ours(args, w):
         dist.destroy_process_group()
 
 
+def run_sweep(args):
+    """The HBM-bound kernels alone on the sweep shapes, one launch at a time
+    with a 256 MB L2 flush in between (the 4,096-token working set is close
+    to the 126 MB L2), median of the timed launches."""
+    import torch
+    from packed_attention_qk_b200 import pqk
+    from packed_attention_qk_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    pk, pk_kind = peaks()
+
+    def dev16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    def timed(fn, reps):
+        ts = []
+        for i in range(args.warmup + reps):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    for T in wl.C5_TOKENS:
+        w = wl.config(5, T)
+        p = wl.prologue_inputs(w)
+        q, k, wq, wk = dev16(p["q"]), dev16(p["k"]), dev16(p["w_q"]), dev16(p["w_k"])
+        pos = torch.from_numpy(p["pos"]).to(dev)
+        qo, ko = torch.empty_like(q), torch.empty_like(k)
+        ms = timed(lambda: pqk.qk_norm_rope(q, k, wq, wk, pos, eps=w.eps, q_out=qo, k_out=ko), args.steps)
+        gbs = w.prologue_bytes() / (ms * 1e-3) / 1e9
+        print(json.dumps({"sweep": "qk_norm_rope", "tokens": T, "heads": w.H, "head_dim": w.D, "us": ms * 1e3,
+                          "gbs": gbs, "frac_hbm": gbs / pk["hbm_gbs"], "peak_gbs": pk["hbm_gbs"],
+                          "peak_kind": pk_kind, "bytes": w.prologue_bytes()}), flush=True)
+        del q, k, qo, ko
+        e = wl.epilogue_inputs(w)
+        x, gate, up = dev16(e["x"]), dev16(e["gate"]), dev16(e["up"])
+        shift, scale = torch.from_numpy(e["shift"]).to(dev), torch.from_numpy(e["scale"]).to(dev)
+        cu = torch.from_numpy(e["cu_seqlens"]).to(dev)
+        h, act = torch.empty_like(x), torch.empty_like(gate)
+        ms = timed(lambda: pqk.modulate_swiglu(x, shift, scale, cu, gate=gate, up=up, eps=w.eps, h=h, act=act),
+                   args.steps)
+        gbs = w.epilogue_bytes() / (ms * 1e-3) / 1e9
+        print(json.dumps({"sweep": "modulate_swiglu", "tokens": T, "hidden": w.C, "ffn": w.F, "us": ms * 1e3,
+                          "gbs": gbs, "frac_hbm": gbs / pk["hbm_gbs"], "peak_gbs": pk["hbm_gbs"],
+                          "peak_kind": pk_kind, "bytes": w.epilogue_bytes()}), flush=True)
+        del x, gate, up, h, act
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
     from packed_attention_qk_b200 import workloads as wl
+    if args.sweep:
+        run_sweep(args)
+        return
     w = wl.config(args.config)
     if args.tokens:
         w = wl.Workload(f"one request of {args.tokens} tokens, {w.H} heads x {w.D}, hidden {w.C}, ffn {w.F}", w.seed,
