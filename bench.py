@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="prologue/epilogue bandwidth sweep (40 heads x 128; hidden 5,120, FFN 13,824) instead "
                          "of the step; one JSON line per kernel and token count")
+    ap.add_argument("--outliers", action="store_true",
+                    help="K with 0.1%% of its entries scaled x20 (the outlier variant of the 4-request batch)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -140,7 +142,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ inputs
 
-def make_inputs(w, device):
+def make_inputs(w, device, outliers=False):
     import torch
     from packed_attention_qk_b200 import workloads as wl
 
@@ -148,6 +150,8 @@ def make_inputs(w, device):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
 
     p = wl.prologue_inputs(w)
+    if outliers:
+        p["k"] = wl.bf16_k_with_outliers(w.seed, (w.T, w.H, w.D))
     a = {"v": wl.bf16_normal(w.seed, "v", (w.T, w.H, w.D))}
     e = wl.epilogue_inputs(w, with_branch=False)
     d = {"q": dev16(p["q"]), "k": dev16(p["k"]), "v": dev16(a["v"]), "w_q": dev16(p["w_q"]),
@@ -286,7 +290,7 @@ def run_ours(args, w):
     ranks = Ranks(world, dev)
     barrier, max_over_ranks = ranks.barrier, ranks.max
 
-    d = make_inputs(w, dev)
+    d = make_inputs(w, dev, outliers=args.outliers)
     o = alloc_outputs(w, d)
     torch.cuda.synchronize()
     for _ in range(args.warmup):
@@ -445,7 +449,8 @@ def run_ours(args, w):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "tokens_per_gpu": w.T, "requests_per_gpu": w.B, "heads": w.H,
+        "config": {"workload": w.name + (" (K outliers)" if args.outliers else ""), "tokens_per_gpu": w.T,
+                   "requests_per_gpu": w.B, "heads": w.H,
                    "head_dim": w.D, "hidden": w.C, "ffn": w.F,
                    "l2": "inputs larger than L2 (Q, K, V 357 MB each; prologue 1.43 GB; epilogue 4.3 GB)"},
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",

@@ -69,6 +69,18 @@ def test_many_requests():
     check(x, w.H, w.D, what="60 requests")
 
 
+@pytest.mark.parametrize("n_req", [3000, 9000])
+def test_thousands_of_short_requests(n_req):
+    # above 8,192 requests the schedule keeps the given order instead of
+    # longest first; both must give every row its own request's attention
+    g = np.random.default_rng(n_req)
+    lens = [int(v) for v in g.integers(0, 40, n_req)]
+    lens[n_req // 2] = 300
+    w, x = custom_inputs(lens, 2, 64, seed=n_req)
+    rows = np.sort(g.choice(w.T, size=512, replace=False)).astype(np.int32)
+    check(x, w.H, w.D, rows=rows, what=f"{n_req} requests")
+
+
 @pytest.mark.parametrize("D", [64, 128])
 def test_peaked_scores(D):
     # Q x 8: the softmax concentrates on a few keys, O is close to single V rows
