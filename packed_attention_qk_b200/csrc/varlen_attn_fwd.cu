@@ -233,16 +233,17 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, int valid, float (&s
 
 __device__ __forceinline__ float row_max(const float (&s)[128]) {
   if constexpr (kPacked) {
-    // four chains of three-input maxima over 2 new columns each
-    float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+    // eight independent chains of three-input maxima (two new columns each),
+    // then a three-level tree
+    float m[8];
 #pragma unroll
-    for (int c = 4; c < 128; c += 8) {
-      m0 = max3(m0, s[c], s[c + 1]);
-      m1 = max3(m1, s[c + 2], s[c + 3]);
-      m2 = max3(m2, s[c + 4], s[c + 5]);
-      m3 = max3(m3, s[c + 6], s[c + 7]);
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(s[i], s[i + 8]);
+#pragma unroll
+    for (int c = 16; c < 128; c += 16) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = max3(m[i], s[c + i], s[c + 8 + i]);
     }
-    return max3(m0, m1, fmaxf(m2, m3));
+    return fmaxf(max3(m[0], m[1], m[2]), max3(m[3], m[4], fmaxf(m[5], fmaxf(m[6], m[7]))));
   } else {
     float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
@@ -450,16 +451,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < wk.n_kv; ++j) {
           const uint32_t v_idx = cons_idx++;
           const bool more = j + 1 < wk.n_kv;
+          const uint32_t nk_idx = more ? cons_idx++ : 0;
+          // V_j and K_{j+1} are waited for here, while P0 is still being
+          // computed, not between O0 += P0 V_j and S0 = Q0 K_{j+1}^T
           if (!(ok = wait_stage(v_idx))) break;
+          if (more && !(ok = wait_stage(nk_idx))) break;
           if (!(ok = mbar_wait(p_full(0), p_phase, abort_flag, p.timeout_ns))) break;
           tc_fence_after_sync();
           issue_pv(0, v_idx % L::kStages, j > 0);
           if (!more) tc_commit(o_done(0));
-          uint32_t nk_idx = 0;
           if (more) {
-            nk_idx = cons_idx++;
-            if (!(ok = wait_stage(nk_idx))) break;
-            tc_fence_after_sync();
             issue_qk(0, nk_idx % L::kStages);
             tc_commit(s_full(0));
           }
