@@ -409,27 +409,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t p_phase = 0;
       int wt = 0;
       bool ok = true;
+      // Descriptor low words of Q0 and of stage 0 (K: K-major, V: MN-major
+      // with 64-wide column slabs kSlabBytes apart); one high word for all.
+      constexpr uint32_t kDescHi = smem_desc_hi_sw128(1024);
+      constexpr uint32_t kTileWords = L::kTileBytes >> 4;
+      const uint32_t q_lo = smem_desc_lo(q_smem, 16);
+      const uint32_t k_lo = smem_desc_lo(kv_smem, 16);
+      const uint32_t v_lo = smem_desc_lo(kv_smem, kSlabBytes);
       // S_i = Q_i K^T over D/16 K-steps of 16 (32 bytes inside the 128-byte row)
       auto issue_qk = [&](int i, int stage) {
-        const uint32_t qa = q_smem + i * L::kTileBytes;
-        const uint32_t kb = kv_smem + stage * L::kTileBytes;
+        const uint32_t a0 = q_lo + i * kTileWords;
+        const uint32_t b0 = k_lo + stage * kTileWords;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k / 4) * kSlabBytes + (k % 4) * 32;
-          mma_bf16_ss(tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1), smem_desc_sw128(qa + off, 16, 1024),
-                      smem_desc_sw128(kb + off, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+          const uint32_t off = ((k / 4) * kSlabBytes + (k % 4) * 32) >> 4;
+          mma_bf16_ss_w(tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1), a0 + off, b0 + off, kDescHi, kIdescQK,
+                        k > 0 ? 1u : 0u);
         }
       };
       // O_i (+)= P_i V over kBN/16 K-steps; V is MN-major: 64-wide column
       // slabs kSlabBytes apart, 8-row groups 1024 bytes apart
       auto issue_pv = [&](int i, int stage, bool accumulate) {
-        const uint32_t vb = kv_smem + stage * L::kTileBytes;
+        const uint32_t b0 = v_lo + stage * kTileWords;
         const uint32_t p_col = tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1);
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k) {
-          mma_bf16_ts(tmem + (i == 0 ? L::kTmemO0 : L::kTmemO1), p_col + 8 * k,
-                      smem_desc_sw128(vb + k * 2048, kSlabBytes, 1024), kIdescPV,
-                      (accumulate || k > 0) ? 1u : 0u);
+          mma_bf16_ts_w(tmem + (i == 0 ? L::kTmemO0 : L::kTmemO1), p_col + 8 * k, b0 + ((k * 2048) >> 4), kDescHi,
+                        kIdescPV, (accumulate || k > 0) ? 1u : 0u);
         }
       };
       auto wait_stage = [&](uint32_t idx) {
