@@ -52,8 +52,11 @@ def load(path: str):
                                             C.c_int, C.c_double, C.c_double, C.c_int, i32p, C.c_int64, f64p]
     L.oracle_qk_fullc_norm_rope.argtypes = [vp, C.c_int, C.c_int64, vp, C.c_int, i32p, C.c_int64, C.c_int, C.c_int,
                                             C.c_double, C.c_double, C.c_int, i32p, C.c_int64, f64p]
+    L.oracle_varlen_attn_skip.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
+                                          C.c_int, C.c_double, C.c_double, i32p, C.c_int64, f64p, f64p,
+                                          C.POINTER(C.c_int64)]
     for f in (L.oracle_qk_norm_rope, L.oracle_qk_norm_rope_3axis, L.oracle_qk_fullc_norm_rope, L.oracle_varlen_attn,
-              L.oracle_modulate_swiglu):
+              L.oracle_varlen_attn_skip, L.oracle_modulate_swiglu):
         f.restype = C.c_int
     L.oracle_num_threads.restype = C.c_int
     return L
@@ -169,6 +172,30 @@ def varlen_attn(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndar
     if rc:
         raise ValueError("oracle_varlen_attn: invalid arguments")
     return o, lse
+
+
+def varlen_attn_skip(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, tau: float,
+                     rows=None, want_lse: bool = True):
+    """Attention with key blocks skipped where negligible (oracle_varlen_attn_skip).
+    Returns (o [nrows, H, D], lse [nrows, H] or None, counts): counts is
+    (skipped 32-row blocks, skipped 128-row tiles) over all (block, head, key
+    block) triples when rows is None, else None."""
+    T, H, D = q.shape
+    assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
+    q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    r, n = _rows(rows)
+    n = n if r is not None else T
+    o = np.empty((n, H, D), np.float64)
+    lse = np.empty((n, H), np.float64) if want_lse else None
+    counts = np.zeros(2, np.int64)
+    rc = lib().oracle_varlen_attn_skip(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32),
+                                       int(cu.shape[0]) - 1, T, H, D, scale, float(tau), _ptr(r, C.c_int32),
+                                       n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
+                                       _ptr(counts, C.c_int64))
+    if rc:
+        raise ValueError("oracle_varlen_attn_skip: invalid arguments")
+    return o, lse, (tuple(int(c) for c in counts) if r is None else None)
 
 
 def modulate_swiglu(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, gate_res: np.ndarray,

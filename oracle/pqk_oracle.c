@@ -22,6 +22,9 @@
  *                             request, valid tokens only (first page, section
  *                             "长序列注意力与通信优化"; second page, bullet
  *                             "Long-sequence attention & communication").
+ *   oracle_varlen_attn_skip -- the same attention with key blocks skipped
+ *                             where their scores are negligible ("Skip-Softmax";
+ *                             a reading, see the function).
  *   oracle_modulate_swiglu -- modulation + normalisation + gated residual and
  *                             SwiGLU in place of separate SiLU and multiply
  *                             (first page "融合 DiT 算子"; second page bullet
@@ -32,9 +35,9 @@
  * theta_j = base^(-2j/D), pairing, adaLN as h = n*(1+scale)+shift with one
  * vector set per request, x' = x + g*branch, SwiGLU = silu(gate)*up, the
  * softmax scale passed by the caller, LSE in natural log) are listed with
- * the pins that check each function in the repository's design notes. All
- * three functions are pinned by closed forms, brute force and invariants in
- * the CPU test suite.
+ * the pins that check each function in the repository's design notes. Every
+ * function is pinned by closed forms, brute force and invariants in the CPU
+ * test suite.
  *
  * Every function is the plain definition: no blocking, fusion or
  * reordering. Inputs are either bfloat16 bit patterns (widened exactly) or
@@ -279,6 +282,163 @@ int oracle_varlen_attn(const void* q, const void* k, const void* v, int in_kind,
     }
   }
   return bad ? -1 : 0;
+}
+
+/*
+ * Attention with block skipping: "Skip-Softmax" skips the softmax and the
+ * P x V work of unimportant blocks (first page, bullet on TRTLLM_ATTN SAGE and
+ * Skip-Softmax; second page, section "System-wide optimizations in
+ * vLLM-Omni", bullet "Sparse & quantized attention"). The pages name the idea
+ * only. The reading taken:
+ *   - a block is 32 consecutive query rows x 128 consecutive keys of one
+ *     request and head, both counted from the request's first token; key
+ *     blocks are visited in increasing order;
+ *   - with u(r,k) = s(r,k) / ln 2 (the score s includes the softmax scale),
+ *     key block j >= 1 is skipped for query block b when every row r of b
+ *     inside the request has max_{k in j} u(r,k) < M(r) - tau, where M(r) is
+ *     the maximum of u(r,k) over the keys of blocks 0 .. j-1 (key block 0 is
+ *     never skipped);
+ *   - a skipped block contributes nothing: o_r = sum_kept e^(s-m) v /
+ *     sum_kept e^(s-m) with m the maximum over kept keys, lse_r = m + ln(sum).
+ * A very large tau skips nothing and gives oracle_varlen_attn's result.
+ * rows: tokens to output (NULL = all T); each row's whole 32-row block is
+ * evaluated to take that block's decisions. counts (nullable, filled only
+ * when rows == NULL): counts[0] = skipped (32-row block, head, key block)
+ * triples; counts[1] = skipped (128-row tile, head, key block) triples, a
+ * 128-row tile (also counted from the request's first token) skipping a key
+ * block when all of its 32-row blocks inside the request do.
+ */
+#define ORACLE_SKIP_QROWS 32
+#define ORACLE_SKIP_KEYS 128
+#define ORACLE_SKIP_TILE 128
+
+/* Keep flags of the key blocks of query block [r0, r1) (rows of one request
+ * starting at lo, n_keys keys), head h. keep: [ceil(n_keys / 128)]. */
+static void skip_block_flags(const void* q, const void* k, int in_kind, int64_t stride_t, int64_t lo, int64_t n_keys,
+                             int64_t r0, int64_t r1, int h, int D, double scale, double tau, unsigned char* keep) {
+  const int64_t nkb = (n_keys + ORACLE_SKIP_KEYS - 1) / ORACLE_SKIP_KEYS;
+  const int64_t nr = r1 - r0;
+  double* tmax = (double*)malloc(sizeof(double) * (size_t)(nr * nkb));
+  double* qt = (double*)malloc(sizeof(double) * (size_t)D);
+  for (int64_t i = 0; i < nr; ++i) {
+    const int64_t t = r0 + i;
+    for (int d = 0; d < D; ++d) qt[d] = load(q, in_kind, t * stride_t + (int64_t)h * D + d);
+    for (int64_t jb = 0; jb < nkb; ++jb) tmax[i * nkb + jb] = -INFINITY;
+    for (int64_t j = 0; j < n_keys; ++j) {
+      double dot = 0.0;
+      const int64_t key_at = (lo + j) * stride_t + (int64_t)h * D;
+      for (int d = 0; d < D; ++d) dot += qt[d] * load(k, in_kind, key_at + d);
+      const double u = scale * dot / log(2.0);
+      double* tm = &tmax[i * nkb + j / ORACLE_SKIP_KEYS];
+      if (u > *tm) *tm = u;
+    }
+  }
+  for (int64_t jb = 0; jb < nkb; ++jb) {
+    int skip = jb >= 1;
+    for (int64_t i = 0; i < nr && skip; ++i) {
+      double M = -INFINITY;
+      for (int64_t pb = 0; pb < jb; ++pb)
+        if (tmax[i * nkb + pb] > M) M = tmax[i * nkb + pb];
+      if (!(tmax[i * nkb + jb] < M - tau)) skip = 0;
+    }
+    keep[jb] = (unsigned char)!skip;
+  }
+  free(qt);
+  free(tmax);
+}
+
+/* Output row t (of request lo, n_keys), head h, over the kept key blocks. */
+static void skip_row_output(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t, int64_t lo,
+                            int64_t n_keys, int64_t t, int h, int D, double scale, const unsigned char* keep, double* ot,
+                            double* lse_out) {
+  double* sc = (double*)malloc(sizeof(double) * (size_t)n_keys);
+  double* qt = (double*)malloc(sizeof(double) * (size_t)D);
+  for (int d = 0; d < D; ++d) qt[d] = load(q, in_kind, t * stride_t + (int64_t)h * D + d);
+  double m = -INFINITY;
+  for (int64_t j = 0; j < n_keys; ++j) {
+    if (!keep[j / ORACLE_SKIP_KEYS]) continue;
+    double dot = 0.0;
+    const int64_t key_at = (lo + j) * stride_t + (int64_t)h * D;
+    for (int d = 0; d < D; ++d) dot += qt[d] * load(k, in_kind, key_at + d);
+    sc[j] = scale * dot;
+    if (sc[j] > m) m = sc[j];
+  }
+  double mass = 0.0;
+  for (int d = 0; d < D; ++d) ot[d] = 0.0;
+  for (int64_t j = 0; j < n_keys; ++j) {
+    if (!keep[j / ORACLE_SKIP_KEYS]) continue;
+    const double pj = exp(sc[j] - m);
+    mass += pj;
+    const int64_t val_at = (lo + j) * stride_t + (int64_t)h * D;
+    for (int d = 0; d < D; ++d) ot[d] += pj * load(v, in_kind, val_at + d);
+  }
+  for (int d = 0; d < D; ++d) ot[d] /= mass;
+  if (lse_out) *lse_out = m + log(mass);
+  free(sc);
+  free(qt);
+}
+
+int oracle_varlen_attn_skip(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
+                            const int32_t* cu, int B, int64_t T, int H, int D, double scale, double tau,
+                            const int32_t* rows, int64_t nrows, double* o, double* lse, int64_t* counts) {
+  if (check_cu(cu, B, T) || H <= 0 || D <= 0 || isnan(tau)) return -1;
+  if (rows != NULL) {
+    int64_t bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2) reduction(+ : bad)
+    for (int64_t r = 0; r < nrows; ++r) {
+      for (int h = 0; h < H; ++h) {
+        const int64_t t = rows[r];
+        const int seg = (t >= 0 && t < T) ? segment_of(cu, B, t) : -1;
+        if (seg < 0) { ++bad; continue; }
+        const int64_t lo = cu[seg], n_keys = (int64_t)cu[seg + 1] - (int64_t)cu[seg];
+        const int64_t r0 = lo + ((t - lo) / ORACLE_SKIP_QROWS) * ORACLE_SKIP_QROWS;
+        const int64_t r1 = r0 + ORACLE_SKIP_QROWS < lo + n_keys ? r0 + ORACLE_SKIP_QROWS : lo + n_keys;
+        unsigned char* keep = (unsigned char*)malloc((size_t)((n_keys + ORACLE_SKIP_KEYS - 1) / ORACLE_SKIP_KEYS));
+        skip_block_flags(q, k, in_kind, stride_t, lo, n_keys, r0, r1, h, D, scale, tau, keep);
+        skip_row_output(q, k, v, in_kind, stride_t, lo, n_keys, t, h, D, scale, keep, o + (r * H + h) * (int64_t)D,
+                        lse ? &lse[r * H + h] : NULL);
+        free(keep);
+      }
+    }
+    return bad ? -1 : 0;
+  }
+  int64_t n_block = 0, n_tile = 0;
+  for (int seg = 0; seg < B; ++seg) {
+    const int64_t lo = cu[seg], n_keys = (int64_t)cu[seg + 1] - (int64_t)cu[seg];
+    if (n_keys == 0) continue;
+    const int64_t nqb = (n_keys + ORACLE_SKIP_QROWS - 1) / ORACLE_SKIP_QROWS;
+    const int64_t nkb = (n_keys + ORACLE_SKIP_KEYS - 1) / ORACLE_SKIP_KEYS;
+    unsigned char* keep = (unsigned char*)malloc((size_t)(H * nqb * nkb));
+#pragma omp parallel for schedule(dynamic, 1) collapse(2) reduction(+ : n_block)
+    for (int64_t b = 0; b < nqb; ++b) {
+      for (int h = 0; h < H; ++h) {
+        const int64_t r0 = lo + b * ORACLE_SKIP_QROWS;
+        const int64_t r1 = r0 + ORACLE_SKIP_QROWS < lo + n_keys ? r0 + ORACLE_SKIP_QROWS : lo + n_keys;
+        unsigned char* kp = keep + ((int64_t)h * nqb + b) * nkb;
+        skip_block_flags(q, k, in_kind, stride_t, lo, n_keys, r0, r1, h, D, scale, tau, kp);
+        for (int64_t t = r0; t < r1; ++t)
+          skip_row_output(q, k, v, in_kind, stride_t, lo, n_keys, t, h, D, scale, kp, o + (t * H + h) * (int64_t)D,
+                          lse ? &lse[t * H + h] : NULL);
+        for (int64_t jb = 0; jb < nkb; ++jb) n_block += !kp[jb];
+      }
+    }
+    /* a 128-row tile skips key block jb when each of its 32-row blocks inside the request does */
+    const int64_t per_tile = ORACLE_SKIP_TILE / ORACLE_SKIP_QROWS;
+    for (int h = 0; h < H; ++h)
+      for (int64_t tb = 0; tb * per_tile < nqb; ++tb)
+        for (int64_t jb = 0; jb < nkb; ++jb) {
+          int all = 1;
+          for (int64_t b = tb * per_tile; b < (tb + 1) * per_tile && b < nqb; ++b)
+            if (keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;
+          n_tile += all;
+        }
+    free(keep);
+  }
+  if (counts) {
+    counts[0] = n_block;
+    counts[1] = n_tile;
+  }
+  return 0;
 }
 
 /*

@@ -16,7 +16,7 @@ import pytest
 
 from oracle import oracle
 from tests import (test_oracle_attention, test_oracle_fullc, test_oracle_modulate, test_oracle_norm_rope,
-                   test_oracle_rope3)
+                   test_oracle_rope3, test_oracle_skip)
 
 MUTANTS = {
     "attn_drop_scale": ("s[j] = scale * acc;", "s[j] = acc;"),
@@ -50,12 +50,18 @@ MUTANTS = {
     "rope3_ids_of_first_token": ("(double)pos3[t * 3 + axis]", "(double)pos3[axis]"),
     "fullc_mean_over_one_head": ("ms /= (double)width;", "ms /= (double)D;"),
     "fullc_weight_of_first_head": ("* inv * load(w, w_kind, (int64_t)h * D + d);", "* inv * load(w, w_kind, d);"),
+    "skip_first_row_decides": ("for (int64_t i = 0; i < nr && skip; ++i) {", "for (int64_t i = 0; i < 1 && skip; ++i) {"),
+    "skip_query_block_64": ("#define ORACLE_SKIP_QROWS 32", "#define ORACLE_SKIP_QROWS 64"),
+    "skip_threshold_sign": ("if (!(tmax[i * nkb + jb] < M - tau)) skip = 0;", "if (!(tmax[i * nkb + jb] < M + tau)) skip = 0;"),
+    "skip_natural_log_units": ("const double u = scale * dot / log(2.0);", "const double u = scale * dot;"),
+    "skip_tile_counts_any_block": ("if (keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;",
+                                   "if (!keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;"),
 }
 
 
 def _pin_calls():
     for mod in (test_oracle_attention, test_oracle_norm_rope, test_oracle_modulate, test_oracle_rope3,
-                test_oracle_fullc):
+                test_oracle_fullc, test_oracle_skip):
         for name, fn in inspect.getmembers(mod, inspect.isfunction):
             if not name.startswith("test_") or fn.__module__ != mod.__name__:
                 continue
