@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--skip-tau", type=float, default=8.0,
+                    help="threshold (log2 units) of the block-skipping attention timed on the local-attention "
+                         "stand-in after the steps; negative = leave that timing out")
     return ap.parse_args()
 
 
@@ -368,6 +371,44 @@ def run_ours(args, w):
     fullc_us = ev3[0].elapsed_time(ev3[1]) / reps3 * 1e3
     fullc_gbs = (w.prologue_bytes() + 2 * w.H * w.D * 2) / (fullc_us * 1e-6) / 1e9
 
+    # block skipping (Skip-Softmax) on the local-attention stand-in: Q and K
+    # from sinusoids of the (t, h, w) ids plus noise, so that attention weight
+    # sits on nearby tokens as in video; plain and skipping kernels on the
+    # same inputs, and the share of dropped block decisions
+    skip = None
+    if args.skip_tau >= 0:
+        lx = wl.local_attention_inputs(w, amplitude=16.0)
+        lq, lk, lv = (torch.from_numpy(lx[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k", "v"))
+        counts = torch.zeros(2, dtype=torch.int64, device=dev)
+        lo = torch.empty_like(lq)
+        plain = lambda: pqk.varlen_attn_fwd(lq, lk, lv, d["cu"], o=lo, workspace=o["ws"])
+        skipping = lambda c=None: pqk.varlen_attn_fwd_skip(lq, lk, lv, d["cu"], args.skip_tau, o=lo,
+                                                           workspace=o["ws"], skip_counts=c)
+        plain()
+        skipping(counts)
+        torch.cuda.synchronize()
+        times = {}
+        for name, fn in (("plain", plain), ("skip", skipping), ("plain2", plain), ("skip2", skipping)):
+            ev3[0].record()
+            for _ in range(3):
+                fn()
+            ev3[1].record()
+            torch.cuda.synchronize()
+            times[name] = ev3[0].elapsed_time(ev3[1]) / 3
+        if pqk.get_device_status() != 0:
+            raise RuntimeError("device status set during the block-skipping timing")
+        c = counts.cpu().tolist()
+        n32 = sum(((L + 31) // 32) * ((L + 127) // 128) for L in w.seg_lens) * w.H
+        n128 = sum(((L + 127) // 128) ** 2 for L in w.seg_lens) * w.H
+        plain_ms = min(times["plain"], times["plain2"])
+        skip_ms = min(times["skip"], times["skip2"])
+        skip = {"input": "local-attention stand-in: Q, K = 16 x unit sinusoid features of the (t, h, w) ids "
+                         "+ N(0, 1) noise, V ~ N(0, 1)",
+                "tau_log2": args.skip_tau, "plain_ms": plain_ms, "skip_ms": skip_ms,
+                "speedup": plain_ms / skip_ms, "dropped_block_share": c[0] / n32,
+                "skipped_pv_share": c[1] / n128}
+        del lq, lk, lv, lo, lx
+
     # e2e through host buffers: every step copies all of its inputs from
     # pinned host memory to the device (H2D stream), runs the three C-ABI
     # calls (compute stream) and copies its outputs x', h, act back to pinned
@@ -467,7 +508,8 @@ def run_ours(args, w):
                     "qk_norm_rope_3axis_sections": list(sections),
                     "qk_norm_rope_back_to_back_us": rope1_b2b_us,
                     "qk_fullc_norm_rope_us": fullc_us, "qk_fullc_norm_rope_gbs": fullc_gbs,
-                    "qk_fullc_norm_rope_frac_hbm": fullc_gbs / pk["hbm_gbs"]},
+                    "qk_fullc_norm_rope_frac_hbm": fullc_gbs / pk["hbm_gbs"],
+                    "varlen_attn_skip": skip},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * K,

@@ -175,6 +175,40 @@ PQK_API int pqk_varlen_attn_fwd(const void* q, const void* k, const void* v, voi
                         void* stream);
 
 /*
+ * pqk_varlen_attn_fwd_skip -- pqk_varlen_attn_fwd that leaves out the
+ * softmax and the P x V product of key blocks whose scores are negligible
+ * ("Skip-Softmax": first page, bullet on TRTLLM_ATTN SAGE and Skip-Softmax;
+ * second page, bullet "Sparse & quantized attention"). The pages name the
+ * idea only; the rule implemented:
+ *   - blocks are 32 consecutive query rows x 128 consecutive keys of one
+ *     request and head, counted from the request's first token;
+ *   - key block j >= 1 is dropped for a query block when every one of its
+ *     rows t has max_{k in block j} u(t,k) < M(t) - skip_threshold_log2,
+ *     u = softmax_scale * <Q[t,h], K[k,h]> / ln 2 and M(t) the maximum of
+ *     u(t, k) over the keys of blocks 0 .. j-1 (block 0 is always kept);
+ *   - dropped keys contribute nothing to O or lse. Every dropped key has a
+ *     weight below 2^-skip_threshold_log2 of the row's largest, so O moves
+ *     by at most 2 * n_dropped * 2^-skip_threshold_log2 * max|V|.
+ * The decision is taken in fp32 on the tensor-core scores, so rows whose
+ * margin to the threshold is within fp32 rounding may decide either way.
+ *
+ * skip_threshold_log2  >= 0 (+inf keeps every block; NaN or negative is
+ *               PQK_ERR_INVALID_ARG).
+ * skip_counts   NULL, or device uint64 [2], 8-byte aligned, that the call
+ *               adds to: [0] dropped (32-row block, head, key block)
+ *               triples; [1] (128-row tile, head, key block) triples whose
+ *               P x V product was left out because all four of the tile's
+ *               32-row blocks inside the request dropped the key block.
+ * Other arguments, layouts and errors are those of pqk_varlen_attn_fwd.
+ */
+PQK_API int pqk_varlen_attn_fwd_skip(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int64_t q_stride_t, int64_t k_stride_t, int64_t v_stride_t,
+                             int64_t o_stride_t, const int32_t* cu_seqlens, int B, int64_t T, int H,
+                             int D, float softmax_scale, float skip_threshold_log2,
+                             unsigned long long* skip_counts, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/*
  * pqk_varlen_attn_fwd_noalloc -- pqk_varlen_attn_fwd for callers that cannot
  * allocate device memory. The pages have no counterpart: this entry point
  * exists for callers such as plugins or embedded runtimes that are handed

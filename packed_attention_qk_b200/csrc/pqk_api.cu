@@ -178,6 +178,33 @@ int pqk_varlen_attn_fwd(const void* q, const void* k, const void* v, void* o, fl
   return rc == 0 ? PQK_OK : (rc == -2 ? PQK_ERR_INVALID_ARG : PQK_ERR_CUDA);
 }
 
+int pqk_varlen_attn_fwd_skip(const void* q, const void* k, const void* v, void* o, float* lse, int64_t q_stride_t,
+                             int64_t k_stride_t, int64_t v_stride_t, int64_t o_stride_t, const int32_t* cu_seqlens,
+                             int B, int64_t T, int H, int D, float softmax_scale, float skip_threshold_log2,
+                             unsigned long long* skip_counts, void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 1 || T < 0 || H <= 0 || T > INT32_MAX - 512 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return PQK_ERR_INVALID_ARG;
+  if (!(skip_threshold_log2 >= 0.f)) return PQK_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return PQK_ERR_UNSUPPORTED;
+  const int64_t row = static_cast<int64_t>(H) * D;
+  if (q_stride_t < row || k_stride_t < row || v_stride_t < row || o_stride_t < row) return PQK_ERR_INVALID_ARG;
+  if (T == 0) return PQK_OK;
+  if (!q || !k || !v || !o || !cu_seqlens) return PQK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (q_stride_t % 8) || (k_stride_t % 8) || (v_stride_t % 8) || (o_stride_t % 8) ||
+      (reinterpret_cast<uintptr_t>(skip_counts) % 8))
+    return PQK_ERR_MISALIGNED;
+  if (workspace == nullptr || workspace_bytes < pqk_varlen_attn_workspace_size(B)) return PQK_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return PQK_ERR_MISALIGNED;
+  DeviceInfo* d = nullptr;
+  if (int rc = check_device(&d)) return rc;
+  const int rc = pqk::launch_varlen_attn(q, k, v, o, lse, q_stride_t, k_stride_t, v_stride_t, o_stride_t,
+                                         cu_seqlens, B, T, H, D, softmax_scale, workspace, d->status,
+                                         g_timeout_ns.load(), static_cast<cudaStream_t>(stream), d->num_sms,
+                                         true, skip_threshold_log2, skip_counts);
+  return rc == 0 ? PQK_OK : (rc == -2 ? PQK_ERR_INVALID_ARG : PQK_ERR_CUDA);
+}
+
 int pqk_modulate_swiglu(const void* x, const void* branch, void* x_out, void* h, const float* shift,
                         const float* scale, const float* gate_res, const int32_t* cu_seqlens, int B, int64_t T, int C,
                         int norm_type, float eps, const void* gate, const void* up, int64_t gu_stride_t, void* act,

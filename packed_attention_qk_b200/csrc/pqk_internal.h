@@ -30,12 +30,15 @@ int launch_modulate_swiglu(const void* x, const void* branch, void* x_out, void*
 size_t attn_schedule_bytes(int B);
 
 // Prepares and enqueues the attention kernel's TMA descriptors, the schedule
-// builder and the persistent attention kernel. Returns 0, or -1 when a CUDA
-// call failed, -2 when the tensor maps could not be encoded.
+// builder and the persistent attention kernel. skip selects the block-
+// skipping kernel (threshold skip_tau in log2 units; skip_counts nullable,
+// two device counters the kernel adds to). Returns 0, or -1 when a CUDA call
+// failed, -2 when the tensor maps could not be encoded.
 int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, float* lse, int64_t q_stride,
                        int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
                        int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
-                       long long timeout_ns, cudaStream_t stream, int num_sms);
+                       long long timeout_ns, cudaStream_t stream, int num_sms, bool skip = false,
+                       float skip_tau = 0.0f, unsigned long long* skip_counts = nullptr);
 
 int launch_wait_selftest(int* status, long long timeout_ns, cudaStream_t stream);
 

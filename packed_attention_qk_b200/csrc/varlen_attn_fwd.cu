@@ -86,7 +86,9 @@ struct Layout {
   static constexpr int kNumBars = 2 * kStages + 8;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
-  static constexpr int kBytes = kAbortOff + 4;
+  // block-skip votes: one byte per softmax warp, [group][tile parity][warp]
+  static constexpr int kVoteOff = kAbortOff + 4;
+  static constexpr int kBytes = kVoteOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
   static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256, kTmemO1 = 256 + D;
   static_assert(kAlloc <= 232448, "shared memory budget");
@@ -107,6 +109,8 @@ struct AttnParams {
   const int32_t* sched;
   int* status;
   long long timeout_ns;
+  float skip_tau;                        // block-skip threshold (log2 units), kSkip only
+  unsigned long long* skip_counts;       // nullable: [0] skipped warp blocks, [1] skipped O += P V products
 };
 
 struct Work {
@@ -301,7 +305,7 @@ __device__ __forceinline__ float exp_tile_store(const float (&s)[128], float sca
   return (l0 + l1) + (l2 + l3);
 }
 
-template <int D>
+template <int D, bool kSkip>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -325,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto o_done = [&](int i) { return q_full + 48 + 8u * i; };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
+  volatile uint8_t* votes = smem + L::kVoteOff;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -407,6 +412,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
       uint32_t cons_idx = 0;
       uint32_t p_phase = 0;
+      unsigned long long pv_skips = 0;
+      // every softmax warp of group i voted to skip K/V tile j
+      auto group_skips = [&](int i, int j) {
+        return *reinterpret_cast<volatile uint32_t*>(votes + (i * 2 + (j & 1)) * 4) == 0x01010101u;
+      };
       int wt = 0;
       bool ok = true;
       // Descriptor low words of Q0 and of stage 0 (K: K-major, V: MN-major
@@ -443,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
         const Work wk = decode_work(p.sched, p.H, w);
+        const bool q1_in_request = wk.q0 + kBM < wk.seg_start + wk.seg_len;
         if (!(ok = mbar_wait(q_full, wt & 1, abort_flag, p.timeout_ns))) break;
         uint32_t k_stage_idx = cons_idx;
         if (!(ok = wait_stage(k_stage_idx))) break;
@@ -464,7 +475,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (more && !(ok = wait_stage(nk_idx))) break;
           if (!(ok = mbar_wait(p_full(0), p_phase, abort_flag, p.timeout_ns))) break;
           tc_fence_after_sync();
-          issue_pv(0, v_idx % L::kStages, j > 0);
+          if (kSkip && j > 0 && group_skips(0, j)) {
+            ++pv_skips;
+          } else {
+            issue_pv(0, v_idx % L::kStages, j > 0);
+          }
           if (!more) tc_commit(o_done(0));
           if (more) {
             issue_qk(0, nk_idx % L::kStages);
@@ -472,7 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!(ok = mbar_wait(p_full(1), p_phase, abort_flag, p.timeout_ns))) break;
           tc_fence_after_sync();
-          issue_pv(1, v_idx % L::kStages, j > 0);
+          if (kSkip && j > 0 && group_skips(1, j)) {
+            if (q1_in_request) ++pv_skips;
+          } else {
+            issue_pv(1, v_idx % L::kStages, j > 0);
+          }
           if (!more) tc_commit(o_done(1));
           tc_commit(kv_empty(v_idx % L::kStages));
           if (more) {
@@ -484,6 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           p_phase ^= 1u;
         }
       }
+      if (kSkip && p.skip_counts != nullptr && pv_skips != 0) atomicAdd(&p.skip_counts[1], pv_skips);
       if (!ok) {
         raise_abort(abort_flag, p.status);
         // every MMA issued by this thread must complete before the tensor
@@ -506,10 +526,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_phase = 0;
     int wt = 0;
     bool ok = true;
+    unsigned long long warp_skips = 0;
     for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
       const Work wk = decode_work(p.sched, p.H, w);
       const int row = wk.q0 + grp * kBM + r;
       float m = -INFINITY, l = 0.f;
+      float m_seen = -INFINITY;  // block skipping: running maximum over all earlier tiles
       for (int j = 0; j < wk.n_kv; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full(grp), s_phase, abort_flag, p.timeout_ns));
         if (!ok) break;
@@ -520,6 +542,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s[128];
         load_scores(t_s, valid, s);
         const float mx = row_max(s) * p.scale_log2;
+        if constexpr (kSkip) {
+          // Skip-Softmax: this warp's 32 rows drop K/V tile j when every row
+          // of the request has its tile maximum more than skip_tau below its
+          // maximum over tiles 0..j-1. The vote goes to the MMA thread, which
+          // leaves out O_i += P_i V_j when all four warps of the group drop it.
+          const bool in_request = row < wk.seg_start + wk.seg_len;
+          const bool skip = __all_sync(0xffffffffu, !in_request || (j > 0 && mx < m_seen - p.skip_tau));
+          m_seen = fmaxf(m_seen, mx);
+          if (lane == 0) votes[(grp * 2 + (j & 1)) * 4 + (warp & 3)] = skip ? 1 : 0;
+          if (skip) {
+            if (__any_sync(0xffffffffu, in_request) && lane == 0) ++warp_skips;
+            // P = 0 for these rows (the product still runs if another warp keeps the tile)
+            uint32_t zero[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) zero[c] = 0u;
+            tmem_st_x64(t_s, zero);
+            tc_fence_before_sync();
+            mbar_arrive(p_full(grp));
+            continue;
+          }
+        }
         const bool need_rescale = j > 0 && mx > m + kRescaleThreshold;
         float alpha = 1.0f;
         if (j == 0) {
@@ -576,6 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.lse[static_cast<int64_t>(wk.head) * p.T + row] = (m + __log2f(l)) * 0.69314718055994530942f;
       tc_fence_before_sync();
     }
+    if (kSkip && p.skip_counts != nullptr && lane == 0 && warp_skips != 0) atomicAdd(&p.skip_counts[0], warp_skips);
     if (!ok) raise_abort(abort_flag, p.status);
   }
 
@@ -636,14 +680,14 @@ bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t T, int H, int D, in
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool kSkip>
 bool set_smem_attr() {
   static int done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<D>::kAlloc) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kSkip>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Layout<D>::kAlloc) != cudaSuccess)
       return false;
     done[dev] = 1;
   }
@@ -657,7 +701,8 @@ size_t attn_schedule_bytes(int B) { return ((sched_words(B) * sizeof(int32_t)) +
 int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, float* lse, int64_t q_stride,
                        int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
                        int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
-                       long long timeout_ns, cudaStream_t stream, int num_sms) {
+                       long long timeout_ns, cudaStream_t stream, int num_sms, bool skip, float skip_tau,
+                       unsigned long long* skip_counts) {
   CUtensorMap tq, tk, tv;
   if (!make_qkv_map(&tq, q, T, H, D, q_stride) || !make_qkv_map(&tk, k, T, H, D, k_stride) ||
       !make_qkv_map(&tv, v, T, H, D, v_stride))
@@ -675,15 +720,23 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
   p.sched = sched;
   p.status = status;
   p.timeout_ns = timeout_ns;
+  p.skip_tau = skip_tau;
+  p.skip_counts = skip_counts;
   // upper bound of work tiles: every request adds at most one partial block
   const int64_t max_work = static_cast<int64_t>(H) * ((T + kRowsPerWork - 1) / kRowsPerWork + B);
   const int grid = static_cast<int>(max_work < num_sms ? max_work : num_sms);
-  if (D == 128) {
-    if (!set_smem_attr<128>()) return -1;
-    attn_fwd_kernel<128><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+  if (D == 128 && !skip) {
+    if (!set_smem_attr<128, false>()) return -1;
+    attn_fwd_kernel<128, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+  } else if (D == 128) {
+    if (!set_smem_attr<128, true>()) return -1;
+    attn_fwd_kernel<128, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+  } else if (!skip) {
+    if (!set_smem_attr<64, false>()) return -1;
+    attn_fwd_kernel<64, false><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
   } else {
-    if (!set_smem_attr<64>()) return -1;
-    attn_fwd_kernel<64><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<64, true>()) return -1;
+    attn_fwd_kernel<64, true><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

@@ -22,7 +22,7 @@ NORM_RMS, NORM_LAYER, NORM_NONE = 0, 1, 2
 
 # every symbol include/pqk.h declares
 EXPORTS = ("pqk_qk_norm_rope", "pqk_qk_norm_rope_3axis", "pqk_qk_fullc_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd",
-           "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu",
+           "pqk_varlen_attn_fwd_skip", "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu",
            "pqk_get_device_status", "pqk_set_wait_timeout_ns", "pqk_selftest_wait_timeout", "pqk_status_string",
            "pqk_version")
 
@@ -59,6 +59,9 @@ def lib(path: str | None = None) -> C.CDLL:
     L.pqk_varlen_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32, vp, sz,
                                       vp]
     L.pqk_varlen_attn_fwd.restype = i32
+    L.pqk_varlen_attn_fwd_skip.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32, f32,
+                                           vp, vp, sz, vp]
+    L.pqk_varlen_attn_fwd_skip.restype = i32
     L.pqk_varlen_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32,
                                               vp]
     L.pqk_varlen_attn_fwd_noalloc.restype = i32
@@ -181,6 +184,33 @@ def varlen_attn_fwd(q, k, v, cu_seqlens, *, softmax_scale: float | None = None, 
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _token_stride(q, 3), _token_stride(k, 3),
         _token_stride(v, 3), _token_stride(o, 3), _ptr(cu_seqlens), B, T, H, D, scale, _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+def varlen_attn_fwd_skip(q, k, v, cu_seqlens, skip_threshold_log2: float, *, softmax_scale: float | None = None,
+                         o=None, lse=None, workspace=None, want_lse: bool = False, skip_counts=None, stream=None):
+    """Packed varlen attention that drops key blocks whose scores lie more
+    than skip_threshold_log2 (log2 units) below the earlier blocks' maximum
+    for every row of a 32-row query block. skip_counts: None or a device
+    int64 tensor of 2 elements that the call adds to (dropped 32-row blocks,
+    left-out 128-row P x V products). Returns (o, lse or None)."""
+    import torch
+    T, H, D = q.shape
+    B = cu_seqlens.shape[0] - 1
+    scale = softmax_scale if softmax_scale is not None else D ** -0.5
+    if o is None:
+        o = torch.empty((T, H, D), dtype=q.dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((H, T), dtype=torch.float32, device=q.device)
+    ws_bytes = varlen_attn_workspace_size(B)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if skip_counts is not None:
+        assert skip_counts.dtype == torch.int64 and skip_counts.numel() >= 2 and skip_counts.is_contiguous()
+    _check("pqk_varlen_attn_fwd_skip", lib().pqk_varlen_attn_fwd_skip(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _token_stride(q, 3), _token_stride(k, 3),
+        _token_stride(v, 3), _token_stride(o, 3), _ptr(cu_seqlens), B, T, H, D, scale, float(skip_threshold_log2),
+        _ptr(skip_counts), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return o, lse
 
 

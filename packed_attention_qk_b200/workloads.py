@@ -22,7 +22,13 @@ draw one tensor without drawing the others):
   * RMSNorm weights w_q, w_k ~ U(0.5, 1.5), rounded to bfloat16;
   * adaLN shift / scale / gated-residual gate ~ N(0, 0.1) kept in float32;
   * outlier variant: an i.i.d. Bernoulli(0.001) mask over K's elements; masked
-    elements are multiplied by 20 in float32 before the bfloat16 rounding.
+    elements are multiplied by 20 in float32 before the bfloat16 rounding;
+  * block-scaled attention inputs (key-block skipping tests): Q ~ 2.5 N(0, 1);
+    K ~ N(0, 1) times a per-(request, 128-key block) factor, 3 ("strong") or
+    0.02 ("weak") with probability 1/2 each from stream ``skip_blocks``;
+  * local attention inputs (a stand-in for video attention, whose weight sits
+    on nearby tokens): every token gets a unit feature vector of sinusoids of
+    its (t, h, w) ids, Q = K-ish = A * feature + N(0, 1) noise per head.
 bfloat16 tensors are returned as their uint16 bit patterns.
 """
 
@@ -40,6 +46,7 @@ TENSOR_ID = {
     "q": 1, "k": 2, "v": 3, "x": 4, "branch": 5, "gate": 6, "up": 7,
     "w_q": 8, "w_k": 9, "shift": 10, "scale": 11, "gate_res": 12,
     "outlier": 13, "sample_rows": 14, "w_q_full": 15, "w_k_full": 16,
+    "skip_blocks": 17, "q_local": 18, "k_local": 19,
 }
 
 
@@ -289,6 +296,65 @@ def epilogue_inputs(w: Workload, with_branch: bool = False) -> dict[str, np.ndar
     if with_branch:
         d["branch"] = bf16_normal(w.seed, "branch", (w.T, w.C))
     return d
+
+
+def block_scaled_attention_inputs(w: Workload, strong: float = 3.0, weak: float = 0.02,
+                                  q_scale: float = 2.5) -> dict[str, np.ndarray]:
+    """Q ~ q_scale N(0, 1); K ~ N(0, 1) times a factor per (request, block of
+    128 keys counted from the request's first token), ``strong`` or ``weak``
+    with probability 1/2 each; V ~ N(0, 1). Returns bf16 bits plus the block
+    factors (one per block, requests in order)."""
+    shp = (w.T, w.H, w.D)
+    n = w.T * w.H * w.D
+    cu = w.cu_seqlens()
+    nblk = [(int(L) + 127) // 128 for L in w.seg_lens]
+    g = _chunk_rng(w.seed, "skip_blocks", 0)
+    factors = np.where(g.random(int(sum(nblk))) < 0.5, weak, strong).astype(np.float32)
+    per_key = np.empty(w.T, np.float32)
+    b0 = 0
+    for i, L in enumerate(w.seg_lens):
+        lo = int(cu[i])
+        for j in range(nblk[i]):
+            per_key[lo + 128 * j: lo + min(int(L), 128 * (j + 1))] = factors[b0 + j]
+        b0 += nblk[i]
+    q = f32_to_bf16_bits(_draw(w.seed, "q", n, "normal").reshape(shp) * np.float32(q_scale))
+    k = f32_to_bf16_bits(_draw(w.seed, "k", n, "normal").reshape(shp) * per_key[:, None, None])
+    return {"q": q, "k": k, "v": bf16_normal(w.seed, "v", shp), "cu_seqlens": cu, "block_factors": factors}
+
+
+def local_features(pos3: np.ndarray, D: int, base: float = 100.0) -> np.ndarray:
+    """[T, D] unit vectors of sinusoids of the (t, h, w) ids: D/8 frequency
+    pairs for t, 3D/16 each for h and w, frequencies base^(-i/n) per axis;
+    the inner product of two tokens' vectors is the mean over pairs of
+    cos(id difference * frequency)."""
+    n_axis = (D // 8, 3 * D // 16, 3 * D // 16)
+    assert sum(n_axis) * 2 == D
+    cols = []
+    for a, n in enumerate(n_axis):
+        freq = base ** (-np.arange(n) / n)
+        ang = pos3[:, a:a + 1].astype(np.float64) * freq[None, :]
+        cols += [np.cos(ang), np.sin(ang)]
+    f = np.concatenate(cols, axis=1) / np.sqrt(D / 2)
+    return f.astype(np.float32)
+
+
+def local_attention_inputs(w: Workload, amplitude: float = 12.0, noise: float = 1.0,
+                           video_grid: tuple[int, int, int] = (12, 48, 96)) -> dict[str, np.ndarray]:
+    """Q[t, h] = amplitude * f(t) + noise * N(0, 1), K the same with its own
+    noise, V ~ N(0, 1); f = local_features of the (t, h, w) ids (positions3).
+    Drawn head by head (stream chunk = head index) to bound host memory."""
+    f = local_features(w.positions3(video_grid), w.D) * np.float32(amplitude)
+    q = np.empty((w.T, w.H, w.D), np.uint16)
+    k = np.empty((w.T, w.H, w.D), np.uint16)
+
+    def head(h: int) -> None:
+        for name, out in (("q_local", q), ("k_local", k)):
+            z = _chunk_rng(w.seed, name, h).standard_normal((w.T, w.D), dtype=np.float32)
+            out[:, h, :] = f32_to_bf16_bits(f + np.float32(noise) * z)
+
+    with _cf.ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(head, range(w.H)))
+    return {"q": q, "k": k, "v": bf16_normal(w.seed, "v", (w.T, w.H, w.D)), "cu_seqlens": w.cu_seqlens()}
 
 
 def sample_rows(w: Workload, per_segment: int = 256) -> np.ndarray:

@@ -169,3 +169,24 @@ def test_selftest_rejects_bad_timeout(L):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="libpqk.so not found"):
         pqk.lib(str(tmp_path / "libpqk.so"))
+
+
+def attn_skip(L, **kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=None, qs=1024, ks=1024, vs=1024, os_=1024, cu=A, B=2, T=512, H=8, D=128,
+             scale=0.088, tau=8.0, counts=None, ws=A, wsb=4096)
+    a.update(kw)
+    return L.pqk_varlen_attn_fwd_skip(a["q"], a["k"], a["v"], a["o"], a["lse"], a["qs"], a["ks"], a["vs"], a["os_"],
+                                      a["cu"], a["B"], a["T"], a["H"], a["D"], a["scale"], a["tau"], a["counts"],
+                                      a["ws"], a["wsb"], None)
+
+
+def test_varlen_attn_skip_host_errors(L):
+    assert attn_skip(L, tau=-1.0) == ERR_INVALID
+    assert attn_skip(L, tau=float("nan")) == ERR_INVALID
+    assert attn_skip(L, D=96) == ERR_UNSUPPORTED
+    assert attn_skip(L, scale=0.0) == ERR_INVALID
+    assert attn_skip(L, counts=A + 4) == ERR_MISALIGNED
+    assert attn_skip(L, q=U) == ERR_MISALIGNED
+    assert attn_skip(L, ws=None) == ERR_WORKSPACE
+    assert attn_skip(L, T=0, q=None) == 0
+    assert attn_skip(L, T=0, q=None, tau=float("inf")) == 0
