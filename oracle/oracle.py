@@ -55,8 +55,15 @@ def load(path: str):
     L.oracle_varlen_attn_skip.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
                                           C.c_int, C.c_double, C.c_double, i32p, C.c_int64, f64p, f64p,
                                           C.POINTER(C.c_int64)]
+    u8p = C.POINTER(C.c_uint8)
+    L.oracle_quantize_e4m3.argtypes = [vp, C.c_int, C.c_int64, C.c_int64, C.c_int, C.c_int, u8p, f32p]
+    L.oracle_varlen_attn_fp8qk.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
+                                           C.c_int, C.c_double, i32p, C.c_int64, f64p, f64p, u8p, u8p, f32p]
+    L.oracle_e4m3_codes.argtypes = [f32p, C.c_int64, u8p]
+    L.oracle_e4m3_codes.restype = None
     for f in (L.oracle_qk_norm_rope, L.oracle_qk_norm_rope_3axis, L.oracle_qk_fullc_norm_rope, L.oracle_varlen_attn,
-              L.oracle_varlen_attn_skip, L.oracle_modulate_swiglu):
+              L.oracle_varlen_attn_skip, L.oracle_quantize_e4m3, L.oracle_varlen_attn_fp8qk,
+              L.oracle_modulate_swiglu):
         f.restype = C.c_int
     L.oracle_num_threads.restype = C.c_int
     return L
@@ -196,6 +203,50 @@ def varlen_attn_skip(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np
     if rc:
         raise ValueError("oracle_varlen_attn_skip: invalid arguments")
     return o, lse, (tuple(int(c) for c in counts) if r is None else None)
+
+
+def e4m3_codes(x: np.ndarray) -> np.ndarray:
+    """FP8 e4m3 codes (uint8) of float32 values: nearest, ties to even,
+    magnitudes beyond 448 saturating to 448."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().oracle_e4m3_codes(_ptr(x, C.c_float), x.size, _ptr(out, C.c_uint8))
+    return out
+
+
+def quantize_e4m3(x: np.ndarray):
+    """Per-head absmax e4m3 quantisation of [T, H, D]: (codes uint8 [T, H, D], deq float32 [H])."""
+    T, H, D = x.shape
+    x = np.ascontiguousarray(x)
+    codes = np.empty((T, H, D), np.uint8)
+    deq = np.empty(H, np.float32)
+    if lib().oracle_quantize_e4m3(_ptr(x), _kind(x), H * D, T, H, D, _ptr(codes, C.c_uint8), _ptr(deq, C.c_float)):
+        raise ValueError("oracle_quantize_e4m3: invalid arguments")
+    return codes, deq
+
+
+def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, rows=None,
+                      want_lse: bool = True):
+    """Attention with Q and K quantised to e4m3 per head. Returns
+    (o [nrows, H, D], lse [nrows, H] or None, q8, k8 [T, H, D] uint8, deq [2H])."""
+    T, H, D = q.shape
+    assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
+    q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    r, n = _rows(rows)
+    n = n if r is not None else T
+    o = np.empty((n, H, D), np.float64)
+    lse = np.empty((n, H), np.float64) if want_lse else None
+    q8 = np.empty((T, H, D), np.uint8)
+    k8 = np.empty((T, H, D), np.uint8)
+    deq = np.empty(2 * H, np.float32)
+    rc = lib().oracle_varlen_attn_fp8qk(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32),
+                                        int(cu.shape[0]) - 1, T, H, D, scale, _ptr(r, C.c_int32),
+                                        n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
+                                        _ptr(q8, C.c_uint8), _ptr(k8, C.c_uint8), _ptr(deq, C.c_float))
+    if rc:
+        raise ValueError("oracle_varlen_attn_fp8qk: invalid arguments")
+    return o, lse, q8, k8, deq
 
 
 def modulate_swiglu(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, gate_res: np.ndarray,

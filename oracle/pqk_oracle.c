@@ -22,6 +22,8 @@
  *                             request, valid tokens only (first page, section
  *                             "长序列注意力与通信优化"; second page, bullet
  *                             "Long-sequence attention & communication").
+ *   oracle_varlen_attn_fp8qk -- the same attention with Q and K quantised to
+ *                             FP8 e4m3 per head (SAGE FP8, a reading).
  *   oracle_varlen_attn_skip -- the same attention with key blocks skipped
  *                             where their scores are negligible ("Skip-Softmax";
  *                             a reading, see the function).
@@ -282,6 +284,114 @@ int oracle_varlen_attn(const void* q, const void* k, const void* v, int in_kind,
     }
   }
   return bad ? -1 : 0;
+}
+
+/*
+ * FP8 e4m3 ("fn": 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,
+ * no infinities, largest finite 448, subnormal spacing 2^-9): the value of a
+ * code, and the code nearest to a float (ties to even), values beyond 448 in
+ * magnitude saturating to 448.
+ */
+static double e4m3_value(uint8_t c) {
+  const int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return sgn ? -mag : mag;
+}
+
+static uint8_t e4m3_code(float x) {
+  const uint8_t sgn = (x < 0.0f || (x == 0.0f && signbit(x))) ? 0x80 : 0;
+  double a = fabs((double)x);
+  if (a >= 448.0) return (uint8_t)(sgn | 0x7E);
+  int E;
+  frexp(a, &E);                 /* a in [2^(E-1), 2^E) */
+  int e = a > 0.0 ? E - 1 : -6;
+  if (e < -6) e = -6;           /* subnormal spacing below 2^-6 */
+  const double quantum = ldexp(1.0, e - 3);
+  const double r = rint(a / quantum) * quantum; /* ties to even: a / quantum is exact */
+  if (r == 0.0) return sgn;
+  if (r >= 448.0) return (uint8_t)(sgn | 0x7E);
+  frexp(r, &E);
+  e = E - 1;
+  if (e < -6) return (uint8_t)(sgn | (uint8_t)(r / ldexp(1.0, -9)));
+  const int mant = (int)((r / ldexp(1.0, e) - 1.0) * 8.0);
+  return (uint8_t)(sgn | (uint8_t)((e + 7) << 3) | (uint8_t)mant);
+}
+
+/*
+ * Per-head absmax quantisation of a [T, H, D] tensor to e4m3 (a reading of
+ * the SAGE FP8 attention named on the first page, bullet on TRTLLM_ATTN SAGE
+ * and Skip-Softmax: "quantise the attention computation to FP8"): for head
+ * h, amax = max |x| over all tokens and D; in float arithmetic
+ * inv = 448 / amax and code = e4m3(x * inv); the dequantisation factor is
+ * deq = amax / 448 (both 1 when amax = 0). codes: [T, H, D]; deq: [H].
+ */
+int oracle_quantize_e4m3(const void* x, int x_kind, int64_t stride_t, int64_t T, int H, int D, uint8_t* codes,
+                         float* deq) {
+  if (T < 0 || H <= 0 || D <= 0 || stride_t < (int64_t)H * D) return -1;
+  for (int h = 0; h < H; ++h) {
+    float amax = 0.0f;
+    for (int64_t t = 0; t < T; ++t)
+      for (int d = 0; d < D; ++d) {
+        const float v = (float)fabs(load(x, x_kind, t * stride_t + (int64_t)h * D + d));
+        if (v > amax) amax = v;
+      }
+    const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;
+    deq[h] = amax > 0.0f ? amax / 448.0f : 1.0f;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+      for (int d = 0; d < D; ++d) {
+        const float v = (float)load(x, x_kind, t * stride_t + (int64_t)h * D + d);
+        codes[(t * H + h) * (int64_t)D + d] = e4m3_code(v * inv);
+      }
+  }
+  return 0;
+}
+
+/*
+ * Attention with Q and K quantised to e4m3 per head (oracle_quantize_e4m3)
+ * and V, P kept at their precision: the plain attention of
+ * oracle_varlen_attn on Q~ = code(Q) * deq_Q and K~ = code(K) * deq_K.
+ * q8_out, k8_out ([T, H, D]) and deq_out ([2H]: Q's, then K's) are optional.
+ */
+int oracle_varlen_attn_fp8qk(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
+                             const int32_t* cu, int B, int64_t T, int H, int D, double scale,
+                             const int32_t* rows, int64_t nrows, double* o, double* lse, uint8_t* q8_out,
+                             uint8_t* k8_out, float* deq_out) {
+  if (check_cu(cu, B, T) || H <= 0 || D <= 0) return -1;
+  const int64_t n = T * (int64_t)H * D;
+  uint8_t* qc = q8_out ? q8_out : (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
+  uint8_t* kc = k8_out ? k8_out : (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
+  float* dq = (float*)malloc(sizeof(float) * (size_t)H * 2);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  double* kd = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  double* vd = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  int rc = oracle_quantize_e4m3(q, in_kind, stride_t, T, H, D, qc, dq);
+  if (!rc) rc = oracle_quantize_e4m3(k, in_kind, stride_t, T, H, D, kc, dq + H);
+  if (!rc) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+      for (int h = 0; h < H; ++h)
+        for (int d = 0; d < D; ++d) {
+          const int64_t i = (t * H + h) * (int64_t)D + d;
+          qd[i] = e4m3_value(qc[i]) * (double)dq[h];
+          kd[i] = e4m3_value(kc[i]) * (double)dq[H + h];
+          vd[i] = load(v, in_kind, t * stride_t + (int64_t)h * D + d);
+        }
+    rc = oracle_varlen_attn(qd, kd, vd, ORACLE_IN_F64, (int64_t)H * D, cu, B, T, H, D, scale, rows, nrows, o, lse);
+  }
+  if (deq_out) memcpy(deq_out, dq, sizeof(float) * (size_t)H * 2);
+  if (!q8_out) free(qc);
+  if (!k8_out) free(kc);
+  free(dq);
+  free(qd);
+  free(kd);
+  free(vd);
+  return rc;
+}
+
+/* e4m3 codes of a float32 array (the conversion alone, for its pins). */
+void oracle_e4m3_codes(const float* x, int64_t n, uint8_t* codes) {
+  for (int64_t i = 0; i < n; ++i) codes[i] = e4m3_code(x[i]);
 }
 
 /*

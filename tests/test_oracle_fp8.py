@@ -1,0 +1,125 @@
+"""Pins for the oracle's FP8 (e4m3) quantisation and the attention with Q and
+K in FP8 (CPU only).
+
+SAGE quantises the attention computation to FP8 ("FastH3 在八卡 B300 上实现
+完整 MP4 生成快于播放时长", bullet on TRTLLM_ATTN SAGE and Skip-Softmax). The
+quantisation here is a reading: per-head absmax scaling of Q and K to the
+e4m3 range (amax -> 448), nearest-even rounding. Checked against torch's
+float8_e4m3fn conversion (a library routine), the format's own code table,
+error bounds of a 3-bit mantissa, exact cases, and a dense brute force on
+the dequantised inputs.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle
+from tests.bruteforce import padded_masked_attention
+
+
+def e4m3_table():
+    """The 254 finite e4m3 values, from torch's decoder (codes 0x00..0xFF
+    without the two NaN codes)."""
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    return codes, vals
+
+
+def test_codes_match_torch_conversion():
+    g = np.random.default_rng(0)
+    x = np.concatenate([g.uniform(-448, 448, 100000), g.standard_normal(100000) * 0.01, g.standard_normal(50000) * 5,
+                        [0.0, -0.0, 448.0, -448.0, 460.0, 1e-3, 2.0 ** -10, 3 * 2.0 ** -10, 1.5 * 2.0 ** -9,
+                         2.5 * 2.0 ** -9, 1.0625, 1.1875, 1.0625 * 2.0 ** -6, 7.5 * 2.0 ** -9]]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_codes(x), ref)
+
+
+def test_every_code_round_trips_and_midpoints_go_to_even():
+    codes, vals = e4m3_table()
+    assert np.array_equal(oracle.e4m3_codes(vals), codes)
+    # midpoints between neighbouring positive values round to the even code
+    pos = np.sort(vals[vals > 0])
+    mid = ((pos[:-1].astype(np.float64) + pos[1:]) / 2).astype(np.float32)
+    got = oracle.e4m3_codes(mid)
+    lo = oracle.e4m3_codes(pos[:-1])
+    hi = oracle.e4m3_codes(pos[1:])
+    assert np.array_equal(got, np.where(lo % 2 == 0, lo, hi))
+
+
+def test_saturation_beyond_448():
+    x = np.array([464.0, 500.0, 1e6, -600.0, 3.0e38], np.float32)
+    assert list(oracle.e4m3_codes(x)) == [0x7E, 0x7E, 0x7E, 0xFE, 0x7E]
+
+
+def _decode(c):
+    return torch.from_numpy(np.ascontiguousarray(c)).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+
+
+def test_per_head_quantisation_bounds_and_independence():
+    g = np.random.default_rng(1)
+    T, H, D = 300, 3, 16
+    x = g.standard_normal((T, H, D))
+    x[:, 1] *= 1000.0
+    x[:, 2] = 0.0
+    codes, deq = oracle.quantize_e4m3(x)
+    amax = np.abs(x).max(axis=(0, 2))
+    assert deq[0] == np.float32(np.float32(amax[0]) / np.float32(448.0)) and deq[2] == 1.0
+    assert np.all(codes[:, 2] == 0)
+    back = _decode(codes) * deq[None, :, None]
+    # 3 stored mantissa bits: relative error <= 2^-4 in the normal range,
+    # absolute error <= 2^-10 * deq below it
+    err = np.abs(back - x)
+    assert np.all(err <= np.maximum(2.0 ** -4 * np.abs(x), 2.0 ** -10 * deq[None, :, None]) * (1 + 1e-6))
+    # the element with the largest magnitude maps to +-448
+    t, d = np.unravel_index(np.argmax(np.abs(x[:, 0])), (T, D))
+    assert codes[t, 0, d] in (0x7E, 0xFE)
+    # head 0's codes do not depend on head 1's scale
+    x2 = x.copy()
+    x2[:, 1] *= 0.001
+    assert np.array_equal(oracle.quantize_e4m3(x2)[0][:, 0], codes[:, 0])
+
+
+def test_exact_when_inputs_are_e4m3_values_with_absmax_448():
+    codes, vals = e4m3_table()
+    g = np.random.default_rng(2)
+    T, H, D = 200, 2, 16
+    q = g.choice(vals, (T, H, D)).astype(np.float64) * 0.25
+    k = g.choice(vals, (T, H, D)).astype(np.float64) * 0.5
+    q[0, :, 0] = 448.0 * 0.25
+    k[0, :, 0] = 448.0 * 0.5
+    v = g.standard_normal((T, H, D))
+    cu = np.array([0, 77, 200], np.int32)
+    o, lse, q8, k8, deq = oracle.varlen_attn_fp8qk(q, k, v, cu, 0.1)
+    assert np.allclose(deq, [0.25, 0.25, 0.5, 0.5], rtol=0, atol=0)
+    ob, lb = oracle.varlen_attn(q, k, v, cu, 0.1)
+    assert np.max(np.abs(o - ob)) <= 1e-12 and np.max(np.abs(lse - lb)) <= 1e-12
+
+
+def test_matches_bruteforce_on_dequantised_inputs():
+    g = np.random.default_rng(3)
+    T, H, D = 257, 2, 32
+    q, k, v = (g.standard_normal((T, H, D)) for _ in range(3))
+    cu = np.array([0, 1, 130, 257], np.int32)
+    scale = 1.0 / math.sqrt(D)
+    o, lse, q8, k8, deq = oracle.varlen_attn_fp8qk(q, k, v, cu, scale)
+    qd = _decode(q8) * deq[None, :H, None]
+    kd = _decode(k8) * deq[None, H:, None]
+    ob, lb = padded_masked_attention(qd, kd, v, cu, scale)
+    assert np.max(np.abs(o - ob)) <= 1e-12 and np.max(np.abs(lse - lb)) <= 1e-12
+    # and it is not the unquantised attention
+    op, _ = oracle.varlen_attn(q, k, v, cu, scale)
+    assert np.max(np.abs(o - op)) > 1e-4
+
+
+def test_sampled_rows_equal_full_evaluation():
+    g = np.random.default_rng(4)
+    T, H, D = 300, 2, 16
+    q, k, v = (g.standard_normal((T, H, D)) for _ in range(3))
+    cu = np.array([0, 300], np.int32)
+    o, lse, q8, _, _ = oracle.varlen_attn_fp8qk(q, k, v, cu, 0.25)
+    rows = np.array([0, 5, 299], np.int32)
+    o2, l2, q82, _, _ = oracle.varlen_attn_fp8qk(q, k, v, cu, 0.25, rows=rows)
+    assert np.array_equal(o2, o[rows]) and np.array_equal(l2, lse[rows]) and np.array_equal(q82, q8)

@@ -15,8 +15,8 @@ import subprocess
 import pytest
 
 from oracle import oracle
-from tests import (test_oracle_attention, test_oracle_fullc, test_oracle_modulate, test_oracle_norm_rope,
-                   test_oracle_rope3, test_oracle_skip)
+from tests import (test_oracle_attention, test_oracle_fp8, test_oracle_fullc, test_oracle_modulate,
+                   test_oracle_norm_rope, test_oracle_rope3, test_oracle_skip)
 
 MUTANTS = {
     "attn_drop_scale": ("s[j] = scale * acc;", "s[j] = acc;"),
@@ -54,6 +54,15 @@ MUTANTS = {
     "skip_query_block_64": ("#define ORACLE_SKIP_QROWS 32", "#define ORACLE_SKIP_QROWS 64"),
     "skip_threshold_sign": ("if (!(tmax[i * nkb + jb] < M - tau)) skip = 0;", "if (!(tmax[i * nkb + jb] < M + tau)) skip = 0;"),
     "skip_natural_log_units": ("const double u = scale * dot / log(2.0);", "const double u = scale * dot;"),
+    "e4m3_ties_away_from_zero": ("const double r = rint(a / quantum) * quantum;",
+                                 "const double r = round(a / quantum) * quantum;"),
+    "e4m3_two_mantissa_bits": ("const double quantum = ldexp(1.0, e - 3);", "const double quantum = ldexp(1.0, e - 2);"),
+    "fp8_k_dequantised_with_q_scale": ("kd[i] = e4m3_value(kc[i]) * (double)dq[H + h];",
+                                       "kd[i] = e4m3_value(kc[i]) * (double)dq[h];"),
+    "fp8_amax_of_first_token": ("    for (int64_t t = 0; t < T; ++t)\n      for (int d = 0; d < D; ++d) {\n        const float v = (float)fabs(",
+                                "    for (int64_t t = 0; t < 1; ++t)\n      for (int d = 0; d < D; ++d) {\n        const float v = (float)fabs("),
+    "fp8_range_240": ("const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;",
+                      "const float inv = amax > 0.0f ? 240.0f / amax : 1.0f;"),
     "skip_tile_counts_any_block": ("if (keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;",
                                    "if (!keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;"),
 }
@@ -61,7 +70,7 @@ MUTANTS = {
 
 def _pin_calls():
     for mod in (test_oracle_attention, test_oracle_norm_rope, test_oracle_modulate, test_oracle_rope3,
-                test_oracle_fullc, test_oracle_skip):
+                test_oracle_fullc, test_oracle_skip, test_oracle_fp8):
         for name, fn in inspect.getmembers(mod, inspect.isfunction):
             if not name.startswith("test_") or fn.__module__ != mod.__name__:
                 continue
