@@ -59,6 +59,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="leave out the FP8 Q K^T attention timing")
     ap.add_argument("--skip-tau", type=float, default=8.0,
                     help="threshold (log2 units) of the block-skipping attention timed on the local-attention "
                          "stand-in after the steps; negative = leave that timing out")
@@ -409,6 +410,34 @@ def run_ours(args, w):
                 "skipped_pv_share": c[1] / n128}
         del lq, lk, lv, lo, lx
 
+    # FP8 Q K^T (the SAGE reading): the step's normalised Q, K quantised per
+    # head to e4m3, then the attention with S = Q K^T on the FP8 tensor cores
+    fp8 = None
+    if not args.no_fp8 and w.D == 128:
+        q8, k8, deq = pqk.quantize_qk_e4m3(o["qn"], o["kn"])
+        fo = torch.empty_like(o["o"])
+        fp8_attn = lambda: pqk.varlen_attn_fwd_fp8qk(q8, k8, d["v"], deq, d["cu"], o=fo, workspace=o["ws"])
+        fp8_attn()
+        torch.cuda.synchronize()
+        ev3[0].record()
+        for _ in range(reps3):
+            pqk.quantize_qk_e4m3(o["qn"], o["kn"], q8=q8, k8=k8, scales=None)
+        ev3[1].record()
+        torch.cuda.synchronize()
+        quant_us = ev3[0].elapsed_time(ev3[1]) / reps3 * 1e3
+        ev3[0].record()
+        for _ in range(3):
+            fp8_attn()
+        ev3[1].record()
+        torch.cuda.synchronize()
+        fp8_ms = ev3[0].elapsed_time(ev3[1]) / 3
+        if pqk.get_device_status() != 0:
+            raise RuntimeError("device status set during the FP8 timing")
+        fp8 = {"quantize_us": quant_us, "attn_ms": fp8_ms, "attn_tflops": flops / (fp8_ms * 1e-3) / 1e12,
+               "speedup_vs_bf16": att_ms / fp8_ms,
+               "quantize_gbs": (4 * w.T * w.H * w.D + 2 * w.T * w.H * w.D) / (quant_us * 1e-6) / 1e9}
+        del q8, k8, fo
+
     # e2e through host buffers: every step copies all of its inputs from
     # pinned host memory to the device (H2D stream), runs the three C-ABI
     # calls (compute stream) and copies its outputs x', h, act back to pinned
@@ -509,7 +538,7 @@ def run_ours(args, w):
                     "qk_norm_rope_back_to_back_us": rope1_b2b_us,
                     "qk_fullc_norm_rope_us": fullc_us, "qk_fullc_norm_rope_gbs": fullc_gbs,
                     "qk_fullc_norm_rope_frac_hbm": fullc_gbs / pk["hbm_gbs"],
-                    "varlen_attn_skip": skip},
+                    "varlen_attn_skip": skip, "varlen_attn_fp8qk": fp8},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * K,

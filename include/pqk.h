@@ -209,6 +209,44 @@ PQK_API int pqk_varlen_attn_fwd_skip(const void* q, const void* k, const void* v
                              void* stream);
 
 /*
+ * pqk_quantize_qk_e4m3 -- Q and K to FP8 e4m3 for pqk_varlen_attn_fwd_fp8qk
+ * (SAGE quantises the attention computation to FP8: first page, bullet on
+ * TRTLLM_ATTN SAGE and Skip-Softmax; second page, bullet "Sparse & quantized
+ * attention"). The pages give no scheme; the one implemented: per head h of
+ * each tensor, amax = max |x| over all T tokens and D, code = e4m3(x * (448 /
+ * amax)) rounded to nearest even, saturating at +-448 (e4m3 "fn": 4
+ * exponent bits with bias 7, 3 mantissa bits, no infinities); the
+ * dequantisation factor is amax / 448 (1 for an all-zero head).
+ *
+ * q, k      device bf16 [T, H, D], q_stride_t / k_stride_t elements between
+ *           tokens (>= H*D, multiples of 8), 16-byte aligned.
+ * q8, k8    device [T, H, D] bytes, contiguous, 16-byte aligned.
+ * scales    device fp32 [4H], 16-byte aligned: [0, 2H) scratch, [2H, 3H) Q's
+ *           and [3H, 4H) K's dequantisation factors (pass scales + 2H as
+ *           `deq` to the attention). H <= 4096; D 64 or 128.
+ */
+PQK_API int pqk_quantize_qk_e4m3(const void* q, const void* k, int64_t q_stride_t, int64_t k_stride_t, int64_t T,
+                         int H, int D, void* q8, void* k8, float* scales, void* stream);
+
+/*
+ * pqk_varlen_attn_fwd_fp8qk -- pqk_varlen_attn_fwd with S = Q K^T taken on
+ * the FP8 tensor cores from e4m3 Q and K (pqk_quantize_qk_e4m3): for every
+ * token t of request i and head h,
+ *   s(t, j) = softmax_scale * deq[h] * deq[H + h] * <q8[t, h], k8[j, h]>,
+ * then softmax and P V exactly as pqk_varlen_attn_fwd (P rounded to bf16, V
+ * bf16, fp32 accumulation).
+ *
+ * q8, k8    device e4m3 [T, H, D] bytes, contiguous, 16-byte aligned.
+ * deq       device fp32 [2H]: Q's then K's per-head dequantisation factors.
+ * v, o, lse, cu_seqlens, workspace: as pqk_varlen_attn_fwd. D must be 128
+ * (PQK_ERR_UNSUPPORTED otherwise).
+ */
+PQK_API int pqk_varlen_attn_fwd_fp8qk(const void* q8, const void* k8, const void* v, const float* deq, void* o,
+                              float* lse, int64_t v_stride_t, int64_t o_stride_t,
+                              const int32_t* cu_seqlens, int B, int64_t T, int H, int D,
+                              float softmax_scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * pqk_varlen_attn_fwd_noalloc -- pqk_varlen_attn_fwd for callers that cannot
  * allocate device memory. The pages have no counterpart: this entry point
  * exists for callers such as plugins or embedded runtimes that are handed

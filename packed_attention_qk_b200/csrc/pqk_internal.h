@@ -32,13 +32,23 @@ size_t attn_schedule_bytes(int B);
 // Prepares and enqueues the attention kernel's TMA descriptors, the schedule
 // builder and the persistent attention kernel. skip selects the block-
 // skipping kernel (threshold skip_tau in log2 units; skip_counts nullable,
-// two device counters the kernel adds to). Returns 0, or -1 when a CUDA call
-// failed, -2 when the tensor maps could not be encoded.
+// two device counters the kernel adds to). deq non-null selects the kernel
+// with Q, K given as e4m3 bytes ([T, H, D], strides in bytes) and deq their
+// [2H] per-head dequantisation factors (D = 128, no skipping). Returns 0, or
+// -1 when a CUDA call failed, -2 when the tensor maps could not be encoded.
 int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, float* lse, int64_t q_stride,
                        int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
                        int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
                        long long timeout_ns, cudaStream_t stream, int num_sms, bool skip = false,
-                       float skip_tau = 0.0f, unsigned long long* skip_counts = nullptr);
+                       float skip_tau = 0.0f, unsigned long long* skip_counts = nullptr,
+                       const float* deq = nullptr);
+
+// Per-head absmax e4m3 quantisation of Q and K ([T, H, D] bf16, strides in
+// elements) into q8, k8 ([T, H, D] bytes, contiguous). scales: [4H] floats,
+// [0, 2H) scratch (absmax bits), [2H, 4H) the dequantisation factors (Q's
+// heads, then K's). D is 64 or 128.
+int launch_quantize_qk_e4m3(const void* q, const void* k, int64_t q_stride, int64_t k_stride, int64_t T, int H,
+                            int D, void* q8, void* k8, float* scales, cudaStream_t stream, int num_sms);
 
 int launch_wait_selftest(int* status, long long timeout_ns, cudaStream_t stream);
 

@@ -110,6 +110,7 @@ struct AttnParams {
   int* status;
   long long timeout_ns;
   float skip_tau;                        // block-skip threshold (log2 units), kSkip only
+  const float* deq;                      // kFp8: [2H] dequantisation factors of Q's, then K's heads
   unsigned long long* skip_counts;       // nullable: [0] skipped warp blocks, [1] skipped O += P V products
 };
 
@@ -305,11 +306,14 @@ __device__ __forceinline__ float exp_tile_store(const float (&s)[128], float sca
   return (l0 + l1) + (l2 + l3);
 }
 
-template <int D, bool kSkip>
+template <int D, bool kSkip, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using L = Layout<D>;
+  static_assert(!kFp8 || D == 128, "FP8 Q K^T: one 128-byte swizzle row per token");
+  // bytes of one Q or K tile: bf16 slabs, or 128 rows x 128 e4m3 bytes
+  constexpr uint32_t kQKBytes = kFp8 ? static_cast<uint32_t>(kBM) * 128u : static_cast<uint32_t>(L::kTileBytes);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -371,22 +375,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
         const Work wk = decode_work(p.sched, p.H, w);
         if (wt > 0 && !(ok = mbar_wait(q_empty, (wt - 1) & 1, abort_flag, p.timeout_ns))) break;
-        mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+        mbar_arrive_expect_tx(q_full, 2 * kQKBytes);
         ++q_loads;
-        for (int i = 0; i < 2; ++i)
-          for (int sl = 0; sl < L::kSlabs; ++sl)
-            tma_load_3d(q_smem + i * L::kTileBytes + sl * kSlabBytes, &tm_q, q_full, sl * 64, wk.head,
-                        wk.q0 + i * kBM);
+        for (int i = 0; i < 2; ++i) {
+          if constexpr (kFp8) {
+            tma_load_3d(q_smem + i * L::kTileBytes, &tm_q, q_full, 0, wk.head, wk.q0 + i * kBM);
+          } else {
+            for (int sl = 0; sl < L::kSlabs; ++sl)
+              tma_load_3d(q_smem + i * L::kTileBytes + sl * kSlabBytes, &tm_q, q_full, sl * 64, wk.head,
+                          wk.q0 + i * kBM);
+          }
+        }
         for (int j = 0; j < wk.n_kv && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv) {
             const int s = load_idx % L::kStages;
             const uint32_t round = load_idx / L::kStages;
             if (round > 0 && !(ok = mbar_wait(kv_empty(s), (round - 1) & 1, abort_flag, p.timeout_ns))) break;
-            mbar_arrive_expect_tx(kv_full(s), L::kTileBytes);
-            const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
-            for (int sl = 0; sl < L::kSlabs; ++sl)
-              tma_load_3d(kv_smem + s * L::kTileBytes + sl * kSlabBytes, tm, kv_full(s), sl * 64, wk.head,
-                          wk.seg_start + j * kBN);
+            if (kFp8 && kv == 0) {
+              mbar_arrive_expect_tx(kv_full(s), kQKBytes);
+              tma_load_3d(kv_smem + s * L::kTileBytes, &tm_k, kv_full(s), 0, wk.head, wk.seg_start + j * kBN);
+            } else {
+              mbar_arrive_expect_tx(kv_full(s), L::kTileBytes);
+              const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
+              for (int sl = 0; sl < L::kSlabs; ++sl)
+                tma_load_3d(kv_smem + s * L::kTileBytes + sl * kSlabBytes, tm, kv_full(s), sl * 64, wk.head,
+                            wk.seg_start + j * kBN);
+            }
             ++load_idx;
           }
         }
@@ -408,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t kIdescQK = kFp8 ? idesc_e4m3_f32(kBM, kBN) : idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
       uint32_t cons_idx = 0;
       uint32_t p_phase = 0;
@@ -430,11 +444,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_qk = [&](int i, int stage) {
         const uint32_t a0 = q_lo + i * kTileWords;
         const uint32_t b0 = k_lo + stage * kTileWords;
+        if constexpr (kFp8) {
+          // e4m3: K = 32 per instruction, 32 bytes inside the one 128-byte row
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = ((k / 4) * kSlabBytes + (k % 4) * 32) >> 4;
-          mma_bf16_ss_w(tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1), a0 + off, b0 + off, kDescHi, kIdescQK,
+          for (int k = 0; k < D / 32; ++k)
+            mma_f8_ss_w(tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1), a0 + 2 * k, b0 + 2 * k, kDescHi, kIdescQK,
                         k > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = ((k / 4) * kSlabBytes + (k % 4) * 32) >> 4;
+            mma_bf16_ss_w(tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1), a0 + off, b0 + off, kDescHi, kIdescQK,
+                          k > 0 ? 1u : 0u);
+          }
         }
       };
       // O_i (+)= P_i V over kBN/16 K-steps; V is MN-major: 64-wide column
@@ -530,6 +552,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
       const Work wk = decode_work(p.sched, p.H, w);
       const int row = wk.q0 + grp * kBM + r;
+      // log2-domain score factor; FP8 scores carry the two heads' dequantisation factors
+      const float sl2 = kFp8 ? p.scale_log2 * p.deq[wk.head] * p.deq[p.H + wk.head] : p.scale_log2;
       float m = -INFINITY, l = 0.f;
       float m_seen = -INFINITY;  // block skipping: running maximum over all earlier tiles
       for (int j = 0; j < wk.n_kv; ++j) {
@@ -541,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int valid = j == wk.n_kv - 1 ? wk.seg_len - j * kBN : kBN;
         float s[128];
         load_scores(t_s, valid, s);
-        const float mx = row_max(s) * p.scale_log2;
+        const float mx = row_max(s) * sl2;
         if constexpr (kSkip) {
           // Skip-Softmax: this warp's 32 rows drop K/V tile j when every row
           // of the request has its tile maximum more than skip_tau below its
@@ -587,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_x32(t_o + c0, ov);
           }
         }
-        l += exp_tile_store(s, p.scale_log2, -m, t_s);
+        l += exp_tile_store(s, sl2, -m, t_s);
         tc_fence_before_sync();
         mbar_arrive(p_full(grp));
       }
@@ -680,13 +704,27 @@ bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t T, int H, int D, in
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool kSkip>
+// [T, H, D] e4m3 bytes with `stride` elements (bytes) between tokens, read
+// as boxes of 128 bytes x 1 head x 128 tokens, 128-byte swizzled.
+bool make_e4m3_map(CUtensorMap* map, const void* ptr, int64_t T, int H, int D, int64_t stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr || D != 128) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(stride)};
+  const cuuint32_t box[3] = {128, 1, static_cast<cuuint32_t>(kBM)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool kSkip, bool kFp8>
 bool set_smem_attr() {
   static int done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kSkip>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kSkip, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Layout<D>::kAlloc) != cudaSuccess)
       return false;
     done[dev] = 1;
@@ -702,11 +740,12 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
                        int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
                        int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
                        long long timeout_ns, cudaStream_t stream, int num_sms, bool skip, float skip_tau,
-                       unsigned long long* skip_counts) {
+                       unsigned long long* skip_counts, const float* deq) {
   CUtensorMap tq, tk, tv;
-  if (!make_qkv_map(&tq, q, T, H, D, q_stride) || !make_qkv_map(&tk, k, T, H, D, k_stride) ||
-      !make_qkv_map(&tv, v, T, H, D, v_stride))
-    return -2;
+  const bool maps_ok = deq != nullptr
+                           ? make_e4m3_map(&tq, q, T, H, D, q_stride) && make_e4m3_map(&tk, k, T, H, D, k_stride)
+                           : make_qkv_map(&tq, q, T, H, D, q_stride) && make_qkv_map(&tk, k, T, H, D, k_stride);
+  if (!maps_ok || !make_qkv_map(&tv, v, T, H, D, v_stride)) return -2;
   int32_t* sched = static_cast<int32_t*>(workspace);
   build_schedule_kernel<<<1, kSchedThreads, 0, stream>>>(cu_seqlens, B, T, H, sched, status);
   if (cudaGetLastError() != cudaSuccess) return -1;
@@ -722,21 +761,26 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
   p.timeout_ns = timeout_ns;
   p.skip_tau = skip_tau;
   p.skip_counts = skip_counts;
+  p.deq = deq;
   // upper bound of work tiles: every request adds at most one partial block
   const int64_t max_work = static_cast<int64_t>(H) * ((T + kRowsPerWork - 1) / kRowsPerWork + B);
   const int grid = static_cast<int>(max_work < num_sms ? max_work : num_sms);
-  if (D == 128 && !skip) {
-    if (!set_smem_attr<128, false>()) return -1;
-    attn_fwd_kernel<128, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+  if (deq != nullptr) {
+    if (D != 128 || skip) return -1;
+    if (!set_smem_attr<128, false, true>()) return -1;
+    attn_fwd_kernel<128, false, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+  } else if (D == 128 && !skip) {
+    if (!set_smem_attr<128, false, false>()) return -1;
+    attn_fwd_kernel<128, false, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
   } else if (D == 128) {
-    if (!set_smem_attr<128, true>()) return -1;
-    attn_fwd_kernel<128, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<128, true, false>()) return -1;
+    attn_fwd_kernel<128, true, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
   } else if (!skip) {
-    if (!set_smem_attr<64, false>()) return -1;
-    attn_fwd_kernel<64, false><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<64, false, false>()) return -1;
+    attn_fwd_kernel<64, false, false><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
   } else {
-    if (!set_smem_attr<64, true>()) return -1;
-    attn_fwd_kernel<64, true><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<64, true, false>()) return -1;
+    attn_fwd_kernel<64, true, false><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

@@ -22,7 +22,8 @@ NORM_RMS, NORM_LAYER, NORM_NONE = 0, 1, 2
 
 # every symbol include/pqk.h declares
 EXPORTS = ("pqk_qk_norm_rope", "pqk_qk_norm_rope_3axis", "pqk_qk_fullc_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd",
-           "pqk_varlen_attn_fwd_skip", "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu",
+           "pqk_varlen_attn_fwd_skip", "pqk_quantize_qk_e4m3", "pqk_varlen_attn_fwd_fp8qk",
+           "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu",
            "pqk_get_device_status", "pqk_set_wait_timeout_ns", "pqk_selftest_wait_timeout", "pqk_status_string",
            "pqk_version")
 
@@ -62,6 +63,11 @@ def lib(path: str | None = None) -> C.CDLL:
     L.pqk_varlen_attn_fwd_skip.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32, f32,
                                            vp, vp, sz, vp]
     L.pqk_varlen_attn_fwd_skip.restype = i32
+    L.pqk_quantize_qk_e4m3.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp]
+    L.pqk_quantize_qk_e4m3.restype = i32
+    L.pqk_varlen_attn_fwd_fp8qk.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, vp, i32, i64, i32, i32, f32, vp, sz,
+                                            vp]
+    L.pqk_varlen_attn_fwd_fp8qk.restype = i32
     L.pqk_varlen_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32,
                                               vp]
     L.pqk_varlen_attn_fwd_noalloc.restype = i32
@@ -211,6 +217,47 @@ def varlen_attn_fwd_skip(q, k, v, cu_seqlens, skip_threshold_log2: float, *, sof
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _token_stride(q, 3), _token_stride(k, 3),
         _token_stride(v, 3), _token_stride(o, 3), _ptr(cu_seqlens), B, T, H, D, scale, float(skip_threshold_log2),
         _ptr(skip_counts), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+def quantize_qk_e4m3(q, k, *, q8=None, k8=None, scales=None, stream=None):
+    """Per-head absmax e4m3 quantisation of Q and K (bf16 [T, H, D]).
+    Returns (q8, k8 uint8 [T, H, D], deq fp32 [2H] view of ``scales``)."""
+    import torch
+    T, H, D = q.shape
+    if q8 is None:
+        q8 = torch.empty((T, H, D), dtype=torch.uint8, device=q.device)
+    if k8 is None:
+        k8 = torch.empty((T, H, D), dtype=torch.uint8, device=q.device)
+    if scales is None:
+        scales = torch.empty(4 * H, dtype=torch.float32, device=q.device)
+    assert q8.is_contiguous() and k8.is_contiguous() and scales.numel() >= 4 * H
+    _check("pqk_quantize_qk_e4m3", lib().pqk_quantize_qk_e4m3(
+        _ptr(q), _ptr(k), _token_stride(q, 3), _token_stride(k, 3), T, H, D, _ptr(q8), _ptr(k8), _ptr(scales),
+        _stream(stream)))
+    return q8, k8, scales[2 * H:4 * H]
+
+
+def varlen_attn_fwd_fp8qk(q8, k8, v, deq, cu_seqlens, *, softmax_scale: float | None = None, o=None, lse=None,
+                          workspace=None, want_lse: bool = False, stream=None):
+    """Packed varlen attention with Q K^T on the FP8 tensor cores: q8, k8
+    e4m3 bytes [T, H, D] (quantize_qk_e4m3), deq fp32 [2H], v bf16.
+    Returns (o, lse or None)."""
+    import torch
+    T, H, D = v.shape
+    B = cu_seqlens.shape[0] - 1
+    scale = softmax_scale if softmax_scale is not None else D ** -0.5
+    if o is None:
+        o = torch.empty((T, H, D), dtype=v.dtype, device=v.device)
+    if lse is None and want_lse:
+        lse = torch.empty((H, T), dtype=torch.float32, device=v.device)
+    if workspace is None:
+        workspace = torch.empty(varlen_attn_workspace_size(B), dtype=torch.uint8, device=v.device)
+    assert q8.is_contiguous() and k8.is_contiguous() and tuple(q8.shape) == (T, H, D) == tuple(k8.shape)
+    _check("pqk_varlen_attn_fwd_fp8qk", lib().pqk_varlen_attn_fwd_fp8qk(
+        _ptr(q8), _ptr(k8), _ptr(v), _ptr(deq), _ptr(o), _ptr(lse), _token_stride(v, 3), _token_stride(o, 3),
+        _ptr(cu_seqlens), B, T, H, D, scale, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
     return o, lse
 
 

@@ -190,3 +190,37 @@ def test_varlen_attn_skip_host_errors(L):
     assert attn_skip(L, ws=None) == ERR_WORKSPACE
     assert attn_skip(L, T=0, q=None) == 0
     assert attn_skip(L, T=0, q=None, tau=float("inf")) == 0
+
+
+def test_quantize_qk_e4m3_host_errors(L):
+    def call(**kw):
+        a = dict(q=A, k=A, qs=1024, ks=1024, T=16, H=8, D=128, q8=A, k8=A, sc=A)
+        a.update(kw)
+        return L.pqk_quantize_qk_e4m3(a["q"], a["k"], a["qs"], a["ks"], a["T"], a["H"], a["D"], a["q8"], a["k8"],
+                                      a["sc"], None)
+    assert call(D=96) == ERR_UNSUPPORTED
+    assert call(H=0) == ERR_INVALID
+    assert call(H=5000, qs=5000 * 128, ks=5000 * 128) == ERR_INVALID
+    assert call(qs=1000) == ERR_INVALID
+    assert call(sc=None) == ERR_INVALID
+    assert call(q8=U) == ERR_MISALIGNED
+    assert call(sc=U) == ERR_MISALIGNED
+    assert call(ks=1028) == ERR_MISALIGNED
+
+
+def test_varlen_attn_fp8qk_host_errors(L):
+    def call(**kw):
+        a = dict(q8=A, k8=A, v=A, deq=A, o=A, lse=None, vs=1024, os_=1024, cu=A, B=2, T=512, H=8, D=128,
+                 scale=0.088, ws=A, wsb=4096)
+        a.update(kw)
+        return L.pqk_varlen_attn_fwd_fp8qk(a["q8"], a["k8"], a["v"], a["deq"], a["o"], a["lse"], a["vs"], a["os_"],
+                                           a["cu"], a["B"], a["T"], a["H"], a["D"], a["scale"], a["ws"], a["wsb"],
+                                           None)
+    assert call(D=64, vs=512, os_=512) == ERR_UNSUPPORTED
+    assert call(deq=None) == ERR_INVALID
+    assert call(B=0) == ERR_INVALID
+    assert call(vs=512) == ERR_INVALID
+    assert call(k8=U) == ERR_MISALIGNED
+    assert call(deq=A + 2) == ERR_MISALIGNED
+    assert call(ws=None) == ERR_WORKSPACE
+    assert call(T=0, q8=None) == 0
