@@ -398,6 +398,25 @@ def run_ours(args, w):
             times[name] = ev3[0].elapsed_time(ev3[1]) / 3
         if pqk.get_device_status() != 0:
             raise RuntimeError("device status set during the block-skipping timing")
+        # the same with Q K^T in FP8 (SAGE reading), without and with skipping
+        fp8_times = {}
+        if w.D == 128:
+            q8, k8, deq = pqk.quantize_qk_e4m3(lq, lk)
+            fp8_plain = lambda: pqk.varlen_attn_fwd_fp8qk(q8, k8, lv, deq, d["cu"], o=lo, workspace=o["ws"])
+            fp8_skip = lambda: pqk.varlen_attn_fwd_fp8qk(q8, k8, lv, deq, d["cu"], o=lo, workspace=o["ws"],
+                                                         skip_threshold_log2=args.skip_tau)
+            fp8_plain()
+            fp8_skip()
+            torch.cuda.synchronize()
+            for name, fn in (("fp8", fp8_plain), ("fp8_skip", fp8_skip), ("fp8_2", fp8_plain),
+                             ("fp8_skip_2", fp8_skip)):
+                ev3[0].record()
+                for _ in range(3):
+                    fn()
+                ev3[1].record()
+                torch.cuda.synchronize()
+                fp8_times[name] = ev3[0].elapsed_time(ev3[1]) / 3
+            del q8, k8
         c = counts.cpu().tolist()
         n32 = sum(((L + 31) // 32) * ((L + 127) // 128) for L in w.seg_lens) * w.H
         n128 = sum(((L + 127) // 128) ** 2 for L in w.seg_lens) * w.H
@@ -408,6 +427,10 @@ def run_ours(args, w):
                 "tau_log2": args.skip_tau, "plain_ms": plain_ms, "skip_ms": skip_ms,
                 "speedup": plain_ms / skip_ms, "dropped_block_share": c[0] / n32,
                 "skipped_pv_share": c[1] / n128}
+        if fp8_times:
+            f_ms = min(fp8_times["fp8"], fp8_times["fp8_2"])
+            fs_ms = min(fp8_times["fp8_skip"], fp8_times["fp8_skip_2"])
+            skip.update({"fp8qk_ms": f_ms, "fp8qk_skip_ms": fs_ms, "speedup_fp8qk_skip_vs_plain": plain_ms / fs_ms})
         del lq, lk, lv, lo, lx
 
     # FP8 Q K^T (the SAGE reading): the step's normalised Q, K quantised per

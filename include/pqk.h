@@ -238,13 +238,18 @@ PQK_API int pqk_quantize_qk_e4m3(const void* q, const void* k, int64_t q_stride_
  *
  * q8, k8    device e4m3 [T, H, D] bytes, contiguous, 16-byte aligned.
  * deq       device fp32 [2H]: Q's then K's per-head dequantisation factors.
+ * skip_threshold_log2, skip_counts: block skipping as pqk_varlen_attn_fwd_skip,
+ *           decided on these FP8 scores; +inf skips nothing (and counts
+ *           nothing).
  * v, o, lse, cu_seqlens, workspace: as pqk_varlen_attn_fwd. D must be 128
  * (PQK_ERR_UNSUPPORTED otherwise).
  */
 PQK_API int pqk_varlen_attn_fwd_fp8qk(const void* q8, const void* k8, const void* v, const float* deq, void* o,
                               float* lse, int64_t v_stride_t, int64_t o_stride_t,
                               const int32_t* cu_seqlens, int B, int64_t T, int H, int D,
-                              float softmax_scale, void* workspace, size_t workspace_bytes, void* stream);
+                              float softmax_scale, float skip_threshold_log2,
+                              unsigned long long* skip_counts, void* workspace, size_t workspace_bytes,
+                              void* stream);
 
 /*
  * pqk_varlen_attn_fwd_noalloc -- pqk_varlen_attn_fwd for callers that cannot

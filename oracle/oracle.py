@@ -9,6 +9,7 @@ float64); outputs are float64.
 from __future__ import annotations
 
 import ctypes as C
+import math
 import os
 import subprocess
 import threading
@@ -58,7 +59,8 @@ def load(path: str):
     u8p = C.POINTER(C.c_uint8)
     L.oracle_quantize_e4m3.argtypes = [vp, C.c_int, C.c_int64, C.c_int64, C.c_int, C.c_int, u8p, f32p]
     L.oracle_varlen_attn_fp8qk.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
-                                           C.c_int, C.c_double, i32p, C.c_int64, f64p, f64p, u8p, u8p, f32p]
+                                           C.c_int, C.c_double, C.c_double, i32p, C.c_int64, f64p, f64p,
+                                           C.POINTER(C.c_int64), u8p, u8p, f32p]
     L.oracle_e4m3_codes.argtypes = [f32p, C.c_int64, u8p]
     L.oracle_e4m3_codes.restype = None
     for f in (L.oracle_qk_norm_rope, L.oracle_qk_norm_rope_3axis, L.oracle_qk_fullc_norm_rope, L.oracle_varlen_attn,
@@ -226,9 +228,11 @@ def quantize_e4m3(x: np.ndarray):
 
 
 def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, rows=None,
-                      want_lse: bool = True):
-    """Attention with Q and K quantised to e4m3 per head. Returns
-    (o [nrows, H, D], lse [nrows, H] or None, q8, k8 [T, H, D] uint8, deq [2H])."""
+                      want_lse: bool = True, tau: float = math.inf, counts_out: list | None = None):
+    """Attention with Q and K quantised to e4m3 per head (block skipping on
+    the quantised scores for a finite tau; its counts appended to counts_out
+    when given). Returns (o [nrows, H, D], lse [nrows, H] or None, q8, k8
+    [T, H, D] uint8, deq [2H])."""
     T, H, D = q.shape
     assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
     q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
@@ -240,12 +244,16 @@ def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: n
     q8 = np.empty((T, H, D), np.uint8)
     k8 = np.empty((T, H, D), np.uint8)
     deq = np.empty(2 * H, np.float32)
+    counts = np.zeros(2, np.int64)
     rc = lib().oracle_varlen_attn_fp8qk(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32),
-                                        int(cu.shape[0]) - 1, T, H, D, scale, _ptr(r, C.c_int32),
+                                        int(cu.shape[0]) - 1, T, H, D, scale, float(tau), _ptr(r, C.c_int32),
                                         n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
-                                        _ptr(q8, C.c_uint8), _ptr(k8, C.c_uint8), _ptr(deq, C.c_float))
+                                        _ptr(counts, C.c_int64), _ptr(q8, C.c_uint8), _ptr(k8, C.c_uint8),
+                                        _ptr(deq, C.c_float))
     if rc:
         raise ValueError("oracle_varlen_attn_fp8qk: invalid arguments")
+    if counts_out is not None and r is None:
+        counts_out.append(tuple(int(c) for c in counts))
     return o, lse, q8, k8, deq
 
 

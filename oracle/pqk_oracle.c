@@ -347,16 +347,22 @@ int oracle_quantize_e4m3(const void* x, int x_kind, int64_t stride_t, int64_t T,
   return 0;
 }
 
+int oracle_varlen_attn_skip(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
+                            const int32_t* cu, int B, int64_t T, int H, int D, double scale, double tau,
+                            const int32_t* rows, int64_t nrows, double* o, double* lse, int64_t* counts);
+
 /*
  * Attention with Q and K quantised to e4m3 per head (oracle_quantize_e4m3)
  * and V, P kept at their precision: the plain attention of
- * oracle_varlen_attn on Q~ = code(Q) * deq_Q and K~ = code(K) * deq_K.
- * q8_out, k8_out ([T, H, D]) and deq_out ([2H]: Q's, then K's) are optional.
+ * oracle_varlen_attn on Q~ = code(Q) * deq_Q and K~ = code(K) * deq_K, or,
+ * for a finite tau, the block-skipping attention of oracle_varlen_attn_skip
+ * on them (counts as there). q8_out, k8_out ([T, H, D]) and deq_out ([2H]:
+ * Q's, then K's) are optional.
  */
 int oracle_varlen_attn_fp8qk(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
-                             const int32_t* cu, int B, int64_t T, int H, int D, double scale,
-                             const int32_t* rows, int64_t nrows, double* o, double* lse, uint8_t* q8_out,
-                             uint8_t* k8_out, float* deq_out) {
+                             const int32_t* cu, int B, int64_t T, int H, int D, double scale, double tau,
+                             const int32_t* rows, int64_t nrows, double* o, double* lse, int64_t* counts,
+                             uint8_t* q8_out, uint8_t* k8_out, float* deq_out) {
   if (check_cu(cu, B, T) || H <= 0 || D <= 0) return -1;
   const int64_t n = T * (int64_t)H * D;
   uint8_t* qc = q8_out ? q8_out : (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
@@ -377,7 +383,11 @@ int oracle_varlen_attn_fp8qk(const void* q, const void* k, const void* v, int in
           kd[i] = e4m3_value(kc[i]) * (double)dq[H + h];
           vd[i] = load(v, in_kind, t * stride_t + (int64_t)h * D + d);
         }
-    rc = oracle_varlen_attn(qd, kd, vd, ORACLE_IN_F64, (int64_t)H * D, cu, B, T, H, D, scale, rows, nrows, o, lse);
+    if (isinf(tau) && tau > 0)
+      rc = oracle_varlen_attn(qd, kd, vd, ORACLE_IN_F64, (int64_t)H * D, cu, B, T, H, D, scale, rows, nrows, o, lse);
+    else
+      rc = oracle_varlen_attn_skip(qd, kd, vd, ORACLE_IN_F64, (int64_t)H * D, cu, B, T, H, D, scale, tau, rows,
+                                   nrows, o, lse, counts);
   }
   if (deq_out) memcpy(deq_out, dq, sizeof(float) * (size_t)H * 2);
   if (!q8_out) free(qc);

@@ -765,10 +765,14 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
   // upper bound of work tiles: every request adds at most one partial block
   const int64_t max_work = static_cast<int64_t>(H) * ((T + kRowsPerWork - 1) / kRowsPerWork + B);
   const int grid = static_cast<int>(max_work < num_sms ? max_work : num_sms);
-  if (deq != nullptr) {
-    if (D != 128 || skip) return -1;
+  if (deq != nullptr && !skip) {
+    if (D != 128) return -1;
     if (!set_smem_attr<128, false, true>()) return -1;
     attn_fwd_kernel<128, false, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+  } else if (deq != nullptr) {
+    if (D != 128) return -1;
+    if (!set_smem_attr<128, true, true>()) return -1;
+    attn_fwd_kernel<128, true, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
   } else if (D == 128 && !skip) {
     if (!set_smem_attr<128, false, false>()) return -1;
     attn_fwd_kernel<128, false, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);

@@ -9,6 +9,7 @@ built, loading fails with an error.
 from __future__ import annotations
 
 import ctypes as C
+import math
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
@@ -65,8 +66,8 @@ def lib(path: str | None = None) -> C.CDLL:
     L.pqk_varlen_attn_fwd_skip.restype = i32
     L.pqk_quantize_qk_e4m3.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp]
     L.pqk_quantize_qk_e4m3.restype = i32
-    L.pqk_varlen_attn_fwd_fp8qk.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, vp, i32, i64, i32, i32, f32, vp, sz,
-                                            vp]
+    L.pqk_varlen_attn_fwd_fp8qk.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, vp, i32, i64, i32, i32, f32, f32, vp,
+                                            vp, sz, vp]
     L.pqk_varlen_attn_fwd_fp8qk.restype = i32
     L.pqk_varlen_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32,
                                               vp]
@@ -239,9 +240,11 @@ def quantize_qk_e4m3(q, k, *, q8=None, k8=None, scales=None, stream=None):
 
 
 def varlen_attn_fwd_fp8qk(q8, k8, v, deq, cu_seqlens, *, softmax_scale: float | None = None, o=None, lse=None,
-                          workspace=None, want_lse: bool = False, stream=None):
+                          workspace=None, want_lse: bool = False, skip_threshold_log2: float = math.inf,
+                          skip_counts=None, stream=None):
     """Packed varlen attention with Q K^T on the FP8 tensor cores: q8, k8
-    e4m3 bytes [T, H, D] (quantize_qk_e4m3), deq fp32 [2H], v bf16.
+    e4m3 bytes [T, H, D] (quantize_qk_e4m3), deq fp32 [2H], v bf16; block
+    skipping as varlen_attn_fwd_skip when skip_threshold_log2 is finite.
     Returns (o, lse or None)."""
     import torch
     T, H, D = v.shape
@@ -256,8 +259,8 @@ def varlen_attn_fwd_fp8qk(q8, k8, v, deq, cu_seqlens, *, softmax_scale: float | 
     assert q8.is_contiguous() and k8.is_contiguous() and tuple(q8.shape) == (T, H, D) == tuple(k8.shape)
     _check("pqk_varlen_attn_fwd_fp8qk", lib().pqk_varlen_attn_fwd_fp8qk(
         _ptr(q8), _ptr(k8), _ptr(v), _ptr(deq), _ptr(o), _ptr(lse), _token_stride(v, 3), _token_stride(o, 3),
-        _ptr(cu_seqlens), B, T, H, D, scale, _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream(stream)))
+        _ptr(cu_seqlens), B, T, H, D, scale, float(skip_threshold_log2), _ptr(skip_counts), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
     return o, lse
 
 

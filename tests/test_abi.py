@@ -211,11 +211,11 @@ def test_quantize_qk_e4m3_host_errors(L):
 def test_varlen_attn_fp8qk_host_errors(L):
     def call(**kw):
         a = dict(q8=A, k8=A, v=A, deq=A, o=A, lse=None, vs=1024, os_=1024, cu=A, B=2, T=512, H=8, D=128,
-                 scale=0.088, ws=A, wsb=4096)
+                 scale=0.088, tau=float("inf"), counts=None, ws=A, wsb=4096)
         a.update(kw)
         return L.pqk_varlen_attn_fwd_fp8qk(a["q8"], a["k8"], a["v"], a["deq"], a["o"], a["lse"], a["vs"], a["os_"],
-                                           a["cu"], a["B"], a["T"], a["H"], a["D"], a["scale"], a["ws"], a["wsb"],
-                                           None)
+                                           a["cu"], a["B"], a["T"], a["H"], a["D"], a["scale"], a["tau"],
+                                           a["counts"], a["ws"], a["wsb"], None)
     assert call(D=64, vs=512, os_=512) == ERR_UNSUPPORTED
     assert call(deq=None) == ERR_INVALID
     assert call(B=0) == ERR_INVALID
@@ -223,4 +223,7 @@ def test_varlen_attn_fp8qk_host_errors(L):
     assert call(k8=U) == ERR_MISALIGNED
     assert call(deq=A + 2) == ERR_MISALIGNED
     assert call(ws=None) == ERR_WORKSPACE
+    assert call(tau=-1.0) == ERR_INVALID
+    assert call(tau=float("nan")) == ERR_INVALID
+    assert call(counts=A + 4) == ERR_MISALIGNED
     assert call(T=0, q8=None) == 0

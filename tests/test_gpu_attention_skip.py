@@ -35,7 +35,7 @@ def decision_margins(x, tau, scale, blocks=None, per_block=False):
     (request, head, 32-row block, key block >= 1) decisions, in float64.
     blocks: None (all) or a set of (request, 32-row block index). With
     per_block, a dict {(request, block, head): margins of key blocks 1..}."""
-    q, k = wl.bf16_bits_to_f64(x["q"]), wl.bf16_bits_to_f64(x["k"])
+    q, k = (wl.bf16_bits_to_f64(x[n]) if x[n].dtype == np.uint16 else x[n] for n in ("q", "k"))
     cu = x["cu_seqlens"]
     H = q.shape[1]
     worst = math.inf

@@ -135,3 +135,31 @@ def test_fp8_attention_is_deterministic():
     a = [_attn_gpu(x, 0.1) for _ in range(3)]
     for o, lse in a[1:]:
         assert torch.equal(o.view(torch.int16), a[0][0].view(torch.int16)) and torch.equal(lse, a[0][1])
+
+
+@pytest.mark.parametrize("tau", [4.0, 8.0])
+def test_fp8_with_block_skipping_matches_oracle_and_counts(tau):
+    # decisions taken on the FP8 scores: margins checked on the dequantised
+    # Q, K in float64, then outputs and skip counts against the oracle
+    import torch
+    from tests.test_gpu_attention_skip import MARGIN, decision_margins
+    torch_cuda()
+    w = wl.custom([700, 1300, 129], 2, 128, seed=24)
+    x = wl.block_scaled_attention_inputs(w)
+    scale = 1.0 / math.sqrt(128)
+    counts = []
+    ro, rl, q8r, k8r, deqr = oracle.varlen_attn_fp8qk(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, tau=tau,
+                                                      counts_out=counts)
+    H = w.H
+    dec = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    xd = {"q": dec(q8r) * deqr[None, :H, None], "k": dec(k8r) * deqr[None, H:, None], "cu_seqlens": x["cu_seqlens"]}
+    assert decision_margins(xd, tau, scale) >= MARGIN
+    q8, k8, deq = _quantise_gpu(x)
+    c = torch.zeros(2, dtype=torch.int64, device="cuda")
+    o, lse = pqk.varlen_attn_fwd_fp8qk(q8, k8, to_dev_bf16(x["v"]), deq, to_dev(x["cu_seqlens"]), softmax_scale=scale,
+                                       want_lse=True, skip_threshold_log2=tau, skip_counts=c)
+    torch.cuda.synchronize()
+    assert pqk.get_device_status() == 0
+    assert tuple(int(a) for a in c.cpu()) == counts[0] and counts[0][0] > 0
+    assert_attention(bf16_to_f64(o), ro, f"fp8 + skip tau {tau}", peaked=True)
+    assert max_abs(lse.cpu().numpy().astype(np.float64).T, rl) <= LSE_MAX_ABS

@@ -123,3 +123,25 @@ def test_sampled_rows_equal_full_evaluation():
     rows = np.array([0, 5, 299], np.int32)
     o2, l2, q82, _, _ = oracle.varlen_attn_fp8qk(q, k, v, cu, 0.25, rows=rows)
     assert np.array_equal(o2, o[rows]) and np.array_equal(l2, lse[rows]) and np.array_equal(q82, q8)
+
+
+def test_fp8_with_block_skipping_is_skipping_on_the_dequantised_inputs():
+    # composition: FP8 Q K^T with a finite tau = the block-skipping oracle on
+    # the dequantised Q, K (decoded by torch); tau = inf = no skipping
+    g = np.random.default_rng(6)
+    T, H, D = 900, 2, 32
+    q = g.standard_normal((T, H, D)) * 2.5
+    k = g.standard_normal((T, H, D)) * np.repeat(g.choice([0.02, 3.0], math.ceil(T / 128)), 128)[:T, None, None]
+    v = g.standard_normal((T, H, D))
+    cu = np.array([0, 400, T], np.int32)
+    scale = 1.0 / math.sqrt(D)
+    counts = []
+    o, lse, q8, k8, deq = oracle.varlen_attn_fp8qk(q, k, v, cu, scale, tau=6.0, counts_out=counts)
+    qd = _decode(q8) * deq[None, :H, None]
+    kd = _decode(k8) * deq[None, H:, None]
+    os_, ls, cs = oracle.varlen_attn_skip(qd, kd, v, cu, scale, 6.0)
+    assert counts == [cs] and cs[0] > 0
+    assert np.array_equal(o, os_) and np.array_equal(lse, ls)
+    o_inf, _, _, _, _ = oracle.varlen_attn_fp8qk(q, k, v, cu, scale)
+    on, _, _, _, _ = oracle.varlen_attn_fp8qk(q, k, v, cu, scale, tau=math.inf)
+    assert np.array_equal(o_inf, on)
