@@ -147,3 +147,33 @@ def test_local_inputs_sampled_rows():
             share = sum(p[128 * j:128 * (j + 1)].sum() for j in undecided) / p.sum()
             assert max_abs(o[n, h], ro[n, h]) <= 2.0 * share * vmax + 2e-2
     assert n_clear >= len(rows) * H // 2
+
+
+def test_local_inputs_58048_tokens_sampled_rows():
+    # the bench's block-skipping workload (local stand-in at 58,048 tokens,
+    # 24 heads, tau = 8) on 12 sampled rows: decided (row, head) pairs
+    # against the oracle, the others within the bound of either choice
+    w = wl.config(3)
+    x = wl.local_attention_inputs(w, amplitude=16.0)
+    scale, tau = 1.0 / math.sqrt(128), 8.0
+    rows = wl.sample_rows(w, per_segment=12)
+    margins = decision_margins(x, tau, scale, {(0, int(r) // 32) for r in rows}, per_block=True)
+    o, lse, counts = run_skip(x, tau, scale)
+    assert counts[0] > 0
+    o = bf16_to_f64(o)[rows]
+    ro, rl, _ = oracle.varlen_attn_skip(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, tau, rows=rows)
+    q, k = wl.bf16_bits_to_f64(x["q"]), wl.bf16_bits_to_f64(x["k"])
+    vmax = float(np.abs(wl.bf16_bits_to_f64(x["v"])).max())
+    n_clear = 0
+    for n, r in enumerate(rows):
+        for h in range(w.H):
+            undecided = np.nonzero(margins[(0, int(r) // 32, h)] < MARGIN)[0] + 1
+            if undecided.size == 0:
+                n_clear += 1
+                assert_attention(o[n, h], ro[n, h], f"local 58k row {r} head {h}", peaked=True)
+                continue
+            s_row = scale * (k[:, h] @ q[r, h])
+            p = np.exp(s_row - s_row.max())
+            share = sum(p[128 * j:128 * (j + 1)].sum() for j in undecided) / p.sum()
+            assert max_abs(o[n, h], ro[n, h]) <= 2.0 * share * vmax + 2e-2
+    assert n_clear >= len(rows) * w.H // 8

@@ -163,3 +163,15 @@ def test_fp8_with_block_skipping_matches_oracle_and_counts(tau):
     assert tuple(int(a) for a in c.cpu()) == counts[0] and counts[0][0] > 0
     assert_attention(bf16_to_f64(o), ro, f"fp8 + skip tau {tau}", peaked=True)
     assert max_abs(lse.cpu().numpy().astype(np.float64).T, rl) <= LSE_MAX_ABS
+
+
+def test_joint_sequence_58048_sampled():
+    # the bench's workload and launch configuration, on 96 sampled rows
+    w = wl.config(3)
+    x = wl.attention_inputs(w)
+    scale = 1.0 / math.sqrt(w.D)
+    rows = wl.sample_rows(w, per_segment=96)
+    o, lse = _attn_gpu(x, scale)
+    ro, rl, _, _, _ = oracle.varlen_attn_fp8qk(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, rows=rows)
+    assert_attention(bf16_to_f64(o)[rows], ro, "fp8 58,048 tokens sampled")
+    assert max_abs(lse.cpu().numpy().astype(np.float64).T[rows], rl) <= LSE_MAX_ABS
