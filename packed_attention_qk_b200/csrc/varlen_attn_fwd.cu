@@ -312,6 +312,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using L = Layout<D>;
   static_assert(!kFp8 || D == 128, "FP8 Q K^T: one 128-byte swizzle row per token");
+  // FP8 Q K^T: the MMA thread waits for the next V stage (loaded long ago)
+  // while it waits for P1 anyway, and probes the next K stage there without
+  // blocking (its copy may still be in flight), instead of waiting for both
+  // at the top of the next iteration, just before P0 (-3 % time with FP8;
+  // +1 % with bf16 operands, where it is left out).
+  constexpr bool kEarlyKv = kFp8;
   // bytes of one Q or K tile: bf16 slabs, or 128 rows x 128 e4m3 bytes
   constexpr uint32_t kQKBytes = kFp8 ? static_cast<uint32_t>(kBM) * 128u : static_cast<uint32_t>(L::kTileBytes);
   extern __shared__ uint8_t smem_raw[];
@@ -487,14 +493,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(kv_empty(k_stage_idx % L::kStages));
         if (wk.n_kv == 1) tc_commit(q_empty);
         ++cons_idx;
+        // stages of iteration j: V_j and K_{j+1}
+        uint32_t v_idx = cons_idx++;
+        uint32_t nk_idx = wk.n_kv > 1 ? cons_idx++ : 0;
+        bool v_ready = false, k_ready = false;
         for (int j = 0; j < wk.n_kv; ++j) {
-          const uint32_t v_idx = cons_idx++;
           const bool more = j + 1 < wk.n_kv;
-          const uint32_t nk_idx = more ? cons_idx++ : 0;
-          // V_j and K_{j+1} are waited for here, while P0 is still being
-          // computed, not between O0 += P0 V_j and S0 = Q0 K_{j+1}^T
-          if (!(ok = wait_stage(v_idx))) break;
-          if (more && !(ok = wait_stage(nk_idx))) break;
+          // V_j and K_{j+1} are complete before P0 is waited for, so no copy
+          // wait sits between O0 += P0 V_j and S0 = Q0 K_{j+1}^T
+          if (!v_ready && !(ok = wait_stage(v_idx))) break;
+          if (more && !k_ready && !(ok = wait_stage(nk_idx))) break;
           if (!(ok = mbar_wait(p_full(0), p_phase, abort_flag, p.timeout_ns))) break;
           tc_fence_after_sync();
           if (kSkip && j > 0 && group_skips(0, j)) {
@@ -506,6 +514,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (more) {
             issue_qk(0, nk_idx % L::kStages);
             tc_commit(s_full(0));
+          }
+          uint32_t next_v = 0, next_nk = 0;
+          if (more) {
+            next_v = cons_idx++;
+            next_nk = j + 2 < wk.n_kv ? cons_idx++ : 0;
+          }
+          v_ready = k_ready = false;
+          if (kEarlyKv && more) {
+            if (!(ok = wait_stage(next_v))) break;
+            v_ready = true;
+            k_ready = j + 2 < wk.n_kv &&
+                      mbar_test_wait(kv_full(next_nk % L::kStages), (next_nk / L::kStages) & 1);
           }
           if (!(ok = mbar_wait(p_full(1), p_phase, abort_flag, p.timeout_ns))) break;
           tc_fence_after_sync();
@@ -523,6 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (j + 2 == wk.n_kv) tc_commit(q_empty);
           }
           p_phase ^= 1u;
+          v_idx = next_v;
+          nk_idx = next_nk;
         }
       }
       if (kSkip && p.skip_counts != nullptr && pv_skips != 0) atomicAdd(&p.skip_counts[1], pv_skips);
