@@ -41,6 +41,16 @@
 // Every wait is bounded (pqk::mbar_wait); a wait that runs out raises the
 // block's abort flag and the device status word, and the block drains its
 // copies and MMAs in flight (bounded again), frees tensor memory and exits.
+//
+// Two compile-time variants of the same pipeline:
+//   kSkip  block skipping ("Skip-Softmax", first page, bullet on TRTLLM_ATTN
+//          SAGE and Skip-Softmax): a softmax warp whose 32 rows all have the
+//          tile maximum more than skip_tau below their earlier maximum writes
+//          P = 0 and skips its exponentials; the MMA thread leaves out
+//          O_i += P_i V_j when all four warps of the group voted so;
+//   kFp8   Q and K as e4m3 bytes (SAGE FP8): S_i = Q_i K^T from 16 KB tiles
+//          with kind::f8f6f4 MMAs, the heads' dequantisation factors folded
+//          into the softmax scale.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
