@@ -90,7 +90,7 @@ def test_infinite_threshold_is_bitwise_the_plain_kernel(lens, H, D):
 
 
 @pytest.mark.parametrize("lens, H, D, seed", [([700, 1300, 129], 2, 128, 24), ([1000, 37, 640], 3, 64, 8),
-                                              ([2048], 2, 128, 9)])
+                                              ([2048], 2, 128, 9), ([640, 0, 257, 1], 2, 128, 44)])
 @pytest.mark.parametrize("tau", [4.0, 8.0])
 def test_block_scaled_matches_oracle_and_counts(lens, H, D, seed, tau):
     w = wl.custom(lens, H, D, seed=seed)
