@@ -32,6 +32,12 @@
  *   - Input and output buffers must not partially overlap. Exact in-place
  *     use (output pointer == input pointer, same layout) is allowed where
  *     stated.
+ *   - CUDA graphs: the compute calls enqueue only kernels and stream-ordered
+ *     memory operations (tensor maps are encoded on the host and passed by
+ *     value), so they can be captured and replayed. The first call of each
+ *     compute entry point on a device queries and caches device attributes
+ *     and kernel settings; make it before capturing. pqk_get_device_status
+ *     synchronizes and must not be captured.
  */
 #ifndef PQK_H
 #define PQK_H
