@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="leave out the FP8 Q K^T attention timing")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the block call captured once in a CUDA graph and replayed (graph_ms_per_step)")
     ap.add_argument("--skip-tau", type=float, default=8.0,
                     help="threshold (log2 units) of the block-skipping attention timed on the local-attention "
                          "stand-in after the steps; negative = leave that timing out")
@@ -318,6 +320,32 @@ def run_ours(args, w):
     total_ms = max_over_ranks(start.elapsed_time(stop))
     if pqk.get_device_status() != 0:
         raise RuntimeError("device status set during the timed steps")
+    graph_ms = None
+    if args.graph:
+        # the same block call captured once (all calls were made before, so
+        # the library's per-device setup is done) and replayed K times
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(dev)
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cs):
+            with torch.cuda.graph(g, stream=cs):
+                block_call(w, d, o)
+        torch.cuda.current_stream().wait_stream(cs)
+        for _ in range(args.warmup):
+            g.replay()
+        barrier()
+        torch.cuda.synchronize()
+        gs, gt = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        gs.record()
+        for _ in range(K):
+            g.replay()
+        gt.record()
+        torch.cuda.synchronize()
+        barrier()
+        graph_ms = max_over_ranks(gs.elapsed_time(gt)) / K
+        if pqk.get_device_status() != 0:
+            raise RuntimeError("device status set during the graph replays")
+        del g
     pro = [e[0].elapsed_time(e[1]) for e in evs]
     att = [e[1].elapsed_time(e[2]) for e in evs]
     epi = [e[2].elapsed_time(e[3]) for e in evs]
@@ -565,6 +593,7 @@ def run_ours(args, w):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * K,
+        "graph_ms_per_step": graph_ms,
         "clocks": clocks.summary(),
     }
     if rank == 0:
