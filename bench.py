@@ -15,6 +15,14 @@ per second of device time of the whole step (max over ranks); the kernel
 figures and the roofline of the dominant kernel (the attention) are in the
 same line. With N > 1 (torchrun) every rank runs its own request: weak
 scaling, no collective on the data path.
+
+After the timed steps the same line also carries, under ``kernels``: the
+three-axis RoPE, back-to-back and full-width norm timings; the block-
+skipping attention on the local-attention stand-in (``--skip-tau``, plain
+vs skipping vs FP8 Q K^T with and without skipping); the FP8 Q K^T attention
+on the step's inputs (``--no-fp8`` leaves it out); and, with ``--graph``,
+the step replayed as a CUDA graph (``graph_ms_per_step``). ``--config N``
+selects another configuration, ``--sweep`` the HBM bandwidth sweep.
 """
 
 from __future__ import annotations
