@@ -61,10 +61,12 @@ def load(path: str):
     L.oracle_varlen_attn_fp8qk.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
                                            C.c_int, C.c_double, C.c_double, i32p, C.c_int64, f64p, f64p,
                                            C.POINTER(C.c_int64), u8p, u8p, f32p]
+    L.oracle_varlen_attn_fp8.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
+                                         C.c_int, C.c_double, i32p, C.c_int64, f64p, f64p, f32p]
     L.oracle_e4m3_codes.argtypes = [f32p, C.c_int64, u8p]
     L.oracle_e4m3_codes.restype = None
     for f in (L.oracle_qk_norm_rope, L.oracle_qk_norm_rope_3axis, L.oracle_qk_fullc_norm_rope, L.oracle_varlen_attn,
-              L.oracle_varlen_attn_skip, L.oracle_quantize_e4m3, L.oracle_varlen_attn_fp8qk,
+              L.oracle_varlen_attn_skip, L.oracle_quantize_e4m3, L.oracle_varlen_attn_fp8qk, L.oracle_varlen_attn_fp8,
               L.oracle_modulate_swiglu):
         f.restype = C.c_int
     L.oracle_num_threads.restype = C.c_int
@@ -255,6 +257,28 @@ def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: n
     if counts_out is not None and r is None:
         counts_out.append(tuple(int(c) for c in counts))
     return o, lse, q8, k8, deq
+
+
+def varlen_attn_fp8(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, rows=None,
+                    want_lse: bool = True):
+    """Attention with Q, K, V and P in FP8 e4m3 (oracle_varlen_attn_fp8).
+    Returns (o [nrows, H, D], lse [nrows, H] or None, deq [3H])."""
+    T, H, D = q.shape
+    assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
+    q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    r, n = _rows(rows)
+    n = n if r is not None else T
+    o = np.empty((n, H, D), np.float64)
+    lse = np.empty((n, H), np.float64) if want_lse else None
+    deq = np.empty(3 * H, np.float32)
+    rc = lib().oracle_varlen_attn_fp8(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32),
+                                      int(cu.shape[0]) - 1, T, H, D, scale, _ptr(r, C.c_int32),
+                                      n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
+                                      _ptr(deq, C.c_float))
+    if rc:
+        raise ValueError("oracle_varlen_attn_fp8: invalid arguments")
+    return o, lse, deq
 
 
 def modulate_swiglu(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, gate_res: np.ndarray,

@@ -24,6 +24,8 @@
  *                             "Long-sequence attention & communication").
  *   oracle_varlen_attn_fp8qk -- the same attention with Q and K quantised to
  *                             FP8 e4m3 per head (SAGE FP8, a reading).
+ *   oracle_varlen_attn_fp8  -- the attention with Q, K, V and P in FP8 e4m3
+ *                             (the whole SAGE reading).
  *   oracle_varlen_attn_skip -- the same attention with key blocks skipped
  *                             where their scores are negligible ("Skip-Softmax";
  *                             a reading, see the function).
@@ -396,6 +398,98 @@ int oracle_varlen_attn_fp8qk(const void* q, const void* k, const void* v, int in
   free(qd);
   free(kd);
   free(vd);
+  return rc;
+}
+
+/*
+ * Attention with Q, K and V quantised to e4m3 per head and the
+ * probabilities P quantised to e4m3 inside the online softmax: the whole
+ * attention computation in FP8 (SAGE, first page, bullet on TRTLLM_ATTN SAGE
+ * and Skip-Softmax; a reading). Per row, over the key blocks of 128 keys
+ * counted from the request's first token, in order, with u = s / ln 2 the
+ * score of the dequantised Q, K in log2 units:
+ *   - the running maximum m is set by the first block and afterwards moves
+ *     only when a block's maximum exceeds it by more than 8; the sums are
+ *     then scaled by 2^(m_old - m_new);
+ *   - each key adds p = 2^(u - m) to the denominator l and e4m3(p) * v~ to
+ *     the numerator (v~ = code(V) * deq_V; p <= 2^8 stays in e4m3's range);
+ *   - O = numerator / l and lse = (m + log2 l) ln 2.
+ * deq_out: [3H] (Q's, K's, V's dequantisation factors), optional.
+ */
+static void fp8_row(const double* qd, const double* kd, const double* vd, int64_t lo, int64_t n_keys, int64_t t,
+                    int H, int h, int D, double scale, double* ot, double* lse_out) {
+  const double* qr = qd + (t * H + h) * (int64_t)D;
+  double* num = (double*)calloc((size_t)D, sizeof(double));
+  double mrun = -INFINITY, den = 0.0;
+  for (int64_t b0 = 0; b0 < n_keys; b0 += 128) {
+    const int64_t b1 = b0 + 128 < n_keys ? b0 + 128 : n_keys;
+    double ublock[128];
+    double bmax = -INFINITY;
+    for (int64_t j = b0; j < b1; ++j) {
+      const double* kr = kd + ((lo + j) * H + h) * (int64_t)D;
+      double dot = 0.0;
+      for (int d = 0; d < D; ++d) dot += qr[d] * kr[d];
+      ublock[j - b0] = scale * dot / log(2.0);
+      if (ublock[j - b0] > bmax) bmax = ublock[j - b0];
+    }
+    if (b0 == 0) {
+      mrun = bmax;
+    } else if (bmax > mrun + 8.0) {
+      const double alpha = exp2(mrun - bmax);
+      den *= alpha;
+      for (int d = 0; d < D; ++d) num[d] *= alpha;
+      mrun = bmax;
+    }
+    for (int64_t j = b0; j < b1; ++j) {
+      const double pj = exp2(ublock[j - b0] - mrun);
+      const double pq = e4m3_value(e4m3_code((float)pj));
+      den += pj;
+      const double* vr = vd + ((lo + j) * H + h) * (int64_t)D;
+      for (int d = 0; d < D; ++d) num[d] += pq * vr[d];
+    }
+  }
+  for (int d = 0; d < D; ++d) ot[d] = num[d] / den;
+  if (lse_out) *lse_out = (mrun + log2(den)) * log(2.0);
+  free(num);
+}
+
+int oracle_varlen_attn_fp8(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
+                           const int32_t* cu, int B, int64_t T, int H, int D, double scale, const int32_t* rows,
+                           int64_t nrows, double* o, double* lse, float* deq_out) {
+  if (check_cu(cu, B, T) || H <= 0 || D <= 0) return -1;
+  const int64_t n = T * (int64_t)H * D;
+  uint8_t* c8 = (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
+  float* dq = (float*)malloc(sizeof(float) * (size_t)H * 3);
+  double* xd[3];
+  const void* src[3] = {q, k, v};
+  int rc = 0;
+  for (int i = 0; i < 3; ++i) {
+    xd[i] = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    if (!rc) rc = oracle_quantize_e4m3(src[i], in_kind, stride_t, T, H, D, c8, dq + (int64_t)i * H);
+    if (!rc) {
+#pragma omp parallel for schedule(static)
+      for (int64_t e = 0; e < n; ++e) xd[i][e] = e4m3_value(c8[e]) * (double)dq[(int64_t)i * H + (e / D) % H];
+    }
+  }
+  if (!rc) {
+    const int64_t nr = rows ? nrows : T;
+    int64_t bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2) reduction(+ : bad)
+    for (int64_t r = 0; r < nr; ++r) {
+      for (int h = 0; h < H; ++h) {
+        const int64_t t = rows ? rows[r] : r;
+        const int seg = (t >= 0 && t < T) ? segment_of(cu, B, t) : -1;
+        if (seg < 0) { ++bad; continue; }
+        fp8_row(xd[0], xd[1], xd[2], cu[seg], (int64_t)cu[seg + 1] - cu[seg], t, H, h, D, scale,
+                o + (r * H + h) * (int64_t)D, lse ? &lse[r * H + h] : NULL);
+      }
+    }
+    if (bad) rc = -1;
+  }
+  if (deq_out) memcpy(deq_out, dq, sizeof(float) * (size_t)H * 3);
+  for (int i = 0; i < 3; ++i) free(xd[i]);
+  free(c8);
+  free(dq);
   return rc;
 }
 

@@ -145,3 +145,80 @@ def test_fp8_with_block_skipping_is_skipping_on_the_dequantised_inputs():
     o_inf, _, _, _, _ = oracle.varlen_attn_fp8qk(q, k, v, cu, scale)
     on, _, _, _, _ = oracle.varlen_attn_fp8qk(q, k, v, cu, scale, tau=math.inf)
     assert np.array_equal(o_inf, on)
+
+
+# ---------------------------------------------------------------- Q, K, V and P in FP8
+
+def _one_row_case(k_vals, v_vals, scale):
+    """One request, one head, D = 1, q = 1.75: keys k_vals, values v_vals.
+    Every tensor's amax is 1.75 = 448 * 2^-8, so its scale is exactly 2^-8
+    and values that are e4m3 codes times 2^-8 quantise exactly."""
+    L = len(k_vals)
+    q = np.full((L, 1, 1), 1.75)
+    k = np.array(k_vals, np.float64).reshape(L, 1, 1)
+    v = np.array(v_vals, np.float64).reshape(L, 1, 1)
+    o, lse, _ = oracle.varlen_attn_fp8(q, k, v, np.array([0, L], np.int32), scale)
+    return o[0, 0, 0], lse[0, 0]
+
+
+def test_fp8_p_rounds_in_the_numerator_only():
+    # keys 1.75 and 0.875 at scale 0.6 ln 2 / 1.75^2: u = (0.6, 0.3),
+    # p = (1, 2^-0.3) and e4m3(2^-0.3 = 0.81225) = 0.8125 (13/16); values
+    # 1.75 and -1.75
+    o, lse = _one_row_case([1.75, 0.875], [1.75, -1.75], 0.6 * math.log(2.0) / 1.75 ** 2)
+    p2 = 2.0 ** -0.3
+    assert abs(o - 1.75 * (1.0 - 0.8125) / (1.0 + p2)) <= 1e-12
+    assert abs(lse - (0.6 + math.log2(1.0 + p2)) * math.log(2.0)) <= 1e-12
+
+
+def test_fp8_running_maximum_moves_only_beyond_eight():
+    # 128 keys with k = 0 (block 0, u = 0), then one key with k = 1.75
+    # (block 1) whose u is 5.3: within 8 of the maximum, so m stays 0,
+    # p = 2^5.3 = 39.40 and e4m3 rounds it to 40; values 0 then 1.75
+    k = [0.0] * 128 + [1.75]
+    o, _ = _one_row_case(k, [0.0] * 128 + [1.75], 5.3 * math.log(2.0) / 1.75 ** 2)
+    assert abs(o - 1.75 * 40.0 / (128.0 + 2.0 ** 5.3)) <= 1e-12
+    # u = 9.3 is beyond 8: m moves to 9.3, block 0's sums scale by 2^-9.3 and
+    # the new key has p = 1 exactly; block-0 values 0.5
+    o, _ = _one_row_case(k, [0.5] * 128 + [1.75], 9.3 * math.log(2.0) / 1.75 ** 2)
+    a = 2.0 ** -9.3
+    assert abs(o - (128 * 0.5 * a + 1.75) / (128 * a + 1.0)) <= 1e-12
+
+
+def test_fp8_is_exact_on_representable_inputs():
+    # Q, K entries in {0, 1} on dims 2.. with one 1.75 on dims 0 / 1 where the
+    # other tensor is 0 (amax 1.75 -> scale 2^-8 exactly), scale ln 2: integer
+    # log2 scores in [0, 6], so every p is a power of two e4m3 holds; V from
+    # e4m3 values times 2^-6 with amax 7 (scale 2^-6): the FP8 attention then
+    # equals the plain attention
+    g = np.random.default_rng(8)
+    T, H, D = 400, 2, 8
+    q = np.zeros((T, H, D))
+    k = np.zeros((T, H, D))
+    q[:, :, 2:] = g.integers(0, 2, (T, H, D - 2))
+    k[:, :, 2:] = g.integers(0, 2, (T, H, D - 2))
+    q[0, :, 0] = 1.75
+    k[0, :, 1] = 1.75
+    _, vals = e4m3_table()
+    v = g.choice(vals[np.abs(vals) <= 448], (T, H, D)).astype(np.float64) * 2.0 ** -6
+    v[0, :, 0] = 7.0
+    cu = np.array([0, 150, 400], np.int32)
+    o, lse, deq = oracle.varlen_attn_fp8(q, k, v, cu, math.log(2.0))
+    assert np.array_equal(deq, np.array([2.0 ** -8] * 4 + [2.0 ** -6] * 2, np.float32))
+    ob, lb = oracle.varlen_attn(q, k, v, cu, math.log(2.0))
+    assert np.max(np.abs(o - ob)) <= 1e-12 and np.max(np.abs(lse - lb)) <= 1e-12
+
+
+def test_fp8_error_bound_against_exact_p():
+    # P's rounding moves each numerator term by at most 2^-4 of itself, so O
+    # moves by at most 2^-4 max|V~| from the attention with exact P on the
+    # same dequantised Q, K, V
+    g = np.random.default_rng(9)
+    T, H, D = 500, 2, 32
+    q, k, v = (g.standard_normal((T, H, D)) for _ in range(3))
+    cu = np.array([0, 130, 500], np.int32)
+    scale = 1.0 / math.sqrt(D)
+    o, _, deq = oracle.varlen_attn_fp8(q, k, v, cu, scale)
+    dec = [_decode(oracle.quantize_e4m3(x)[0]) * oracle.quantize_e4m3(x)[1][None, :, None] for x in (q, k, v)]
+    ob, _ = padded_masked_attention(dec[0], dec[1], dec[2], cu, scale)
+    assert 0 < np.max(np.abs(o - ob)) <= 2.0 ** -4 * np.abs(dec[2]).max()

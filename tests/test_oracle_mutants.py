@@ -63,6 +63,12 @@ MUTANTS = {
                                 "    for (int64_t t = 0; t < 1; ++t)\n      for (int d = 0; d < D; ++d) {\n        const float v = (float)fabs("),
     "fp8_range_240": ("const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;",
                       "const float inv = amax > 0.0f ? 240.0f / amax : 1.0f;"),
+    "fp8_lazy_threshold_zero": ("} else if (bmax > mrun + 8.0) {", "} else if (bmax > mrun) {"),
+    "fp8_p_not_quantised": ("const double pq = e4m3_value(e4m3_code((float)pj));", "const double pq = pj;"),
+    "fp8_denominator_quantised": ("      den += pj;\n", "      den += pq;\n"),
+    "fp8_numerator_not_rescaled": ("      for (int d = 0; d < D; ++d) num[d] *= alpha;\n", ""),
+    "fp8_v_with_q_scale": ("xd[i][e] = e4m3_value(c8[e]) * (double)dq[(int64_t)i * H + (e / D) % H];",
+                           "xd[i][e] = e4m3_value(c8[e]) * (double)dq[(e / D) % H];"),
     "skip_tile_counts_any_block": ("if (keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;",
                                    "if (!keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;"),
 }
