@@ -492,10 +492,25 @@ def run_ours(args, w):
         fp8_ms = ev3[0].elapsed_time(ev3[1]) / 3
         if pqk.get_device_status() != 0:
             raise RuntimeError("device status set during the FP8 timing")
+        # the whole computation in FP8: V quantised as well, P rounded to e4m3
+        v8, deq_v = pqk.quantize_e4m3(d["v"])
+        deq3 = torch.cat([deq, deq_v]).contiguous()
+        full = lambda: pqk.varlen_attn_fwd_fp8(q8, k8, v8, deq3, d["cu"], o=fo, workspace=o["ws"])
+        full()
+        torch.cuda.synchronize()
+        ev3[0].record()
+        for _ in range(3):
+            full()
+        ev3[1].record()
+        torch.cuda.synchronize()
+        full_ms = ev3[0].elapsed_time(ev3[1]) / 3
+        if pqk.get_device_status() != 0:
+            raise RuntimeError("device status set during the FP8 timing")
         fp8 = {"quantize_us": quant_us, "attn_ms": fp8_ms, "attn_tflops": flops / (fp8_ms * 1e-3) / 1e12,
                "speedup_vs_bf16": att_ms / fp8_ms,
-               "quantize_gbs": (4 * w.T * w.H * w.D + 2 * w.T * w.H * w.D) / (quant_us * 1e-6) / 1e9}
-        del q8, k8, fo
+               "quantize_gbs": (4 * w.T * w.H * w.D + 2 * w.T * w.H * w.D) / (quant_us * 1e-6) / 1e9,
+               "full_fp8_attn_ms": full_ms, "full_fp8_speedup_vs_bf16": att_ms / full_ms}
+        del q8, k8, v8, fo
 
     # e2e through host buffers: every step copies all of its inputs from
     # pinned host memory to the device (H2D stream), runs the three C-ABI

@@ -35,14 +35,15 @@ size_t attn_schedule_bytes(int B);
 // two device counters the kernel adds to). deq non-null selects the kernel
 // with Q, K given as e4m3 bytes ([T, H, D], strides in bytes) and deq their
 // [2H] per-head dequantisation factors (D = 128; skipping may be combined
-// with it). Returns 0, or
+// with it). fp8_pv: V is e4m3 bytes too and P is rounded to e4m3 for P V
+// (deq then [3H], V's last; no skipping). Returns 0, or
 // -1 when a CUDA call failed, -2 when the tensor maps could not be encoded.
 int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, float* lse, int64_t q_stride,
                        int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
                        int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
                        long long timeout_ns, cudaStream_t stream, int num_sms, bool skip = false,
                        float skip_tau = 0.0f, unsigned long long* skip_counts = nullptr,
-                       const float* deq = nullptr);
+                       const float* deq = nullptr, bool fp8_pv = false);
 
 // Per-head absmax e4m3 quantisation of Q and K ([T, H, D] bf16, strides in
 // elements) into q8, k8 ([T, H, D] bytes, contiguous). scales: [4H] floats,
@@ -50,6 +51,11 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
 // heads, then K's). D is 64 or 128.
 int launch_quantize_qk_e4m3(const void* q, const void* k, int64_t q_stride, int64_t k_stride, int64_t T, int H,
                             int D, void* q8, void* k8, float* scales, cudaStream_t stream, int num_sms);
+
+// The same for one tensor x: scales [2H], [0, H) scratch, [H, 2H) its
+// dequantisation factors.
+int launch_quantize_e4m3(const void* x, int64_t x_stride, int64_t T, int H, int D, void* x8, float* scales,
+                         cudaStream_t stream, int num_sms);
 
 int launch_wait_selftest(int* status, long long timeout_ns, cudaStream_t stream);
 

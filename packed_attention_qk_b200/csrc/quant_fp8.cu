@@ -10,8 +10,10 @@
 // head costs precision only for values 2^15 below amax (the subnormal range).
 //
 // HBM-bound, two passes: absmax (read Q, K) and quantise (read Q, K again,
-// write one byte per element). Rows of D bf16 are spread over D/8 lanes
-// (16 bytes each), so a warp covers 32 / (D / 8) (token, head) rows per step.
+// write one byte per element). The same kernels quantise a single tensor
+// (V for the attention with P V in FP8). Rows of D bf16 are spread over D/8
+// lanes (16 bytes each), so a warp covers 32 / (D / 8) (token, head) rows
+// per step.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -56,8 +58,9 @@ __global__ void __launch_bounds__(kThreads) absmax_kernel(const __nv_bfloat16* q
                                                           unsigned* amax) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
-  extern __shared__ unsigned s_max[];  // [2H]: Q's heads, then K's
-  for (int i = threadIdx.x; i < 2 * H; i += blockDim.x) s_max[i] = 0u;
+  extern __shared__ unsigned s_max[];  // [2H]: Q's heads, then K's (when K is given)
+  const int nmax = (k != nullptr ? 2 : 1) * H;
+  for (int i = threadIdx.x; i < nmax; i += blockDim.x) s_max[i] = 0u;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int part = lane % kLanesPerRow;
@@ -72,7 +75,7 @@ __global__ void __launch_bounds__(kThreads) absmax_kernel(const __nv_bfloat16* q
       const int64_t t = r / H;
       h = static_cast<int>(r % H);
       mq = absmax8(ld_nc16(q + t * qs + static_cast<int64_t>(h) * D + part * 8));
-      mk = absmax8(ld_nc16(k + t * ks + static_cast<int64_t>(h) * D + part * 8));
+      if (k != nullptr) mk = absmax8(ld_nc16(k + t * ks + static_cast<int64_t>(h) * D + part * 8));
     }
 #pragma unroll
     for (int off = kLanesPerRow / 2; off > 0; off >>= 1) {
@@ -81,11 +84,11 @@ __global__ void __launch_bounds__(kThreads) absmax_kernel(const __nv_bfloat16* q
     }
     if (part == 0 && r < rows) {
       atomicMax(&s_max[h], __float_as_uint(mq));  // non-negative floats order like their bits
-      atomicMax(&s_max[H + h], __float_as_uint(mk));
+      if (k != nullptr) atomicMax(&s_max[H + h], __float_as_uint(mk));
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < 2 * H; i += blockDim.x)
+  for (int i = threadIdx.x; i < nmax; i += blockDim.x)
     if (s_max[i] != 0u) atomicMax(&amax[i], s_max[i]);
 }
 
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(kThreads) quantise_kernel(const __nv_bfloat16*
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i < 2 * H; i += blockDim.x) {
+    for (int i = threadIdx.x; i < (k != nullptr ? 2 : 1) * H; i += blockDim.x) {
       const float a = __uint_as_float(amax[i]);
       deq[i] = a > 0.f ? a / 448.0f : 1.0f;
     }
@@ -124,19 +127,24 @@ __global__ void __launch_bounds__(kThreads) quantise_kernel(const __nv_bfloat16*
     if (r >= rows) continue;
     const int64_t t = r / H;
     const int h = static_cast<int>(r % H);
-    const uint4 vq = ld_nc16(q + t * qs + static_cast<int64_t>(h) * D + part * 8);
-    const uint4 vk = ld_nc16(k + t * ks + static_cast<int64_t>(h) * D + part * 8);
     const int64_t o = r * D + part * 8;
+    const uint4 vq = ld_nc16(q + t * qs + static_cast<int64_t>(h) * D + part * 8);
     *reinterpret_cast<uint2*>(q8 + o) = quant8(vq, inv_of(amax[h]));
-    *reinterpret_cast<uint2*>(k8 + o) = quant8(vk, inv_of(amax[H + h]));
+    if (k != nullptr) {
+      const uint4 vk = ld_nc16(k + t * ks + static_cast<int64_t>(h) * D + part * 8);
+      *reinterpret_cast<uint2*>(k8 + o) = quant8(vk, inv_of(amax[H + h]));
+    }
   }
 }
 
+// k == nullptr: one tensor; scales is then [2H] ([0, H) scratch, [H, 2H) its
+// dequantisation factors), else [4H] as for Q and K.
 template <int D>
 int launch(const void* q, const void* k, int64_t qs, int64_t ks, int64_t T, int H, void* q8, void* k8,
            float* scales, cudaStream_t stream, int num_sms) {
+  const int n = k != nullptr ? 2 : 1;
   unsigned* amax = reinterpret_cast<unsigned*>(scales);
-  if (cudaMemsetAsync(amax, 0, sizeof(unsigned) * 2 * H, stream) != cudaSuccess) return -1;
+  if (cudaMemsetAsync(amax, 0, sizeof(unsigned) * n * H, stream) != cudaSuccess) return -1;
   constexpr int kRowsPerBlock = (kThreads / 32) * (32 / (D / 8));
   const int64_t blocks_needed = (T * H + kRowsPerBlock - 1) / kRowsPerBlock;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
@@ -146,7 +154,7 @@ int launch(const void* q, const void* k, int64_t qs, int64_t ks, int64_t T, int 
   absmax_kernel<D><<<grid, kThreads, sizeof(unsigned) * 2 * H, stream>>>(qb, kb, qs, ks, T, H, amax);
   if (cudaGetLastError() != cudaSuccess) return -1;
   quantise_kernel<D><<<grid, kThreads, 0, stream>>>(qb, kb, qs, ks, T, H, amax, static_cast<uint8_t*>(q8),
-                                                     static_cast<uint8_t*>(k8), scales + 2 * H);
+                                                     static_cast<uint8_t*>(k8), scales + n * H);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -156,6 +164,12 @@ int launch_quantize_qk_e4m3(const void* q, const void* k, int64_t q_stride, int6
                             int D, void* q8, void* k8, float* scales, cudaStream_t stream, int num_sms) {
   if (D == 128) return launch<128>(q, k, q_stride, k_stride, T, H, q8, k8, scales, stream, num_sms);
   return launch<64>(q, k, q_stride, k_stride, T, H, q8, k8, scales, stream, num_sms);
+}
+
+int launch_quantize_e4m3(const void* x, int64_t x_stride, int64_t T, int H, int D, void* x8, float* scales,
+                         cudaStream_t stream, int num_sms) {
+  if (D == 128) return launch<128>(x, nullptr, x_stride, 0, T, H, x8, nullptr, scales, stream, num_sms);
+  return launch<64>(x, nullptr, x_stride, 0, T, H, x8, nullptr, scales, stream, num_sms);
 }
 
 }  // namespace pqk

@@ -172,6 +172,23 @@ __device__ __forceinline__ void mma_f8_ss_w(uint32_t d_tmem, uint32_t a_lo, uint
       : "memory");
 }
 
+// D(tmem) (+)= A(tmem) * B(smem), kind::f8f6f4 (A: 8-bit, four K-consecutive
+// values per 32-bit tensor-memory column; K = 32 per instruction), B's
+// descriptor given as its (low, high) words.
+__device__ __forceinline__ void mma_f8_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      ".reg .b64 db;\n"
+      "setp.ne.b32 p, %5, 0;\n"
+      "mov.b64 db, {%2, %3};\n"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %4, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D(tmem) (+)= A(tmem) * B(smem), kind::f16, B's descriptor given as its
 // (low, high) words.
 __device__ __forceinline__ void mma_bf16_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
@@ -224,9 +241,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
 }
 
 // Instruction descriptor of kind::f8f6f4 with A and B e4m3 (format 0 in bits
-// 7-9 and 10-12), both K-major, fp32 accumulator; N >> 3, M >> 4 as above.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
-  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+// 7-9 and 10-12), A K-major, B K- or MN-major (bit 16; MN-major is valid for
+// e4m3), fp32 accumulator; N >> 3, M >> 4 as above.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool b_mn_major = false) {
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 
@@ -321,6 +340,14 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` in bits 0-15.
+// Two floats to two e4m3 codes (nearest even, saturating at 448): lo in the
+// low byte of the result.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -291,10 +291,26 @@ __device__ __forceinline__ void exp4(const float (&s)[128], int c, float scale_l
 }
 
 // p_c = 2^(s_c * scale_log2 - m) for the 128 columns, rounded to bf16 pairs
-// and written over the first 64 columns of S at `t_p` (tensor memory); returns
-// their fp32 sum. Waits for its tensor-memory stores before returning.
+// and written over the first 64 columns of S at `t_p` (tensor memory), or,
+// with kE4m3P, rounded to e4m3 (four per column) over the first 32; returns
+// their unrounded fp32 sum. Waits for its tensor-memory stores before
+// returning.
+template <bool kE4m3P>
 __device__ __forceinline__ float exp_tile_store(const float (&s)[128], float scale_log2, float neg_m, uint32_t t_p) {
   float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+  if constexpr (kE4m3P) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 128; c += 4) {
+      float e[4];
+      exp4(s, c, scale_log2, neg_m, e);
+      add2_acc(l0, l1, e[0], e[1]);
+      add2_acc(l2, l3, e[2], e[3]);
+      pk[c / 4] = pack_e4m3x2(e[0], e[1]) | (pack_e4m3x2(e[2], e[3]) << 16);
+    }
+    tmem_st_x32(t_p, pk);
+    return (l0 + l1) + (l2 + l3);
+  }
   uint32_t pk[64];
 #pragma unroll
   for (int c = 0; c < 128; c += 4) {
@@ -316,12 +332,13 @@ __device__ __forceinline__ float exp_tile_store(const float (&s)[128], float sca
   return (l0 + l1) + (l2 + l3);
 }
 
-template <int D, bool kSkip, bool kFp8>
+template <int D, bool kSkip, bool kFp8, bool kFp8Pv>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using L = Layout<D>;
   static_assert(!kFp8 || D == 128, "FP8 Q K^T: one 128-byte swizzle row per token");
+  static_assert(!kFp8Pv || (kFp8 && !kSkip), "FP8 P V comes with FP8 Q K^T, without block skipping");
   // FP8 Q K^T: the MMA thread waits for the next V stage (loaded long ago)
   // while it waits for P1 anyway, and probes the next K stage there without
   // blocking (its copy may still be in flight), instead of waiting for both
@@ -407,9 +424,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = load_idx % L::kStages;
             const uint32_t round = load_idx / L::kStages;
             if (round > 0 && !(ok = mbar_wait(kv_empty(s), (round - 1) & 1, abort_flag, p.timeout_ns))) break;
-            if (kFp8 && kv == 0) {
+            if ((kFp8 && kv == 0) || (kFp8Pv && kv == 1)) {
+              // one 128-byte e4m3 row per token: a single 16 KB box
               mbar_arrive_expect_tx(kv_full(s), kQKBytes);
-              tma_load_3d(kv_smem + s * L::kTileBytes, &tm_k, kv_full(s), 0, wk.head, wk.seg_start + j * kBN);
+              tma_load_3d(kv_smem + s * L::kTileBytes, kv == 0 ? &tm_k : &tm_v, kv_full(s), 0, wk.head,
+                          wk.seg_start + j * kBN);
             } else {
               mbar_arrive_expect_tx(kv_full(s), L::kTileBytes);
               const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
@@ -440,6 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdescQK = kFp8 ? idesc_e4m3_f32(kBM, kBN) : idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
+      constexpr uint32_t kIdescPV8 = idesc_e4m3_f32(kBM, D, true);
       uint32_t cons_idx = 0;
       uint32_t p_phase = 0;
       unsigned long long pv_skips = 0;
@@ -480,10 +500,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](int i, int stage, bool accumulate) {
         const uint32_t b0 = v_lo + stage * kTileWords;
         const uint32_t p_col = tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1);
+        if constexpr (kFp8Pv) {
+          // e4m3 P (four keys per column, 8 columns per K = 32 step) and V as
+          // 128-byte rows: MN-major, one swizzle atom wide, 32 keys = 4096 bytes
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
-          mma_bf16_ts_w(tmem + (i == 0 ? L::kTmemO0 : L::kTmemO1), p_col + 8 * k, b0 + ((k * 2048) >> 4), kDescHi,
-                        kIdescPV, (accumulate || k > 0) ? 1u : 0u);
+          for (int k = 0; k < kBN / 32; ++k)
+            mma_f8_ts_w(tmem + (i == 0 ? L::kTmemO0 : L::kTmemO1), p_col + 8 * k, b0 + ((k * 4096) >> 4), kDescHi,
+                        kIdescPV8, (accumulate || k > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int k = 0; k < kBN / 16; ++k) {
+            mma_bf16_ts_w(tmem + (i == 0 ? L::kTmemO0 : L::kTmemO1), p_col + 8 * k, b0 + ((k * 2048) >> 4),
+                          kDescHi, kIdescPV, (accumulate || k > 0) ? 1u : 0u);
+          }
         }
       };
       auto wait_stage = [&](uint32_t idx) {
@@ -643,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_x32(t_o + c0, ov);
           }
         }
-        l += exp_tile_store(s, sl2, -m, t_s);
+        l += exp_tile_store<kFp8Pv>(s, sl2, -m, t_s);
         tc_fence_before_sync();
         mbar_arrive(p_full(grp));
       }
@@ -652,7 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(o_done(grp), wt & 1, abort_flag, p.timeout_ns));
       if (!ok) break;
       tc_fence_after_sync();
-      const float inv_l = 1.0f / l;
+      // FP8 P V accumulates V's codes: its dequantisation factor comes in here
+      const float inv_l = (kFp8Pv ? p.deq[2 * p.H + wk.head] : 1.0f) / l;
       const bool valid_row = row < wk.seg_start + wk.seg_len;
       __nv_bfloat16* dst = p.o + static_cast<int64_t>(row) * p.o_stride + wk.head * D;
 #pragma unroll
@@ -750,13 +780,13 @@ bool make_e4m3_map(CUtensorMap* map, const void* ptr, int64_t T, int H, int D, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool kSkip, bool kFp8>
+template <int D, bool kSkip, bool kFp8, bool kFp8Pv>
 bool set_smem_attr() {
   static int done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kSkip, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kSkip, kFp8, kFp8Pv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Layout<D>::kAlloc) != cudaSuccess)
       return false;
     done[dev] = 1;
@@ -772,12 +802,13 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
                        int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
                        int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
                        long long timeout_ns, cudaStream_t stream, int num_sms, bool skip, float skip_tau,
-                       unsigned long long* skip_counts, const float* deq) {
+                       unsigned long long* skip_counts, const float* deq, bool fp8_pv) {
   CUtensorMap tq, tk, tv;
   const bool maps_ok = deq != nullptr
                            ? make_e4m3_map(&tq, q, T, H, D, q_stride) && make_e4m3_map(&tk, k, T, H, D, k_stride)
                            : make_qkv_map(&tq, q, T, H, D, q_stride) && make_qkv_map(&tk, k, T, H, D, k_stride);
-  if (!maps_ok || !make_qkv_map(&tv, v, T, H, D, v_stride)) return -2;
+  const bool v_ok = fp8_pv ? make_e4m3_map(&tv, v, T, H, D, v_stride) : make_qkv_map(&tv, v, T, H, D, v_stride);
+  if (!maps_ok || !v_ok) return -2;
   int32_t* sched = static_cast<int32_t*>(workspace);
   build_schedule_kernel<<<1, kSchedThreads, 0, stream>>>(cu_seqlens, B, T, H, sched, status);
   if (cudaGetLastError() != cudaSuccess) return -1;
@@ -797,26 +828,30 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
   // upper bound of work tiles: every request adds at most one partial block
   const int64_t max_work = static_cast<int64_t>(H) * ((T + kRowsPerWork - 1) / kRowsPerWork + B);
   const int grid = static_cast<int>(max_work < num_sms ? max_work : num_sms);
-  if (deq != nullptr && !skip) {
+  if (fp8_pv) {
+    if (D != 128 || deq == nullptr || skip) return -1;
+    if (!set_smem_attr<128, false, true, true>()) return -1;
+    attn_fwd_kernel<128, false, true, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+  } else if (deq != nullptr && !skip) {
     if (D != 128) return -1;
-    if (!set_smem_attr<128, false, true>()) return -1;
-    attn_fwd_kernel<128, false, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<128, false, true, false>()) return -1;
+    attn_fwd_kernel<128, false, true, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
   } else if (deq != nullptr) {
     if (D != 128) return -1;
-    if (!set_smem_attr<128, true, true>()) return -1;
-    attn_fwd_kernel<128, true, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<128, true, true, false>()) return -1;
+    attn_fwd_kernel<128, true, true, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
   } else if (D == 128 && !skip) {
-    if (!set_smem_attr<128, false, false>()) return -1;
-    attn_fwd_kernel<128, false, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<128, false, false, false>()) return -1;
+    attn_fwd_kernel<128, false, false, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
   } else if (D == 128) {
-    if (!set_smem_attr<128, true, false>()) return -1;
-    attn_fwd_kernel<128, true, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<128, true, false, false>()) return -1;
+    attn_fwd_kernel<128, true, false, false><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
   } else if (!skip) {
-    if (!set_smem_attr<64, false, false>()) return -1;
-    attn_fwd_kernel<64, false, false><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<64, false, false, false>()) return -1;
+    attn_fwd_kernel<64, false, false, false><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
   } else {
-    if (!set_smem_attr<64, true, false>()) return -1;
-    attn_fwd_kernel<64, true, false><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
+    if (!set_smem_attr<64, true, false, false>()) return -1;
+    attn_fwd_kernel<64, true, false, false><<<grid, kThreads, Layout<64>::kAlloc, stream>>>(tq, tk, tv, p);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

@@ -23,7 +23,8 @@ NORM_RMS, NORM_LAYER, NORM_NONE = 0, 1, 2
 
 # every symbol include/pqk.h declares
 EXPORTS = ("pqk_qk_norm_rope", "pqk_qk_norm_rope_3axis", "pqk_qk_fullc_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd",
-           "pqk_varlen_attn_fwd_skip", "pqk_quantize_qk_e4m3", "pqk_varlen_attn_fwd_fp8qk",
+           "pqk_varlen_attn_fwd_skip", "pqk_quantize_qk_e4m3", "pqk_varlen_attn_fwd_fp8qk", "pqk_quantize_e4m3",
+           "pqk_varlen_attn_fwd_fp8",
            "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu",
            "pqk_get_device_status", "pqk_set_wait_timeout_ns", "pqk_selftest_wait_timeout", "pqk_status_string",
            "pqk_version")
@@ -69,6 +70,10 @@ def lib(path: str | None = None) -> C.CDLL:
     L.pqk_varlen_attn_fwd_fp8qk.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, vp, i32, i64, i32, i32, f32, f32, vp,
                                             vp, sz, vp]
     L.pqk_varlen_attn_fwd_fp8qk.restype = i32
+    L.pqk_quantize_e4m3.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp]
+    L.pqk_quantize_e4m3.restype = i32
+    L.pqk_varlen_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, i32, i64, i32, i32, f32, vp, sz, vp]
+    L.pqk_varlen_attn_fwd_fp8.restype = i32
     L.pqk_varlen_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32,
                                               vp]
     L.pqk_varlen_attn_fwd_noalloc.restype = i32
@@ -261,6 +266,45 @@ def varlen_attn_fwd_fp8qk(q8, k8, v, deq, cu_seqlens, *, softmax_scale: float | 
         _ptr(q8), _ptr(k8), _ptr(v), _ptr(deq), _ptr(o), _ptr(lse), _token_stride(v, 3), _token_stride(o, 3),
         _ptr(cu_seqlens), B, T, H, D, scale, float(skip_threshold_log2), _ptr(skip_counts), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+def quantize_e4m3(x, *, x8=None, scales=None, stream=None):
+    """Per-head absmax e4m3 quantisation of one bf16 [T, H, D] tensor.
+    Returns (x8 uint8 [T, H, D], deq fp32 [H] view of ``scales``)."""
+    import torch
+    T, H, D = x.shape
+    if x8 is None:
+        x8 = torch.empty((T, H, D), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(2 * H, dtype=torch.float32, device=x.device)
+    assert x8.is_contiguous() and scales.numel() >= 2 * H
+    _check("pqk_quantize_e4m3", lib().pqk_quantize_e4m3(_ptr(x), _token_stride(x, 3), T, H, D, _ptr(x8),
+                                                         _ptr(scales), _stream(stream)))
+    return x8, scales[H:2 * H]
+
+
+def varlen_attn_fwd_fp8(q8, k8, v8, deq, cu_seqlens, *, softmax_scale: float | None = None, o=None, lse=None,
+                        workspace=None, want_lse: bool = False, stream=None):
+    """The attention with Q K^T and P V on the FP8 tensor cores: q8, k8, v8
+    e4m3 bytes [T, H, D]; deq fp32 [3H] (Q's, K's, V's factors). Returns
+    (o bf16 [T, H, D], lse or None)."""
+    import torch
+    T, H, D = q8.shape
+    B = cu_seqlens.shape[0] - 1
+    scale = softmax_scale if softmax_scale is not None else D ** -0.5
+    if o is None:
+        o = torch.empty((T, H, D), dtype=torch.bfloat16, device=q8.device)
+    if lse is None and want_lse:
+        lse = torch.empty((H, T), dtype=torch.float32, device=q8.device)
+    if workspace is None:
+        workspace = torch.empty(varlen_attn_workspace_size(B), dtype=torch.uint8, device=q8.device)
+    for t in (q8, k8, v8):
+        assert t.is_contiguous() and tuple(t.shape) == (T, H, D)
+    assert deq.is_contiguous() and deq.numel() >= 3 * H
+    _check("pqk_varlen_attn_fwd_fp8", lib().pqk_varlen_attn_fwd_fp8(
+        _ptr(q8), _ptr(k8), _ptr(v8), _ptr(deq), _ptr(o), _ptr(lse), _token_stride(o, 3), _ptr(cu_seqlens), B, T, H,
+        D, scale, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return o, lse
 
 

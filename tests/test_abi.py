@@ -227,3 +227,23 @@ def test_varlen_attn_fp8qk_host_errors(L):
     assert call(tau=float("nan")) == ERR_INVALID
     assert call(counts=A + 4) == ERR_MISALIGNED
     assert call(T=0, q8=None) == 0
+
+
+def test_quantize_e4m3_and_fp8_attention_host_errors(L):
+    assert L.pqk_quantize_e4m3(A, 1024, 16, 8, 96, A, A, None) == ERR_UNSUPPORTED
+    assert L.pqk_quantize_e4m3(A, 1000, 16, 8, 128, A, A, None) == ERR_INVALID
+    assert L.pqk_quantize_e4m3(A, 1024, 16, 8, 128, U, A, None) == ERR_MISALIGNED
+    assert L.pqk_quantize_e4m3(A, 1024, 16, 8, 128, A, None, None) == ERR_INVALID
+
+    def call(**kw):
+        a = dict(q8=A, k8=A, v8=A, deq=A, o=A, lse=None, os_=1024, cu=A, B=2, T=512, H=8, D=128, scale=0.088, ws=A,
+                 wsb=4096)
+        a.update(kw)
+        return L.pqk_varlen_attn_fwd_fp8(a["q8"], a["k8"], a["v8"], a["deq"], a["o"], a["lse"], a["os_"], a["cu"],
+                                         a["B"], a["T"], a["H"], a["D"], a["scale"], a["ws"], a["wsb"], None)
+    assert call(D=64, os_=512) == ERR_UNSUPPORTED
+    assert call(v8=None) == ERR_INVALID
+    assert call(v8=U) == ERR_MISALIGNED
+    assert call(os_=512) == ERR_INVALID
+    assert call(ws=None) == ERR_WORKSPACE
+    assert call(T=0, q8=None) == 0

@@ -175,3 +175,89 @@ def test_joint_sequence_58048_sampled():
     ro, rl, _, _, _ = oracle.varlen_attn_fp8qk(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, rows=rows)
     assert_attention(bf16_to_f64(o)[rows], ro, "fp8 58,048 tokens sampled")
     assert max_abs(lse.cpu().numpy().astype(np.float64).T[rows], rl) <= LSE_MAX_ABS
+
+
+# ---------------------------------------------------------------- Q, K, V and P in FP8
+
+def _full_fp8_gpu(x, scale):
+    torch = torch_cuda()
+    q8, k8, deq_qk = _quantise_gpu(x)
+    v8, deq_v = pqk.quantize_e4m3(to_dev_bf16(x["v"]))
+    deq = torch.cat([deq_qk, deq_v]).contiguous()
+    o, lse = pqk.varlen_attn_fwd_fp8(q8, k8, v8, deq, to_dev(x["cu_seqlens"]), softmax_scale=scale, want_lse=True)
+    torch.cuda.synchronize()
+    assert pqk.get_device_status() == 0
+    return o, lse, v8, deq
+
+
+def _check_full_fp8(x, scale, what, rows=None):
+    """Element-wise against the oracle, each row allowed, beyond the attention
+    tolerance, one e4m3 step (2^-4 relative) of its largest-weight key: the
+    kernel rounds fp32 probabilities, the oracle float64 ones, so a value
+    lying on an e4m3 rounding boundary may round differently."""
+    o, lse, v8, deq = _full_fp8_gpu(x, scale)
+    ro, rl, rdeq = oracle.varlen_attn_fp8(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, rows=rows)
+    T, H, D = x["q"].shape
+    assert np.array_equal(deq.cpu().numpy(), rdeq)
+    sel = np.arange(T) if rows is None else rows
+    g = bf16_to_f64(o)[sel]
+    assert rel_l2(g, ro) <= 1e-2, what
+    # largest softmax weight per (row, head), from the dequantised Q, K
+    q8, k8, _ = _quantise_gpu(x)
+    dq = deq.cpu().numpy().astype(np.float64)
+    import torch
+    dec = lambda c: torch.from_numpy(c.cpu().numpy()).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    qd, kd = dec(q8) * dq[None, :H, None], dec(k8) * dq[None, H:2 * H, None]
+    vmax = float(np.abs(dec(v8)).max() * dq[2 * H:].max())
+    cu = x["cu_seqlens"]
+    for n, t in enumerate(sel):
+        i = int(np.searchsorted(cu, t, side="right") - 1)
+        lo, hi = int(cu[i]), int(cu[i + 1])
+        for h in range(H):
+            s = scale * (kd[lo:hi, h] @ qd[t, h])
+            wmax = float(np.exp(s - s.max()).max() / np.exp(s - s.max()).sum())
+            err = float(np.max(np.abs(g[n, h] - ro[n, h])))
+            assert err <= 2e-2 + 2.0 ** -3 * wmax * vmax, f"{what}: row {t} head {h} error {err:.3e}"
+    assert max_abs(lse.cpu().numpy().astype(np.float64).T[sel], rl) <= LSE_MAX_ABS
+
+
+def test_v_quantisation_is_bitwise_the_oracle():
+    torch = torch_cuda()
+    w = wl.custom([300, 0, 513, 1], 3, 128, seed=41)
+    x = wl.attention_inputs(w)
+    v8, deq = pqk.quantize_e4m3(to_dev_bf16(x["v"]))
+    torch.cuda.synchronize()
+    rc, rd = oracle.quantize_e4m3(x["v"])
+    assert np.array_equal(v8.cpu().numpy(), rc) and np.array_equal(deq.cpu().numpy(), rd)
+
+
+@pytest.mark.parametrize("lens", [[1], [129], [255, 256, 257], [300, 0, 513, 1], [384, 17, 2, 640]])
+def test_full_fp8_attention(lens):
+    w = wl.custom(lens, 3, 128, seed=sum(lens) + 43)
+    _check_full_fp8(wl.attention_inputs(w), 1.0 / math.sqrt(128), f"full fp8 {lens}")
+
+
+def test_full_fp8_attention_peaked():
+    w = wl.custom([700, 1300], 2, 128, seed=44)
+    x = wl.attention_inputs(w)
+    x["q"] = wl.f32_to_bf16_bits(wl.bf16_bits_to_f32(x["q"]) * np.float32(8.0))
+    _check_full_fp8(x, 1.0 / math.sqrt(128), "full fp8 peaked")
+
+
+def test_full_fp8_attention_16k_sampled_and_error_against_bf16():
+    w = wl.custom([16384], 4, 128, seed=45)
+    x = wl.attention_inputs(w)
+    rows = wl.sample_rows(w, per_segment=64)
+    _check_full_fp8(x, 1.0 / math.sqrt(128), "full fp8 16k", rows=rows)
+    ro, _, _ = oracle.varlen_attn_fp8(x["q"], x["k"], x["v"], x["cu_seqlens"], 1.0 / math.sqrt(128), rows=rows)
+    po, _ = oracle.varlen_attn(x["q"], x["k"], x["v"], x["cu_seqlens"], 1.0 / math.sqrt(128), rows=rows)
+    assert 1e-4 < rel_l2(ro, po) < 0.1
+
+
+def test_full_fp8_attention_is_deterministic():
+    torch = torch_cuda()
+    w = wl.custom([1000, 2000], 4, 128, seed=46)
+    x = wl.attention_inputs(w)
+    a = [_full_fp8_gpu(x, 0.1) for _ in range(3)]
+    for o, lse, _, _ in a[1:]:
+        assert torch.equal(o.view(torch.int16), a[0][0].view(torch.int16)) and torch.equal(lse, a[0][1])
