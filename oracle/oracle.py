@@ -63,11 +63,15 @@ def load(path: str):
                                            C.POINTER(C.c_int64), u8p, u8p, f32p]
     L.oracle_varlen_attn_fp8.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
                                          C.c_int, C.c_double, i32p, C.c_int64, f64p, f64p, f32p]
+    L.oracle_linear_gated_residual.argtypes = [vp, C.c_int64, vp, vp, C.c_int, f32p, i32p, C.c_int, C.c_int64,
+                                               C.c_int, C.c_int, i32p, C.c_int64, f64p]
+    L.oracle_linear_swiglu.argtypes = [vp, C.c_int64, vp, C.c_int, C.c_int64, C.c_int, C.c_int, i32p, C.c_int64,
+                                       f64p]
     L.oracle_e4m3_codes.argtypes = [f32p, C.c_int64, u8p]
     L.oracle_e4m3_codes.restype = None
     for f in (L.oracle_qk_norm_rope, L.oracle_qk_norm_rope_3axis, L.oracle_qk_fullc_norm_rope, L.oracle_varlen_attn,
               L.oracle_varlen_attn_skip, L.oracle_quantize_e4m3, L.oracle_varlen_attn_fp8qk, L.oracle_varlen_attn_fp8,
-              L.oracle_modulate_swiglu):
+              L.oracle_modulate_swiglu, L.oracle_linear_gated_residual, L.oracle_linear_swiglu):
         f.restype = C.c_int
     L.oracle_num_threads.restype = C.c_int
     return L
@@ -311,3 +315,51 @@ def modulate_swiglu(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, gate_re
     if rc:
         raise ValueError("oracle_modulate_swiglu: invalid arguments")
     return xo, h, act
+
+
+def _token_rows(a: np.ndarray):
+    """A [T, K] array whose rows may be a strided view: (array, row stride)."""
+    assert a.ndim == 2 and a.strides[1] == a.itemsize
+    return a, a.strides[0] // a.itemsize
+
+
+def linear_gated_residual(a: np.ndarray, w: np.ndarray, x=None, gate_res=None, cu_seqlens=None, rows=None):
+    """x + gate_res[request] * (a @ w.T) per token (a: [T, K], w: [N, K],
+    x: [T, N]); with x None the product alone. float64 [rows, N]."""
+    a, a_stride = _token_rows(a)
+    T, K = a.shape
+    w = np.ascontiguousarray(w)
+    N = w.shape[0]
+    assert w.shape == (N, K) and w.dtype == a.dtype
+    B, cu, g = 0, None, None
+    if x is not None:
+        x = np.ascontiguousarray(x)
+        assert x.shape == (T, N) and x.dtype == a.dtype
+        g = np.ascontiguousarray(gate_res, dtype=np.float32)
+        cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+        B = int(cu.shape[0]) - 1
+        assert g.shape == (B, N)
+    r, n = _rows(rows)
+    out = np.empty((n if r is not None else T, N), np.float64)
+    rc = lib().oracle_linear_gated_residual(_ptr(a), a_stride, _ptr(w), _ptr(x), _kind(a), _ptr(g, C.c_float),
+                                            _ptr(cu, C.c_int32), B, T, K, N, _ptr(r, C.c_int32), n, _ptr(out, C.c_double))
+    if rc:
+        raise ValueError("oracle_linear_gated_residual: invalid arguments")
+    return out
+
+
+def linear_swiglu(a: np.ndarray, w1: np.ndarray, rows=None):
+    """silu(a @ w1[:F].T) * (a @ w1[F:].T) per token (a: [T, K], w1: [2F, K]).
+    float64 [rows, F]."""
+    a, a_stride = _token_rows(a)
+    T, K = a.shape
+    w1 = np.ascontiguousarray(w1)
+    assert w1.ndim == 2 and w1.shape[1] == K and w1.shape[0] % 2 == 0 and w1.dtype == a.dtype
+    F = w1.shape[0] // 2
+    r, n = _rows(rows)
+    act = np.empty((n if r is not None else T, F), np.float64)
+    rc = lib().oracle_linear_swiglu(_ptr(a), a_stride, _ptr(w1), _kind(a), T, K, F, _ptr(r, C.c_int32), n,
+                                    _ptr(act, C.c_double))
+    if rc:
+        raise ValueError("oracle_linear_swiglu: invalid arguments")
+    return act

@@ -33,6 +33,10 @@
  *                             SwiGLU in place of separate SiLU and multiply
  *                             (first page "融合 DiT 算子"; second page bullet
  *                             "Fused DiT operators").
+ *   oracle_linear_gated_residual, oracle_linear_swiglu -- the linear
+ *                             layers around them with the gated residual or
+ *                             SwiGLU as their epilogue (same passages; the
+ *                             fusion into the GEMM is a reading).
  *
  * The pages state the operations, not their conventions; the readings taken
  * where they are silent (norm per head over head_dim, norm before RoPE,
@@ -710,6 +714,74 @@ int oracle_modulate_swiglu(const void* x, const void* branch, int in_kind, const
       }
     }
     free(xp);
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * A linear layer whose epilogue is the gated residual: the output
+ * projection after attention (or W2 after SwiGLU) followed by the residual
+ * add with the adaLN gate, the fusion of residual connections into fewer
+ * launches ("FastH3 在八卡 B300 上实现完整 MP4 生成快于播放时长", section
+ * "融合 DiT 算子"; "MiniMax H3 FastH3 real-time serving with vLLM-Omni",
+ * bullet "Fused DiT operators"). Per token t of request s and feature n:
+ *   y[t, n]  = sum_k a[t, k] * w[n, k]         (w: [N, K], out x in features)
+ *   x'[t, n] = x[t, n] + gate_res[s, n] * y[t, n]
+ * x == NULL: the product alone (x' = y; gate_res and cu unused).
+ * a: [T, K] with a_stride elements between tokens; x: [T, N]; gate_res:
+ * [B, N] float32. Output float64 rows [nrows, N] for the tokens in rows
+ * (all T when rows is NULL).
+ */
+int oracle_linear_gated_residual(const void* a, int64_t a_stride, const void* w, const void* x, int in_kind,
+                                 const float* gate_res, const int32_t* cu, int B, int64_t T, int K, int N,
+                                 const int32_t* rows, int64_t nrows, double* out) {
+  if (T < 0 || K <= 0 || N <= 0 || a_stride < K) return -1;
+  if (x && (gate_res == NULL || check_cu(cu, B, T))) return -1;
+  if (rows == NULL) nrows = T;
+  int64_t bad = 0;
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t t = rows ? rows[r] : r;
+    if (t < 0 || t >= T) { ++bad; continue; }
+    const int seg = x ? segment_of(cu, B, t) : 0;
+    for (int n = 0; n < N; ++n) {
+      double y = 0.0;
+      for (int k = 0; k < K; ++k) y += load(a, in_kind, t * a_stride + k) * load(w, in_kind, (int64_t)n * K + k);
+      out[r * N + n] = x ? load(x, in_kind, t * N + n) + (double)gate_res[(int64_t)seg * N + n] * y : y;
+    }
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * A linear layer whose epilogue is SwiGLU: W1 of the feed-forward with
+ * silu(gate) * up applied to its two halves in place of separate SiLU and
+ * multiply passes (same passages). The first F rows of w1 give the SiLU
+ * operand, the last F rows the linear one. Per token t and feature f:
+ *   g = sum_k a[t, k] * w1[f, k]
+ *   u = sum_k a[t, k] * w1[F + f, k]
+ *   act[t, f] = g / (1 + exp(-g)) * u     (gv, uv below)
+ * a: [T, K] with a_stride elements between tokens; w1: [2F, K]. Output
+ * float64 rows [nrows, F].
+ */
+int oracle_linear_swiglu(const void* a, int64_t a_stride, const void* w1, int in_kind, int64_t T, int K, int F,
+                         const int32_t* rows, int64_t nrows, double* act) {
+  if (T < 0 || K <= 0 || F <= 0 || a_stride < K) return -1;
+  if (rows == NULL) nrows = T;
+  int64_t bad = 0;
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t t = rows ? rows[r] : r;
+    if (t < 0 || t >= T) { ++bad; continue; }
+    for (int f = 0; f < F; ++f) {
+      double gv = 0.0, uv = 0.0;
+      for (int k = 0; k < K; ++k) {
+        const double av = load(a, in_kind, t * a_stride + k);
+        gv += av * load(w1, in_kind, (int64_t)f * K + k);
+        uv += av * load(w1, in_kind, ((int64_t)F + f) * K + k);
+      }
+      act[r * (int64_t)F + f] = gv / (1.0 + exp(-gv)) * uv;
+    }
   }
   return bad ? -1 : 0;
 }

@@ -15,8 +15,8 @@ import subprocess
 import pytest
 
 from oracle import oracle
-from tests import (test_oracle_attention, test_oracle_fp8, test_oracle_fullc, test_oracle_modulate,
-                   test_oracle_norm_rope, test_oracle_rope3, test_oracle_skip)
+from tests import (test_oracle_attention, test_oracle_fp8, test_oracle_fullc, test_oracle_linear,
+                   test_oracle_modulate, test_oracle_norm_rope, test_oracle_rope3, test_oracle_skip)
 
 MUTANTS = {
     "attn_drop_scale": ("s[j] = scale * acc;", "s[j] = acc;"),
@@ -69,6 +69,15 @@ MUTANTS = {
     "fp8_numerator_not_rescaled": ("      for (int d = 0; d < D; ++d) num[d] *= alpha;\n", ""),
     "fp8_v_with_q_scale": ("xd[i][e] = e4m3_value(c8[e]) * (double)dq[(int64_t)i * H + (e / D) % H];",
                            "xd[i][e] = e4m3_value(c8[e]) * (double)dq[(e / D) % H];"),
+    "linear_w_transposed": ("load(w, in_kind, (int64_t)n * K + k)", "load(w, in_kind, (int64_t)k * N + n)"),
+    "linear_gate_of_first_request": ("(double)gate_res[(int64_t)seg * N + n] * y", "(double)gate_res[n] * y"),
+    "linear_residual_sign": ("load(x, in_kind, t * N + n) + (double)gate_res", "load(x, in_kind, t * N + n) - (double)gate_res"),
+    "linear_a_stride_ignored": ("y += load(a, in_kind, t * a_stride + k)", "y += load(a, in_kind, t * K + k)"),
+    "linear_drop_last_k": ("for (int k = 0; k < K; ++k) y += ", "for (int k = 0; k < K - 1; ++k) y += "),
+    "linear_swiglu_halves_swapped": ("act[r * (int64_t)F + f] = gv / (1.0 + exp(-gv)) * uv;",
+                                     "act[r * (int64_t)F + f] = uv / (1.0 + exp(-uv)) * gv;"),
+    "linear_swiglu_up_from_gate_rows": ("uv += av * load(w1, in_kind, ((int64_t)F + f) * K + k);",
+                                        "uv += av * load(w1, in_kind, (int64_t)f * K + k);"),
     "skip_tile_counts_any_block": ("if (keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;",
                                    "if (!keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;"),
 }
@@ -76,7 +85,7 @@ MUTANTS = {
 
 def _pin_calls():
     for mod in (test_oracle_attention, test_oracle_norm_rope, test_oracle_modulate, test_oracle_rope3,
-                test_oracle_fullc, test_oracle_skip, test_oracle_fp8):
+                test_oracle_fullc, test_oracle_skip, test_oracle_fp8, test_oracle_linear):
         for name, fn in inspect.getmembers(mod, inspect.isfunction):
             if not name.startswith("test_") or fn.__module__ != mod.__name__:
                 continue
