@@ -20,7 +20,10 @@ After the timed steps the same line also carries, under ``kernels``: the
 three-axis RoPE, back-to-back and full-width norm timings; the block-
 skipping attention on the local-attention stand-in (``--skip-tau``, plain
 vs skipping vs FP8 Q K^T with and without skipping); the FP8 Q K^T attention
-on the step's inputs (``--no-fp8`` leaves it out); and, with ``--graph``,
+on the step's inputs (``--no-fp8`` leaves it out); the block's three linear
+layers with the gated residual or SwiGLU in the GEMM epilogue, on the step's
+own activations, against cuBLAS plus torch epilogues (``linear_epilogue``;
+``--no-linear`` leaves it out); and, with ``--graph``,
 the step replayed as a CUDA graph (``graph_ms_per_step``). ``--config N``
 selects another configuration, ``--sweep`` the HBM bandwidth sweep.
 """
@@ -68,6 +71,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="leave out the FP8 Q K^T attention timing")
+    ap.add_argument("--no-linear", action="store_true",
+                    help="leave out the linear layers with the fused epilogues (gated residual, SwiGLU)")
     ap.add_argument("--graph", action="store_true",
                     help="also time the block call captured once in a CUDA graph and replayed (graph_ms_per_step)")
     ap.add_argument("--skip-tau", type=float, default=8.0,
@@ -207,6 +212,82 @@ def block_call(w, d, o, ev=None):
 
 
 LAUNCHES_PER_STEP = 4  # qk_norm_rope, schedule builder, attention, modulate_swiglu
+
+
+def time_linear_layers(w, d, o, pk, pk_kind, reps=3):
+    """The block's three linear layers with their fused epilogues on the
+    step's own activations (attention output, h, act) and random-init
+    weights: the output projection and W2 with the gated residual, W1 with
+    SwiGLU. Each is timed against cuBLAS (torch's linear) followed by the
+    same epilogue as torch element-wise kernels, and the GEMM alone (ours
+    without epilogue vs cuBLAS)."""
+    import torch
+    import torch.nn.functional as Fnn
+    from packed_attention_qk_b200 import pqk
+    from packed_attention_qk_b200 import workloads as wl
+    dev = d["x"].device
+
+    def dev_w(name, n_out, n_in):
+        bits = wl.bf16_linear_weight(w.seed, name, n_out, n_in)
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    T, Cd, F = w.T, w.C, w.F
+    w_o, w1, w2 = dev_w("w_o", Cd, Cd), dev_w("w1", 2 * F, Cd), dev_w("w2", Cd, F)
+    a_o = o["o"].view(T, w.H * w.D)
+    x, gr, cu = d["x"], d["gate_res"], d["cu"]
+    # torch's epilogue broadcasts one gate row (one request) or gathers one per token
+    gr_tok = gr[0] if w.B == 1 else torch.repeat_interleave(gr, torch.tensor(w.seg_lens, device=dev), dim=0)
+    out_c, out_f = torch.empty_like(x), torch.empty_like(o["act"])
+    layers = {
+        "o_proj": (lambda: pqk.linear_gated_residual(a_o, w_o, x=x, gate_res=gr, cu_seqlens=cu, out=out_c),
+                   lambda: pqk.linear_gated_residual(a_o, w_o, out=out_c),
+                   lambda: Fnn.linear(a_o, w_o),
+                   lambda: torch.addcmul(x, gr_tok, Fnn.linear(a_o, w_o)),
+                   2.0 * T * (w.H * w.D) * Cd),
+        "w1_swiglu": (lambda: pqk.linear_swiglu(o["h"], w1, act=out_f),
+                      None,
+                      lambda: Fnn.linear(o["h"], w1),
+                      lambda: (lambda y: Fnn.silu(y[:, :F]) * y[:, F:])(Fnn.linear(o["h"], w1)),
+                      2.0 * T * Cd * 2 * F),
+        "w2": (lambda: pqk.linear_gated_residual(o["act"], w2, x=x, gate_res=gr, cu_seqlens=cu, out=out_c),
+               lambda: pqk.linear_gated_residual(o["act"], w2, out=out_c),
+               lambda: Fnn.linear(o["act"], w2),
+               lambda: torch.addcmul(x, gr_tok, Fnn.linear(o["act"], w2)),
+               2.0 * T * F * Cd),
+    }
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def ms(fn):
+        fn()
+        torch.cuda.synchronize()
+        ev[0].record()
+        for _ in range(reps):
+            fn()
+        ev[1].record()
+        torch.cuda.synchronize()
+        return ev[0].elapsed_time(ev[1]) / reps
+
+    res, fused_total, unfused_total, flops_total = {}, 0.0, 0.0, 0.0
+    for name, (fused, gemm_only, cublas, cublas_epi, flops) in layers.items():
+        f_ms = ms(fused)
+        r = {"fused_ms": f_ms, "fused_tflops": flops / (f_ms * 1e-3) / 1e12,
+             "cublas_gemm_ms": ms(cublas), "cublas_plus_torch_epilogue_ms": ms(cublas_epi)}
+        if gemm_only is not None:
+            r["gemm_only_ms"] = ms(gemm_only)
+        r["speedup_vs_cublas_plus_epilogue"] = r["cublas_plus_torch_epilogue_ms"] / f_ms
+        res[name] = r
+        fused_total += f_ms
+        unfused_total += r["cublas_plus_torch_epilogue_ms"]
+        flops_total += flops
+    if pqk.get_device_status() != 0:
+        raise RuntimeError("device status set during the linear-layer timing")
+    tflops = flops_total / (fused_total * 1e-3) / 1e12
+    res.update({"fused_total_ms": fused_total, "unfused_total_ms": unfused_total,
+                "speedup_vs_cublas_plus_epilogue": unfused_total / fused_total, "fused_tflops": tflops,
+                "frac_of_bf16_burst": tflops / pk["bf16_tflops"], "peak_kind": f"{pk_kind} bf16 burst",
+                "weights": "random-init N(0, 1/in) bf16"})
+    del w_o, w1, w2, out_c, out_f
+    return res
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -512,6 +593,10 @@ def run_ours(args, w):
                "full_fp8_attn_ms": full_ms, "full_fp8_speedup_vs_bf16": att_ms / full_ms}
         del q8, k8, v8, fo
 
+    lin = None
+    if not args.no_linear and w.H * w.D == w.C:
+        lin = time_linear_layers(w, d, o, pk, pk_kind)
+
     # e2e through host buffers: every step copies all of its inputs from
     # pinned host memory to the device (H2D stream), runs the three C-ABI
     # calls (compute stream) and copies its outputs x', h, act back to pinned
@@ -612,7 +697,7 @@ def run_ours(args, w):
                     "qk_norm_rope_back_to_back_us": rope1_b2b_us,
                     "qk_fullc_norm_rope_us": fullc_us, "qk_fullc_norm_rope_gbs": fullc_gbs,
                     "qk_fullc_norm_rope_frac_hbm": fullc_gbs / pk["hbm_gbs"],
-                    "varlen_attn_skip": skip, "varlen_attn_fp8qk": fp8},
+                    "varlen_attn_skip": skip, "varlen_attn_fp8qk": fp8, "linear_epilogue": lin},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * K,

@@ -347,6 +347,56 @@ PQK_API int pqk_modulate_swiglu(const void* x, const void* branch, void* x_out, 
                         void* act, int F, void* stream);
 
 /*
+ * pqk_linear_gated_residual -- a linear layer whose epilogue is the gated
+ * residual: the output projection after attention (or W2 after SwiGLU)
+ * with the residual add of the adaLN-gated branch done on the GEMM's fp32
+ * accumulator, instead of writing the branch and re-reading it (first
+ * page, section "融合 DiT 算子": residual connections among the fused DiT
+ * operators; second page, bullet "Fused DiT operators"). For every token t
+ * of request s:
+ *   out[t, n] = x[t, n] + gate_res[s, n] * sum_k a[t, k] * w[n, k]
+ * With x and gate_res both NULL: out = a w^T (the product alone; cu_seqlens
+ * and B unused). tcgen05 tensor cores, fp32 accumulation, bf16 output
+ * rounded to nearest even.
+ *
+ * a           device bf16 [T, K], rows a_stride_t elements apart.
+ * w           device bf16 [N, K] contiguous (out x in features).
+ * x           device bf16 [T, N], rows x_stride_t apart, or NULL.
+ * gate_res    device fp32 [B, N] (one gate per request), or NULL with x.
+ * cu_seqlens  device int32 [B+1] (must be valid; not re-checked here).
+ * out         device bf16 [T, N], rows out_stride_t apart; may equal x
+ *             (same stride); no other overlap with an input.
+ * K, N        multiples of 8, >= 8; T <= 2^31 - 257. Pointers 16-byte
+ *             aligned, strides multiples of 8 elements.
+ * Errors: PQK_ERR_INVALID_ARG / PQK_ERR_MISALIGNED before anything is
+ * enqueued; a pipeline wait that runs out records PQK_ERR_TIMEOUT in the
+ * device status word (see pqk_get_device_status).
+ */
+PQK_API int pqk_linear_gated_residual(const void* a, int64_t a_stride_t, const void* w, const void* x,
+                                      int64_t x_stride_t, const float* gate_res, const int32_t* cu_seqlens,
+                                      int B, void* out, int64_t out_stride_t, int64_t T, int K, int N,
+                                      void* stream);
+
+/*
+ * pqk_linear_swiglu -- W1 of the feed-forward with SwiGLU as its epilogue:
+ * silu(gate) * up computed from the GEMM's fp32 accumulators, so that the
+ * [T, 2F] product is never written (first page, section "融合 DiT 算子":
+ * SwiGLU in place of separate SiLU and multiply; second page, bullet
+ * "Fused DiT operators"). The first F rows of w1 give the SiLU operand, the
+ * last F rows the linear one:
+ *   act[t, f] = silu(sum_k a[t, k] w1[f, k]) * sum_k a[t, k] w1[F + f, k],
+ *   silu(g) = g / (1 + exp(-g)).
+ *
+ * a           device bf16 [T, K], rows a_stride_t elements apart.
+ * w1          device bf16 [2F, K] contiguous.
+ * act         device bf16 [T, F], rows act_stride_t apart.
+ * K, F        multiples of 8, >= 8. Alignment and errors as
+ *             pqk_linear_gated_residual.
+ */
+PQK_API int pqk_linear_swiglu(const void* a, int64_t a_stride_t, const void* w1, void* act, int64_t act_stride_t,
+                              int64_t T, int K, int F, void* stream);
+
+/*
  * pqk_get_device_status -- synchronises `stream`, then returns and clears
  * the current device's status word: PQK_OK, PQK_ERR_TIMEOUT or
  * PQK_ERR_BAD_SEQLENS (the first condition recorded since the last read),
@@ -356,7 +406,7 @@ PQK_API int pqk_get_device_status(void* stream);
 
 /*
  * pqk_set_wait_timeout_ns -- upper bound, in nanoseconds, on every wait of
- * the attention pipeline (default 1e9). A wait that runs out records
+ * the attention and linear-layer pipelines (default 1e9). A wait that runs out records
  * PQK_ERR_TIMEOUT, its thread block stops issuing work, waits (again
  * bounded) for its copies in flight, frees its tensor memory and exits.
  * Values <= 0 restore the default. Affects calls enqueued afterwards.

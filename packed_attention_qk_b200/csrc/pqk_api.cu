@@ -315,6 +315,43 @@ int pqk_modulate_swiglu(const void* x, const void* branch, void* x_out, void* h,
              : PQK_OK;
 }
 
+int pqk_linear_gated_residual(const void* a, int64_t a_stride_t, const void* w, const void* x, int64_t x_stride_t,
+                              const float* gate_res, const int32_t* cu_seqlens, int B, void* out,
+                              int64_t out_stride_t, int64_t T, int K, int N, void* stream) {
+  if (T < 0 || T > INT32_MAX - 256 || K < 8 || N < 8 || K % 8 || N % 8) return PQK_ERR_INVALID_ARG;
+  const bool residual = x != nullptr || gate_res != nullptr;
+  if (residual && (x == nullptr || gate_res == nullptr || cu_seqlens == nullptr || B < 1 || x_stride_t < N))
+    return PQK_ERR_INVALID_ARG;
+  if (a_stride_t < K || out_stride_t < N) return PQK_ERR_INVALID_ARG;
+  if (T == 0) return PQK_OK;
+  if (!a || !w || !out) return PQK_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(out) || !aligned16(x) || !aligned16(gate_res) ||
+      (a_stride_t % 8) || (out_stride_t % 8) || (residual && (x_stride_t % 8)))
+    return PQK_ERR_MISALIGNED;
+  DeviceInfo* d = nullptr;
+  if (int rc = check_device(&d)) return rc;
+  const int rc = pqk::launch_linear(residual ? pqk::kEpiGatedResidual : pqk::kEpiNone, a, a_stride_t, w, x,
+                                    x_stride_t, gate_res, cu_seqlens, B, out, out_stride_t, T, K, N, d->status,
+                                    g_timeout_ns.load(), static_cast<cudaStream_t>(stream), d->num_sms);
+  return rc == 0 ? PQK_OK : (rc == -2 ? PQK_ERR_INVALID_ARG : PQK_ERR_CUDA);
+}
+
+int pqk_linear_swiglu(const void* a, int64_t a_stride_t, const void* w1, void* act, int64_t act_stride_t, int64_t T,
+                      int K, int F, void* stream) {
+  if (T < 0 || T > INT32_MAX - 256 || K < 8 || F < 8 || K % 8 || F % 8) return PQK_ERR_INVALID_ARG;
+  if (a_stride_t < K || act_stride_t < F) return PQK_ERR_INVALID_ARG;
+  if (T == 0) return PQK_OK;
+  if (!a || !w1 || !act) return PQK_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w1) || !aligned16(act) || (a_stride_t % 8) || (act_stride_t % 8))
+    return PQK_ERR_MISALIGNED;
+  DeviceInfo* d = nullptr;
+  if (int rc = check_device(&d)) return rc;
+  const int rc = pqk::launch_linear(pqk::kEpiSwiglu, a, a_stride_t, w1, nullptr, 0, nullptr, nullptr, 0, act,
+                                    act_stride_t, T, K, F, d->status, g_timeout_ns.load(),
+                                    static_cast<cudaStream_t>(stream), d->num_sms);
+  return rc == 0 ? PQK_OK : (rc == -2 ? PQK_ERR_INVALID_ARG : PQK_ERR_CUDA);
+}
+
 int pqk_get_device_status(void* stream) {
   DeviceInfo* d = current_device();
   if (d == nullptr) return PQK_ERR_CUDA;

@@ -57,6 +57,19 @@ int launch_quantize_qk_e4m3(const void* q, const void* k, int64_t q_stride, int6
 int launch_quantize_e4m3(const void* x, int64_t x_stride, int64_t T, int H, int D, void* x8, float* scales,
                          cudaStream_t stream, int num_sms);
 
+// Epilogues of the linear-layer GEMM (launch_linear).
+constexpr int kEpiNone = 0;           // out = A W^T
+constexpr int kEpiGatedResidual = 1;  // out = x + gate_res[request] * (A W^T)
+constexpr int kEpiSwiglu = 2;         // out = silu(A W[:N]^T) * (A W[N:]^T), W [2N, K]
+
+// Persistent tcgen05 GEMM out[T, N] = epilogue(A[T, K] W^T) with bf16 A, W
+// (W row-major [N, K], or [2N, K] for SwiGLU) and bf16 out. x, gate_res, cu
+// and B are used by the gated residual only. Returns 0, -1 when a CUDA call
+// failed, -2 when the tensor maps could not be encoded.
+int launch_linear(int epi, const void* a, int64_t a_stride, const void* w, const void* x, int64_t x_stride,
+                  const float* gate_res, const int32_t* cu, int B, void* out, int64_t out_stride, int64_t T, int K,
+                  int N, int* status, long long timeout_ns, cudaStream_t stream, int num_sms);
+
 int launch_wait_selftest(int* status, long long timeout_ns, cudaStream_t stream);
 
 // Status codes written by kernels into the device status word (same values

@@ -105,6 +105,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 2-D tiled bulk tensor copy global -> shared (c0 innermost).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 // Allocates `ncols` tensor-memory columns (power of two >= 32) for this CTA
@@ -339,7 +348,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
-// Two fp32 -> packed bf16x2 (round to nearest even); `lo` in bits 0-15.
 // Two floats to two e4m3 codes (nearest even, saturating at 448): lo in the
 // low byte of the result.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
@@ -348,6 +356,7 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Two fp32 -> packed bf16x2 (round to nearest even); `lo` in bits 0-15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

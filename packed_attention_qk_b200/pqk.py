@@ -25,7 +25,7 @@ NORM_RMS, NORM_LAYER, NORM_NONE = 0, 1, 2
 EXPORTS = ("pqk_qk_norm_rope", "pqk_qk_norm_rope_3axis", "pqk_qk_fullc_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd",
            "pqk_varlen_attn_fwd_skip", "pqk_quantize_qk_e4m3", "pqk_varlen_attn_fwd_fp8qk", "pqk_quantize_e4m3",
            "pqk_varlen_attn_fwd_fp8",
-           "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu",
+           "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu", "pqk_linear_gated_residual", "pqk_linear_swiglu",
            "pqk_get_device_status", "pqk_set_wait_timeout_ns", "pqk_selftest_wait_timeout", "pqk_status_string",
            "pqk_version")
 
@@ -80,6 +80,10 @@ def lib(path: str | None = None) -> C.CDLL:
     L.pqk_modulate_swiglu.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, f32, vp, vp, i64, vp,
                                       i32, vp]
     L.pqk_modulate_swiglu.restype = i32
+    L.pqk_linear_gated_residual.argtypes = [vp, i64, vp, vp, i64, vp, vp, i32, vp, i64, i64, i32, i32, vp]
+    L.pqk_linear_gated_residual.restype = i32
+    L.pqk_linear_swiglu.argtypes = [vp, i64, vp, vp, i64, i64, i32, i32, vp]
+    L.pqk_linear_swiglu.restype = i32
     L.pqk_get_device_status.argtypes = [vp]
     L.pqk_get_device_status.restype = i32
     L.pqk_set_wait_timeout_ns.argtypes = [i64]
@@ -348,6 +352,39 @@ def modulate_swiglu(x, shift, scale, cu_seqlens, *, gate_res=None, branch=None, 
         _ptr(x), _ptr(branch), _ptr(x_out), _ptr(h), _ptr(shift), _ptr(scale), _ptr(gate_res), _ptr(cu_seqlens),
         B, T, Cdim, norm_type, eps, _ptr(gate), _ptr(up), gu_stride, _ptr(act), F, _stream(stream)))
     return x_out, h, act
+
+
+def linear_gated_residual(a, w, *, x=None, gate_res=None, cu_seqlens=None, out=None, stream=None):
+    """out = x + gate_res[request] * (a @ w.T) on the tensor cores (the
+    residual add in the GEMM's epilogue); with x None the product alone.
+    a: [T, K] bf16 (rows may be strided), w: [N, K] bf16, x: [T, N] bf16,
+    gate_res: [B, N] fp32. out may be x (in place)."""
+    import torch
+    T, K = a.shape
+    N = w.shape[0]
+    assert w.shape == (N, K) and w.is_contiguous()
+    if out is None:
+        out = torch.empty((T, N), dtype=a.dtype, device=a.device)
+    B = 0 if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    x_stride = 0 if x is None else _token_stride(x, 2)
+    _check("pqk_linear_gated_residual", lib().pqk_linear_gated_residual(
+        _ptr(a), _token_stride(a, 2), _ptr(w), _ptr(x), x_stride, _ptr(gate_res), _ptr(cu_seqlens), B, _ptr(out),
+        _token_stride(out, 2), T, K, N, _stream(stream)))
+    return out
+
+
+def linear_swiglu(a, w1, *, act=None, stream=None):
+    """act = silu(a @ w1[:F].T) * (a @ w1[F:].T) on the tensor cores (SwiGLU
+    in the GEMM's epilogue). a: [T, K] bf16, w1: [2F, K] bf16."""
+    import torch
+    T, K = a.shape
+    F = w1.shape[0] // 2
+    assert w1.shape == (2 * F, K) and w1.is_contiguous()
+    if act is None:
+        act = torch.empty((T, F), dtype=a.dtype, device=a.device)
+    _check("pqk_linear_swiglu", lib().pqk_linear_swiglu(
+        _ptr(a), _token_stride(a, 2), _ptr(w1), _ptr(act), _token_stride(act, 2), T, K, F, _stream(stream)))
+    return act
 
 
 def get_device_status(stream=None) -> int:

@@ -28,7 +28,11 @@ draw one tensor without drawing the others):
     0.02 ("weak") with probability 1/2 each from stream ``skip_blocks``;
   * local attention inputs (a stand-in for video attention, whose weight sits
     on nearby tokens): every token gets a unit feature vector of sinusoids of
-    its (t, h, w) ids, Q = K-ish = A * feature + N(0, 1) noise per head.
+    its (t, h, w) ids, Q = K-ish = A * feature + N(0, 1) noise per head;
+  * linear layers around the fused operators: inputs (attention output, h,
+    SwiGLU output) ~ N(0, 1); weights [out, in] ~ N(0, 1 / in) drawn as
+    float32 and scaled before the one bfloat16 rounding (random
+    initialisation; no trained weights exist here).
 bfloat16 tensors are returned as their uint16 bit patterns.
 """
 
@@ -47,6 +51,7 @@ TENSOR_ID = {
     "w_q": 8, "w_k": 9, "shift": 10, "scale": 11, "gate_res": 12,
     "outlier": 13, "sample_rows": 14, "w_q_full": 15, "w_k_full": 16,
     "skip_blocks": 17, "q_local": 18, "k_local": 19,
+    "attn_out": 20, "w_o": 21, "h_in": 22, "w1": 23, "act_in": 24, "w2": 25,
 }
 
 
@@ -355,6 +360,37 @@ def local_attention_inputs(w: Workload, amplitude: float = 12.0, noise: float = 
     with _cf.ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
         list(ex.map(head, range(w.H)))
     return {"q": q, "k": k, "v": bf16_normal(w.seed, "v", (w.T, w.H, w.D)), "cu_seqlens": w.cu_seqlens()}
+
+
+def bf16_linear_weight(seed: int, name: str, n_out: int, n_in: int) -> np.ndarray:
+    """[n_out, n_in] weight ~ N(0, 1 / n_in), rounded once to bfloat16."""
+    scale = np.float32(1.0 / np.sqrt(n_in))
+    out = np.empty(n_out * n_in, np.uint16)
+    for c in range((n_out * n_in + CHUNK - 1) // CHUNK):
+        lo, hi = c * CHUNK, min(n_out * n_in, (c + 1) * CHUNK)
+        out[lo:hi] = f32_to_bf16_bits(_chunk_values(seed, name, c, hi - lo, "normal") * scale)
+    return out.reshape(n_out, n_in)
+
+
+def linear_inputs(w: Workload, which: str) -> dict[str, np.ndarray]:
+    """Operands of one linear layer of the block, bf16 bits:
+    ``"o_proj"``: a = attention output [T, C], w = W_o [C, C], plus x, gate_res
+    for the gated residual; ``"w1"``: a = h [T, C], w = W1 [2F, C] (gate rows,
+    then up rows); ``"w2"``: a = SwiGLU output [T, F], w = W2 [C, F], plus x,
+    gate_res."""
+    T, Cd, F = w.T, w.C, w.F
+    if which == "o_proj":
+        d = {"a": bf16_normal(w.seed, "attn_out", (T, Cd)), "w": bf16_linear_weight(w.seed, "w_o", Cd, Cd)}
+    elif which == "w1":
+        return {"a": bf16_normal(w.seed, "h_in", (T, Cd)), "w": bf16_linear_weight(w.seed, "w1", 2 * F, Cd)}
+    elif which == "w2":
+        d = {"a": bf16_normal(w.seed, "act_in", (T, F)), "w": bf16_linear_weight(w.seed, "w2", Cd, F)}
+    else:
+        raise ValueError(which)
+    d["x"] = bf16_normal(w.seed, "x", (T, Cd))
+    d["gate_res"] = f32_modulation(w.seed, "gate_res", (w.B, Cd))
+    d["cu_seqlens"] = w.cu_seqlens()
+    return d
 
 
 def sample_rows(w: Workload, per_segment: int = 256) -> np.ndarray:

@@ -247,3 +247,43 @@ def test_quantize_e4m3_and_fp8_attention_host_errors(L):
     assert call(os_=512) == ERR_INVALID
     assert call(ws=None) == ERR_WORKSPACE
     assert call(T=0, q8=None) == 0
+
+
+def lin(L, **kw):
+    a = dict(a=A, a_stride=256, w=A, x=A, x_stride=512, gr=A, cu=A, B=2, out=A, out_stride=512, T=300, K=256, N=512)
+    a.update(kw)
+    return L.pqk_linear_gated_residual(a["a"], a["a_stride"], a["w"], a["x"], a["x_stride"], a["gr"], a["cu"], a["B"],
+                                       a["out"], a["out_stride"], a["T"], a["K"], a["N"], None)
+
+
+def test_linear_gated_residual_host_errors(L):
+    assert lin(L, K=12) == ERR_INVALID                       # K not a multiple of 8
+    assert lin(L, N=4) == ERR_INVALID
+    assert lin(L, T=-1) == ERR_INVALID
+    assert lin(L, T=2 ** 31) == ERR_INVALID                  # token coordinates are int32
+    assert lin(L, a_stride=128) == ERR_INVALID               # stride below K
+    assert lin(L, out_stride=256) == ERR_INVALID
+    assert lin(L, gr=None) == ERR_INVALID                    # x without its gate
+    assert lin(L, x=None) == ERR_INVALID                     # gate without x
+    assert lin(L, cu=None) == ERR_INVALID
+    assert lin(L, B=0) == ERR_INVALID
+    assert lin(L, x_stride=256) == ERR_INVALID
+    assert lin(L, T=0) == 0                                   # nothing to do, nothing enqueued
+    assert lin(L, a=None) == ERR_INVALID
+    assert lin(L, w=U) == ERR_MISALIGNED
+    assert lin(L, out=U) == ERR_MISALIGNED
+    assert lin(L, a_stride=260) == ERR_MISALIGNED             # rows not 16-byte aligned
+    assert lin(L, x=None, gr=None, cu=None, B=0, x_stride=0, a=U) == ERR_MISALIGNED   # the product alone
+
+
+def test_linear_swiglu_host_errors(L):
+    f = lambda **kw: L.pqk_linear_swiglu(kw.get("a", A), kw.get("a_stride", 256), kw.get("w1", A), kw.get("act", A),
+                                         kw.get("act_stride", 512), kw.get("T", 300), kw.get("K", 256),
+                                         kw.get("F", 512), None)
+    assert f(K=20) == ERR_INVALID
+    assert f(F=4) == ERR_INVALID
+    assert f(act_stride=500) == ERR_INVALID
+    assert f(T=0) == 0
+    assert f(w1=None) == ERR_INVALID
+    assert f(act=U) == ERR_MISALIGNED
+    assert f(act_stride=516) == ERR_MISALIGNED

@@ -45,6 +45,9 @@ int main(void) {
   if (pqk_varlen_attn_fwd_noalloc(a, a, a, a, NULL, 1024, 1024, 1024, 1024, a, 5000, 512, 8, 128, 0.1f, NULL) !=
       PQK_ERR_WORKSPACE)
     ++fails;
+  if (pqk_linear_gated_residual(a, 256, a, a, 512, NULL, a, 2, a, 512, 300, 256, 512, NULL) != PQK_ERR_INVALID_ARG)
+    ++fails;
+  if (pqk_linear_swiglu(a, 256, a, (void*)0x10004, 512, 300, 256, 512, NULL) != PQK_ERR_MISALIGNED) ++fails;
   printf("%d\n", fails);
   return fails != 0;
 }
