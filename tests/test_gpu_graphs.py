@@ -59,3 +59,42 @@ def test_captured_block_call_replays_bitwise(lens, H, D):
         assert torch.equal(o[k].view(torch.int16) if o[k].dtype == torch.bfloat16 else o[k],
                            v.view(torch.int16) if v.dtype == torch.bfloat16 else v), k
     del g
+
+
+def test_captured_linear_layers_replay_bitwise():
+    """The fused-epilogue GEMMs (tensor maps encoded on the host, passed by
+    value) captured once: the O-projection writing x', W1 with SwiGLU, and W2
+    adding its gated branch to x'; replays equal the direct calls bit for
+    bit."""
+    torch = torch_cuda()
+    w = wl.custom([300, 0, 700], 4, 64, C=256, F=384, seed=17)
+    lo, l1, l2 = (wl.linear_inputs(w, n) for n in ("o_proj", "w1", "w2"))
+    a, wo, w1, w2 = to_dev_bf16(lo["a"]), to_dev_bf16(lo["w"]), to_dev_bf16(l1["w"]), to_dev_bf16(l2["w"])
+    x, gr, cu = to_dev_bf16(lo["x"]), to_dev(lo["gate_res"]), to_dev(lo["cu_seqlens"])
+    h = to_dev_bf16(l1["a"])
+    xp, act, x2 = torch.empty_like(x), torch.empty((w.T, w.F), dtype=torch.bfloat16, device="cuda"), torch.empty_like(x)
+
+    def layers():
+        pqk.linear_gated_residual(a, wo, x=x, gate_res=gr, cu_seqlens=cu, out=xp)
+        pqk.linear_swiglu(h, w1, act=act)
+        pqk.linear_gated_residual(act, w2, x=xp, gate_res=gr, cu_seqlens=cu, out=x2)
+
+    layers()                                     # direct calls (the first on the device precede capture)
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (xp, act, x2)]
+    for t in (xp, act, x2):
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            layers()
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert pqk.get_device_status() == 0
+    for got, want in zip((xp, act, x2), ref):
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    del g
