@@ -25,7 +25,8 @@ layers with the gated residual or SwiGLU in the GEMM epilogue, on the step's
 own activations, against cuBLAS plus torch epilogues (``linear_epilogue``;
 ``--no-linear`` leaves it out); and, with ``--graph``,
 the step replayed as a CUDA graph (``graph_ms_per_step``). ``--config N``
-selects another configuration, ``--sweep`` the HBM bandwidth sweep.
+selects another configuration, ``--sweep`` the HBM bandwidth sweep,
+``--linear-sweep`` the fused-epilogue linear layers on a range of shapes.
 """
 
 from __future__ import annotations
@@ -71,6 +72,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="leave out the FP8 Q K^T attention timing")
+    ap.add_argument("--linear-sweep", action="store_true",
+                    help="the fused-epilogue linear layers alone against cuBLAS on a range of token counts and "
+                         "widths (one JSON line per shape) instead of the step")
     ap.add_argument("--no-linear", action="store_true",
                     help="leave out the linear layers with the fused epilogues (gated residual, SwiGLU)")
     ap.add_argument("--graph", action="store_true",
@@ -710,6 +714,36 @@ def run_ours(args, w):
         dist.destroy_process_group()
 
 
+def run_linear_sweep(args):
+    """The block's three linear layers with fused epilogues, alone, against
+    cuBLAS plus torch epilogues, on the 4,096- and 58,048-token widths and on
+    the 40-head sweep widths (hidden 5,120, FFN 13,824) at its four token
+    counts. Activations are drawn on the device (torch's CUDA generator,
+    N(0, 1), seeded per shape) to keep the multi-GB inputs off the host;
+    weights as in the step."""
+    import torch
+    from packed_attention_qk_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    pk, pk_kind = peaks()
+    shapes = [(4096, 16, 2048, 5632), (58048, 24, 3072, 8192)] + [(T, 40, 5120, 13824) for T in wl.C5_TOKENS]
+    for T, H, Cd, F in shapes:
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(T * 7 + Cd * 3 + F)
+
+        def randn(*shape, scale=1.0, dtype=torch.bfloat16):
+            return (torch.randn(*shape, generator=gen, device=dev) * scale).to(dtype)
+
+        w = wl.Workload(f"linear layers, {T} tokens, hidden {Cd}, ffn {F}", 5, [T], H=H, D=Cd // H, C=Cd, F=F,
+                        pos_runs=[[T]])
+        d = {"x": randn(T, Cd), "gate_res": randn(1, Cd, scale=0.1, dtype=torch.float32),
+             "cu": torch.tensor([0, T], dtype=torch.int32, device=dev)}
+        o = {"o": randn(T, H, Cd // H), "h": randn(T, Cd), "act": randn(T, F)}
+        res = time_linear_layers(w, d, o, pk, pk_kind)
+        print(json.dumps({"sweep": "linear_epilogue", "tokens": T, "hidden": Cd, "ffn": F, **res}), flush=True)
+        del d, o
+        torch.cuda.empty_cache()
+
+
 def run_sweep(args):
     """The HBM-bound kernels alone on the sweep shapes, one launch at a time
     with a 256 MB L2 flush in between (the 4,096-token working set is close
@@ -769,6 +803,9 @@ def main():
     from packed_attention_qk_b200 import workloads as wl
     if args.sweep:
         run_sweep(args)
+        return
+    if args.linear_sweep:
+        run_linear_sweep(args)
         return
     w = wl.config(args.config)
     if args.tokens:
