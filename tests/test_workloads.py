@@ -101,3 +101,13 @@ def test_linear_inputs_shapes_and_gate_rows_first():
     assert w2["a"].shape == (128, 192) and w2["w"].shape == (128, 192) and np.array_equal(w2["x"], o["x"])
     with pytest.raises(ValueError):
         wl.linear_inputs(w, "qkv")
+
+
+def test_batch_positions_reuse_the_joint_layout_for_its_58k_request():
+    c4 = wl.config(4)
+    pos = c4.positions()
+    cu = c4.cu_seqlens()
+    assert pos[cu[1] - 1] == 12344 and pos[cu[1]] == 0                 # 0..L-1 for plain requests
+    third = pos[cu[2]:cu[3]]
+    assert np.array_equal(third, wl.config(3).positions())              # text / audio / video runs of the 58k one
+    assert pos[-1] == 87071
