@@ -43,3 +43,39 @@ def test_oracle_matches_stored_tiny_config_outputs():
     for name, t in (("x_out", xo), ("h", h), ("act", act)):
         _summary_close(t, g[name]["summary"])
         np.testing.assert_allclose([t[r, :8] for r in rows], g[name]["first"], atol=1e-12)
+
+
+def test_oracle_variants_match_stored_tiny_config_outputs():
+    g = json.load(open(GOLDEN))
+    rows = g["rows"]
+    w = wl.config(1)
+    p, a = wl.prologue_inputs(w), wl.attention_inputs(w)
+    scale = 1.0 / math.sqrt(w.D)
+    y = oracle.qk_norm_rope_3axis(p["q"], p["w_q"], w.positions3(video_grid=(2, 10, 10)), (8, 12, 12), w.eps,
+                                  w.rope_base)
+    _summary_close(y, g["q_norm_rope_3axis"]["summary"])
+    np.testing.assert_allclose([y[r, 0, :8] for r in rows], g["q_norm_rope_3axis"]["head0"], atol=1e-12)
+    y = oracle.qk_fullc_norm_rope(p["q"], wl.fullc_weights(w)["w_q"], p["pos"], w.eps, w.rope_base)
+    _summary_close(y, g["q_fullc_norm_rope"]["summary"])
+    np.testing.assert_allclose([y[r, 0, :8] for r in rows], g["q_fullc_norm_rope"]["head0"], atol=1e-12)
+    b = wl.block_scaled_attention_inputs(w)
+    o, lse, counts = oracle.varlen_attn_skip(b["q"], b["k"], b["v"], b["cu_seqlens"], scale, 4.0)
+    assert list(counts) == g["attn_skip_tau4"]["counts"]
+    _summary_close(o, g["attn_skip_tau4"]["summary"])
+    _summary_close(lse, g["attn_skip_tau4"]["lse_summary"])
+    np.testing.assert_allclose([o[r, 0, :8] for r in rows], g["attn_skip_tau4"]["head0"], atol=1e-12)
+    for key, fn in (("attn_fp8qk", oracle.varlen_attn_fp8qk), ("attn_fp8", oracle.varlen_attn_fp8)):
+        res = fn(a["q"], a["k"], a["v"], a["cu_seqlens"], scale)
+        o, lse, deq = res[0], res[1], res[-1]
+        assert np.array_equal(np.asarray(deq, np.float32), np.asarray(g[key]["deq"], np.float32))
+        _summary_close(o, g[key]["summary"])
+        _summary_close(lse, g[key]["lse_summary"])
+        np.testing.assert_allclose([o[r, 0, :8] for r in rows], g[key]["head0"], atol=1e-12)
+    for name in ("o_proj", "w1", "w2"):
+        d = wl.linear_inputs(w, name)
+        if name == "w1":
+            y = oracle.linear_swiglu(d["a"], d["w"])
+        else:
+            y = oracle.linear_gated_residual(d["a"], d["w"], d["x"], d["gate_res"], d["cu_seqlens"])
+        _summary_close(y, g[f"linear_{name}"]["summary"])
+        np.testing.assert_allclose([y[r, :8] for r in rows], g[f"linear_{name}"]["first"], atol=1e-12)
