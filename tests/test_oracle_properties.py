@@ -7,7 +7,9 @@ does not come from the oracle itself.
   * RMSNorm + RoPE preserves every pair's norm of the normalised, weighted
     row and depends on positions only through their differences in dot
     products;
-  * e4m3 codes = torch's float8_e4m3fn conversion.
+  * e4m3 codes = torch's float8_e4m3fn conversion;
+  * the linear layers with their fused epilogues = numpy's matmul followed
+    by the residual or SwiGLU, over random request mixes and token strides.
 """
 
 import math
@@ -83,3 +85,30 @@ def test_e4m3_codes_equal_torch(values):
     x = np.array(values, np.float32)
     ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.array_equal(oracle.e4m3_codes(x), ref)
+
+
+@settings(max_examples=25, deadline=None)
+@given(lens=lens_st, K=st.integers(1, 40), N=st.integers(1, 24), pad=st.integers(0, 7),
+       seed=st.integers(0, 2 ** 31 - 1))
+def test_linear_gated_residual_equals_numpy(lens, K, N, pad, seed):
+    # random request mixes (empty ones included) and a token stride of K + pad
+    g = np.random.default_rng(seed)
+    T = sum(lens)
+    wide = g.standard_normal((T, K + pad))
+    a = wide[:, :K]
+    w, x = g.standard_normal((N, K)), g.standard_normal((T, N))
+    gr = g.standard_normal((len(lens), N)).astype(np.float32)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    seg = np.repeat(np.arange(len(lens)), lens)
+    ref = x + gr.astype(np.float64)[seg] * (a @ w.T)
+    assert np.max(np.abs(oracle.linear_gated_residual(a, w, x, gr, cu) - ref)) <= 1e-10
+
+
+@settings(max_examples=25, deadline=None)
+@given(T=st.integers(1, 30), K=st.integers(1, 40), F=st.integers(1, 24), seed=st.integers(0, 2 ** 31 - 1))
+def test_linear_swiglu_equals_numpy(T, K, F, seed):
+    g = np.random.default_rng(seed)
+    a, w1 = g.standard_normal((T, K)), g.standard_normal((2 * F, K))
+    gate, up = a @ w1[:F].T, a @ w1[F:].T
+    ref = gate / (1.0 + np.exp(-gate)) * up
+    assert np.max(np.abs(oracle.linear_swiglu(a, w1) - ref) / np.maximum(1.0, np.abs(ref))) <= 1e-12
