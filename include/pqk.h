@@ -366,8 +366,10 @@ PQK_API int pqk_modulate_swiglu(const void* x, const void* branch, void* x_out, 
  * cu_seqlens  device int32 [B+1] (must be valid; not re-checked here).
  * out         device bf16 [T, N], rows out_stride_t apart; may equal x
  *             (same stride); no other overlap with an input.
- * K, N        multiples of 8, >= 8; T <= 2^31 - 257. Pointers 16-byte
- *             aligned, strides multiples of 8 elements.
+ * K, N        multiples of 8, >= 8; T <= 2^31 - 257, and the number of
+ *             128 x 128 output tiles, ceil(T/128) * ceil(N/128), below
+ *             2^31 - 2^20. Pointers 16-byte aligned, strides multiples of 8
+ *             elements.
  * Errors: PQK_ERR_INVALID_ARG / PQK_ERR_MISALIGNED before anything is
  * enqueued; a pipeline wait that runs out records PQK_ERR_TIMEOUT in the
  * device status word (see pqk_get_device_status).
@@ -390,8 +392,8 @@ PQK_API int pqk_linear_gated_residual(const void* a, int64_t a_stride_t, const v
  * a           device bf16 [T, K], rows a_stride_t elements apart.
  * w1          device bf16 [2F, K] contiguous.
  * act         device bf16 [T, F], rows act_stride_t apart.
- * K, F        multiples of 8, >= 8. Alignment and errors as
- *             pqk_linear_gated_residual.
+ * K, F        multiples of 8, >= 8. Size limits (with F for N), alignment
+ *             and errors as pqk_linear_gated_residual.
  */
 PQK_API int pqk_linear_swiglu(const void* a, int64_t a_stride_t, const void* w1, void* act, int64_t act_stride_t,
                               int64_t T, int K, int F, void* stream);

@@ -61,6 +61,14 @@ int check_device(DeviceInfo** out) {
   return PQK_OK;
 }
 
+// The linear-layer kernel indexes its output tiles (128 tokens x 128
+// columns at the finest) with 32-bit integers: keep their count, plus a grid
+// stride of headroom, inside that range.
+bool linear_tiles_fit(int64_t T, int N) {
+  const int64_t tiles = ((T + 127) / 128) * ((static_cast<int64_t>(N) + 127) / 128);
+  return tiles <= static_cast<int64_t>(INT32_MAX) - (1 << 20);
+}
+
 }  // namespace
 
 extern "C" {
@@ -319,6 +327,7 @@ int pqk_linear_gated_residual(const void* a, int64_t a_stride_t, const void* w, 
                               const float* gate_res, const int32_t* cu_seqlens, int B, void* out,
                               int64_t out_stride_t, int64_t T, int K, int N, void* stream) {
   if (T < 0 || T > INT32_MAX - 256 || K < 8 || N < 8 || K % 8 || N % 8) return PQK_ERR_INVALID_ARG;
+  if (!linear_tiles_fit(T, N)) return PQK_ERR_INVALID_ARG;
   const bool residual = x != nullptr || gate_res != nullptr;
   if (residual && (x == nullptr || gate_res == nullptr || cu_seqlens == nullptr || B < 1 || x_stride_t < N))
     return PQK_ERR_INVALID_ARG;
@@ -339,6 +348,7 @@ int pqk_linear_gated_residual(const void* a, int64_t a_stride_t, const void* w, 
 int pqk_linear_swiglu(const void* a, int64_t a_stride_t, const void* w1, void* act, int64_t act_stride_t, int64_t T,
                       int K, int F, void* stream) {
   if (T < 0 || T > INT32_MAX - 256 || K < 8 || F < 8 || K % 8 || F % 8) return PQK_ERR_INVALID_ARG;
+  if (!linear_tiles_fit(T, F)) return PQK_ERR_INVALID_ARG;
   if (a_stride_t < K || act_stride_t < F) return PQK_ERR_INVALID_ARG;
   if (T == 0) return PQK_OK;
   if (!a || !w1 || !act) return PQK_ERR_INVALID_ARG;

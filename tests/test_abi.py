@@ -274,6 +274,8 @@ def test_linear_gated_residual_host_errors(L):
     assert lin(L, out=U) == ERR_MISALIGNED
     assert lin(L, a_stride=260) == ERR_MISALIGNED             # rows not 16-byte aligned
     assert lin(L, x=None, gr=None, cu=None, B=0, x_stride=0, a=U) == ERR_MISALIGNED   # the product alone
+    # more output tiles than 32-bit tile indices can count
+    assert lin(L, T=2 ** 31 - 300, N=2 ** 30, x_stride=2 ** 30, out_stride=2 ** 30) == ERR_INVALID
 
 
 def test_linear_swiglu_host_errors(L):
@@ -287,3 +289,4 @@ def test_linear_swiglu_host_errors(L):
     assert f(w1=None) == ERR_INVALID
     assert f(act=U) == ERR_MISALIGNED
     assert f(act_stride=516) == ERR_MISALIGNED
+    assert f(T=2 ** 31 - 300, F=2 ** 30, act_stride=2 ** 30) == ERR_INVALID
