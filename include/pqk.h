@@ -169,7 +169,9 @@ PQK_API size_t pqk_varlen_attn_workspace_size(int B);
  *               empty requests are allowed. Checked on the device: a
  *               violation sets PQK_ERR_BAD_SEQLENS in the status word and
  *               the call writes no output.
- * D             64 or 128. B >= 1, T >= 0.
+ * D             64 or 128. B >= 1, 0 <= T <= 2^31 - 513, and the work
+ *               tiles of the schedule, (ceil(T/256) + B) * H, below
+ *               2^31 - 2^20 (the other attention entry points alike).
  * workspace     device memory of at least pqk_varlen_attn_workspace_size(B)
  *               bytes, 16-byte aligned; it only holds this call's schedule
  *               and may be reused once the call has completed on `stream`.

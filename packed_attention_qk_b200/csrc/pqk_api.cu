@@ -69,6 +69,13 @@ bool linear_tiles_fit(int64_t T, int N) {
   return tiles <= static_cast<int64_t>(INT32_MAX) - (1 << 20);
 }
 
+// The attention's tile schedule counts its work tiles (256 query rows x one
+// head) in 32-bit integers; their number is at most (ceil(T/256) + B) * H.
+bool attn_tiles_fit(int64_t T, int B, int H) {
+  const int64_t tiles = ((T + 255) / 256 + B) * static_cast<int64_t>(H);
+  return tiles <= static_cast<int64_t>(INT32_MAX) - (1 << 20);
+}
+
 }  // namespace
 
 extern "C" {
@@ -168,6 +175,7 @@ int pqk_varlen_attn_fwd(const void* q, const void* k, const void* v, void* o, fl
                         size_t workspace_bytes, void* stream) {
   if (B < 1 || T < 0 || H <= 0 || T > INT32_MAX - 512 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     return PQK_ERR_INVALID_ARG;
+  if (!attn_tiles_fit(T, B, H)) return PQK_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return PQK_ERR_UNSUPPORTED;
   const int64_t row = static_cast<int64_t>(H) * D;
   if (q_stride_t < row || k_stride_t < row || v_stride_t < row || o_stride_t < row) return PQK_ERR_INVALID_ARG;
@@ -192,6 +200,7 @@ int pqk_varlen_attn_fwd_skip(const void* q, const void* k, const void* v, void* 
                              unsigned long long* skip_counts, void* workspace, size_t workspace_bytes, void* stream) {
   if (B < 1 || T < 0 || H <= 0 || T > INT32_MAX - 512 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     return PQK_ERR_INVALID_ARG;
+  if (!attn_tiles_fit(T, B, H)) return PQK_ERR_INVALID_ARG;
   if (!(skip_threshold_log2 >= 0.f)) return PQK_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return PQK_ERR_UNSUPPORTED;
   const int64_t row = static_cast<int64_t>(H) * D;
@@ -238,6 +247,7 @@ int pqk_varlen_attn_fwd_fp8qk(const void* q8, const void* k8, const void* v, con
                               void* stream) {
   if (B < 1 || T < 0 || H <= 0 || T > INT32_MAX - 512 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     return PQK_ERR_INVALID_ARG;
+  if (!attn_tiles_fit(T, B, H)) return PQK_ERR_INVALID_ARG;
   if (!(skip_threshold_log2 >= 0.f)) return PQK_ERR_INVALID_ARG;
   if (D != 128) return PQK_ERR_UNSUPPORTED;
   const int64_t row = static_cast<int64_t>(H) * D;
@@ -278,6 +288,7 @@ int pqk_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, cons
                             float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
   if (B < 1 || T < 0 || H <= 0 || T > INT32_MAX - 512 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     return PQK_ERR_INVALID_ARG;
+  if (!attn_tiles_fit(T, B, H)) return PQK_ERR_INVALID_ARG;
   if (D != 128) return PQK_ERR_UNSUPPORTED;
   const int64_t row = static_cast<int64_t>(H) * D;
   if (o_stride_t < row) return PQK_ERR_INVALID_ARG;

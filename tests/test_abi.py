@@ -144,6 +144,20 @@ def mod(L, **kw):
                                  None)
 
 
+def test_attention_rejects_more_work_tiles_than_32_bits_count(L):
+    # (ceil(T/256) + B) * H above 2^31 - 2^20: refused on the host for every attention entry
+    T, H = 2 ** 31 - 600, 4096
+    assert L.pqk_varlen_attn_fwd(A, A, A, A, None, H * 128, H * 128, H * 128, H * 128, A, 1, T, H, 128, 0.1, A,
+                                 4096, None) == ERR_INVALID
+    assert L.pqk_varlen_attn_fwd_skip(A, A, A, A, None, H * 128, H * 128, H * 128, H * 128, A, 1, T, H, 128, 0.1,
+                                      8.0, None, A, 4096, None) == ERR_INVALID
+    assert L.pqk_varlen_attn_fwd_fp8qk(A, A, A, A, A, None, H * 128, H * 128, A, 1, T, H, 128, 0.1,
+                                       float("inf"), None, A, 4096, None) == ERR_INVALID
+    assert L.pqk_varlen_attn_fwd_fp8(A, A, A, A, A, None, H * 128, A, 1, T, H, 128, 0.1, A, 4096, None) == ERR_INVALID
+    # (the no-allocation entry looks up its device array first and then forwards to pqk_varlen_attn_fwd, so the
+    # same check applies to it on a GPU; without one it stops at the lookup)
+
+
 def test_modulate_swiglu_host_errors(L):
     assert mod(L, C=250) == ERR_INVALID
     assert mod(L, C=16392) == ERR_INVALID
