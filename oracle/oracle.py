@@ -54,15 +54,18 @@ def load(path: str):
     L.oracle_qk_fullc_norm_rope.argtypes = [vp, C.c_int, C.c_int64, vp, C.c_int, i32p, C.c_int64, C.c_int, C.c_int,
                                             C.c_double, C.c_double, C.c_int, i32p, C.c_int64, f64p]
     L.oracle_varlen_attn_skip.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
-                                          C.c_int, C.c_double, C.c_double, i32p, C.c_int64, f64p, f64p,
-                                          C.POINTER(C.c_int64)]
+                                          C.c_int, C.c_double, C.c_double, C.c_int, C.c_int, C.c_int, i32p,
+                                          C.c_int64, f64p, f64p, C.POINTER(C.c_int64)]
     u8p = C.POINTER(C.c_uint8)
     L.oracle_quantize_e4m3.argtypes = [vp, C.c_int, C.c_int64, C.c_int64, C.c_int, C.c_int, u8p, f32p]
     L.oracle_varlen_attn_fp8qk.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
-                                           C.c_int, C.c_double, C.c_double, i32p, C.c_int64, f64p, f64p,
-                                           C.POINTER(C.c_int64), u8p, u8p, f32p]
+                                           C.c_int, C.c_double, C.c_double, C.c_int, C.c_int, C.c_int, i32p,
+                                           C.c_int64, f64p, f64p, C.POINTER(C.c_int64), u8p, u8p, f32p]
     L.oracle_varlen_attn_fp8.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
                                          C.c_int, C.c_double, i32p, C.c_int64, f64p, f64p, f32p]
+    L.oracle_varlen_attn_fp8_online.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
+                                                C.c_int, C.c_double, C.c_int, C.c_double, i32p, C.c_int64, f64p,
+                                                f64p, f32p]
     L.oracle_linear_gated_residual.argtypes = [vp, C.c_int64, vp, vp, C.c_int, f32p, i32p, C.c_int, C.c_int64,
                                                C.c_int, C.c_int, i32p, C.c_int64, f64p]
     L.oracle_linear_swiglu.argtypes = [vp, C.c_int64, vp, C.c_int, C.c_int64, C.c_int, C.c_int, i32p, C.c_int64,
@@ -71,7 +74,7 @@ def load(path: str):
     L.oracle_e4m3_codes.restype = None
     for f in (L.oracle_qk_norm_rope, L.oracle_qk_norm_rope_3axis, L.oracle_qk_fullc_norm_rope, L.oracle_varlen_attn,
               L.oracle_varlen_attn_skip, L.oracle_quantize_e4m3, L.oracle_varlen_attn_fp8qk, L.oracle_varlen_attn_fp8,
-              L.oracle_modulate_swiglu, L.oracle_linear_gated_residual, L.oracle_linear_swiglu):
+              L.oracle_varlen_attn_fp8_online, L.oracle_modulate_swiglu, L.oracle_linear_gated_residual, L.oracle_linear_swiglu):
         f.restype = C.c_int
     L.oracle_num_threads.restype = C.c_int
     return L
@@ -190,24 +193,27 @@ def varlen_attn(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndar
 
 
 def varlen_attn_skip(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, tau: float,
-                     rows=None, want_lse: bool = True):
+                     *, block, tile_rows: int, rows=None, want_lse: bool = True):
     """Attention with key blocks skipped where negligible (oracle_varlen_attn_skip).
-    Returns (o [nrows, H, D], lse [nrows, H] or None, counts): counts is
-    (skipped 32-row blocks, skipped 128-row tiles) over all (block, head, key
-    block) triples when rows is None, else None."""
+    block = (query rows, keys) of a decision block; tile_rows (a multiple of
+    the block's rows) groups query blocks for the second count. Returns
+    (o [nrows, H, D], lse [nrows, H] or None, counts): counts is (skipped
+    query blocks, skipped tiles) over all (block, head, key block) triples
+    when rows is None, else None."""
     T, H, D = q.shape
     assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
     q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    qrows, kblock = (int(b) for b in block)
     r, n = _rows(rows)
     n = n if r is not None else T
     o = np.empty((n, H, D), np.float64)
     lse = np.empty((n, H), np.float64) if want_lse else None
     counts = np.zeros(2, np.int64)
     rc = lib().oracle_varlen_attn_skip(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32),
-                                       int(cu.shape[0]) - 1, T, H, D, scale, float(tau), _ptr(r, C.c_int32),
-                                       n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
-                                       _ptr(counts, C.c_int64))
+                                       int(cu.shape[0]) - 1, T, H, D, scale, float(tau), qrows, kblock,
+                                       int(tile_rows), _ptr(r, C.c_int32), n if r is not None else 0,
+                                       _ptr(o, C.c_double), _ptr(lse, C.c_double), _ptr(counts, C.c_int64))
     if rc:
         raise ValueError("oracle_varlen_attn_skip: invalid arguments")
     return o, lse, (tuple(int(c) for c in counts) if r is None else None)
@@ -234,15 +240,23 @@ def quantize_e4m3(x: np.ndarray):
 
 
 def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, rows=None,
-                      want_lse: bool = True, tau: float = math.inf, counts_out: list | None = None):
+                      want_lse: bool = True, tau: float = math.inf, skip_block=None, skip_tile_rows=None,
+                      counts_out: list | None = None):
     """Attention with Q and K quantised to e4m3 per head (block skipping on
-    the quantised scores for a finite tau; its counts appended to counts_out
-    when given). Returns (o [nrows, H, D], lse [nrows, H] or None, q8, k8
-    [T, H, D] uint8, deq [2H])."""
+    the quantised scores for a finite tau, with the geometry skip_block =
+    (query rows, keys) and skip_tile_rows as in varlen_attn_skip; its counts
+    appended to counts_out when given). Returns (o [nrows, H, D], lse
+    [nrows, H] or None, q8, k8 [T, H, D] uint8, deq [2H])."""
     T, H, D = q.shape
     assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
     q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    if math.isinf(tau) and tau > 0:
+        qrows, kblock, tile_rows = 1, 1, 1
+    else:
+        if skip_block is None or skip_tile_rows is None:
+            raise ValueError("a finite tau needs the block geometry (skip_block, skip_tile_rows)")
+        (qrows, kblock), tile_rows = (int(b) for b in skip_block), int(skip_tile_rows)
     r, n = _rows(rows)
     n = n if r is not None else T
     o = np.empty((n, H, D), np.float64)
@@ -252,10 +266,10 @@ def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: n
     deq = np.empty(2 * H, np.float32)
     counts = np.zeros(2, np.int64)
     rc = lib().oracle_varlen_attn_fp8qk(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32),
-                                        int(cu.shape[0]) - 1, T, H, D, scale, float(tau), _ptr(r, C.c_int32),
-                                        n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
-                                        _ptr(counts, C.c_int64), _ptr(q8, C.c_uint8), _ptr(k8, C.c_uint8),
-                                        _ptr(deq, C.c_float))
+                                        int(cu.shape[0]) - 1, T, H, D, scale, float(tau), qrows, kblock, tile_rows,
+                                        _ptr(r, C.c_int32), n if r is not None else 0, _ptr(o, C.c_double),
+                                        _ptr(lse, C.c_double), _ptr(counts, C.c_int64), _ptr(q8, C.c_uint8),
+                                        _ptr(k8, C.c_uint8), _ptr(deq, C.c_float))
     if rc:
         raise ValueError("oracle_varlen_attn_fp8qk: invalid arguments")
     if counts_out is not None and r is None:
@@ -263,10 +277,7 @@ def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: n
     return o, lse, q8, k8, deq
 
 
-def varlen_attn_fp8(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, rows=None,
-                    want_lse: bool = True):
-    """Attention with Q, K, V and P in FP8 e4m3 (oracle_varlen_attn_fp8).
-    Returns (o [nrows, H, D], lse [nrows, H] or None, deq [3H])."""
+def _fp8_call(fn, name, q, k, v, cu_seqlens, scale, rows, want_lse, extra):
     T, H, D = q.shape
     assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
     q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
@@ -276,13 +287,31 @@ def varlen_attn_fp8(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.
     o = np.empty((n, H, D), np.float64)
     lse = np.empty((n, H), np.float64) if want_lse else None
     deq = np.empty(3 * H, np.float32)
-    rc = lib().oracle_varlen_attn_fp8(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32),
-                                      int(cu.shape[0]) - 1, T, H, D, scale, _ptr(r, C.c_int32),
-                                      n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
-                                      _ptr(deq, C.c_float))
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32), int(cu.shape[0]) - 1, T, H, D, scale,
+            *extra, _ptr(r, C.c_int32), n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
+            _ptr(deq, C.c_float))
     if rc:
-        raise ValueError("oracle_varlen_attn_fp8: invalid arguments")
+        raise ValueError(f"{name}: invalid arguments")
     return o, lse, deq
+
+
+def varlen_attn_fp8(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, rows=None,
+                    want_lse: bool = True):
+    """Attention with Q, K, V and P in FP8 e4m3, P rounded against each row's
+    exact maximum (oracle_varlen_attn_fp8). Returns (o [nrows, H, D], lse
+    [nrows, H] or None, deq [3H])."""
+    return _fp8_call(lib().oracle_varlen_attn_fp8, "oracle_varlen_attn_fp8", q, k, v, cu_seqlens, scale, rows,
+                     want_lse, ())
+
+
+def varlen_attn_fp8_online(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, *,
+                           kblock: int, threshold: float, rows=None, want_lse: bool = True):
+    """The same FP8 attention in the rounding order of an online softmax over
+    blocks of kblock keys whose running maximum moves only past threshold
+    (log2 units): a streaming implementation's schedule, not the definition
+    (oracle_varlen_attn_fp8_online). Returns (o, lse or None, deq [3H])."""
+    return _fp8_call(lib().oracle_varlen_attn_fp8_online, "oracle_varlen_attn_fp8_online", q, k, v, cu_seqlens, scale,
+                     rows, want_lse, (int(kblock), float(threshold)))
 
 
 def modulate_swiglu(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, gate_res: np.ndarray,

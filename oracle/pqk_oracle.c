@@ -25,10 +25,16 @@
  *   oracle_varlen_attn_fp8qk -- the same attention with Q and K quantised to
  *                             FP8 e4m3 per head (SAGE FP8, a reading).
  *   oracle_varlen_attn_fp8  -- the attention with Q, K, V and P in FP8 e4m3
- *                             (the whole SAGE reading).
+ *                             (the whole SAGE reading), P rounded against
+ *                             each row's exact maximum.
+ *   oracle_varlen_attn_fp8_online -- the same quantities in the rounding
+ *                             order of an online softmax with a lazily moved
+ *                             maximum (a streaming implementation's schedule,
+ *                             block size and threshold given by the caller).
  *   oracle_varlen_attn_skip -- the same attention with key blocks skipped
  *                             where their scores are negligible ("Skip-Softmax";
- *                             a reading, see the function).
+ *                             a reading, see the function; the block geometry
+ *                             is the caller's).
  *   oracle_modulate_swiglu -- modulation + normalisation + gated residual and
  *                             SwiGLU in place of separate SiLU and multiply
  *                             (first page "融合 DiT 算子"; second page bullet
@@ -355,20 +361,22 @@ int oracle_quantize_e4m3(const void* x, int x_kind, int64_t stride_t, int64_t T,
 
 int oracle_varlen_attn_skip(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
                             const int32_t* cu, int B, int64_t T, int H, int D, double scale, double tau,
-                            const int32_t* rows, int64_t nrows, double* o, double* lse, int64_t* counts);
+                            int qrows, int kblock, int tile_rows, const int32_t* rows, int64_t nrows, double* o,
+                            double* lse, int64_t* counts);
 
 /*
  * Attention with Q and K quantised to e4m3 per head (oracle_quantize_e4m3)
  * and V, P kept at their precision: the plain attention of
  * oracle_varlen_attn on Q~ = code(Q) * deq_Q and K~ = code(K) * deq_K, or,
  * for a finite tau, the block-skipping attention of oracle_varlen_attn_skip
- * on them (counts as there). q8_out, k8_out ([T, H, D]) and deq_out ([2H]:
- * Q's, then K's) are optional.
+ * on them with the block geometry (qrows, kblock, tile_rows) given (counts as
+ * there; the geometry is unused for an infinite tau). q8_out, k8_out
+ * ([T, H, D]) and deq_out ([2H]: Q's, then K's) are optional.
  */
 int oracle_varlen_attn_fp8qk(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
                              const int32_t* cu, int B, int64_t T, int H, int D, double scale, double tau,
-                             const int32_t* rows, int64_t nrows, double* o, double* lse, int64_t* counts,
-                             uint8_t* q8_out, uint8_t* k8_out, float* deq_out) {
+                             int qrows, int kblock, int tile_rows, const int32_t* rows, int64_t nrows, double* o,
+                             double* lse, int64_t* counts, uint8_t* q8_out, uint8_t* k8_out, float* deq_out) {
   if (check_cu(cu, B, T) || H <= 0 || D <= 0) return -1;
   const int64_t n = T * (int64_t)H * D;
   uint8_t* qc = q8_out ? q8_out : (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
@@ -392,8 +400,8 @@ int oracle_varlen_attn_fp8qk(const void* q, const void* k, const void* v, int in
     if (isinf(tau) && tau > 0)
       rc = oracle_varlen_attn(qd, kd, vd, ORACLE_IN_F64, (int64_t)H * D, cu, B, T, H, D, scale, rows, nrows, o, lse);
     else
-      rc = oracle_varlen_attn_skip(qd, kd, vd, ORACLE_IN_F64, (int64_t)H * D, cu, B, T, H, D, scale, tau, rows,
-                                   nrows, o, lse, counts);
+      rc = oracle_varlen_attn_skip(qd, kd, vd, ORACLE_IN_F64, (int64_t)H * D, cu, B, T, H, D, scale, tau, qrows,
+                                   kblock, tile_rows, rows, nrows, o, lse, counts);
   }
   if (deq_out) memcpy(deq_out, dq, sizeof(float) * (size_t)H * 2);
   if (!q8_out) free(qc);
@@ -407,27 +415,69 @@ int oracle_varlen_attn_fp8qk(const void* q, const void* k, const void* v, int in
 
 /*
  * Attention with Q, K and V quantised to e4m3 per head and the
- * probabilities P quantised to e4m3 inside the online softmax: the whole
- * attention computation in FP8 (SAGE, first page, bullet on TRTLLM_ATTN SAGE
- * and Skip-Softmax; a reading). Per row, over the key blocks of 128 keys
- * counted from the request's first token, in order, with u = s / ln 2 the
- * score of the dequantised Q, K in log2 units:
- *   - the running maximum m is set by the first block and afterwards moves
- *     only when a block's maximum exceeds it by more than 8; the sums are
- *     then scaled by 2^(m_old - m_new);
- *   - each key adds p = 2^(u - m) to the denominator l and e4m3(p) * v~ to
- *     the numerator (v~ = code(V) * deq_V; p <= 2^8 stays in e4m3's range);
- *   - O = numerator / l and lse = (m + log2 l) ln 2.
- * deq_out: [3H] (Q's, K's, V's dequantisation factors), optional.
+ * probabilities P quantised to e4m3: the whole attention computation in FP8
+ * (SAGE, first page, bullet on TRTLLM_ATTN SAGE and Skip-Softmax; a
+ * reading). With Q~, K~, V~ the dequantised tensors (code * deq per head),
+ * for query row t of request i and head h:
+ *   s_j  = scale * <q~_t, k~_j>,  j in request i
+ *   m    = max_j s_j,  p_j = exp(s_j - m)          (so 0 < p_j <= 1)
+ *   o_t  = sum_j e4m3(p_j) v~_j / sum_j p_j         (P rounded in the numerator only)
+ *   lse_t = m + ln sum_j p_j.
+ * e4m3(p) is the code nearest to p taken as a float (oracle_e4m3_codes),
+ * read back as its value. deq_out: [3H] (Q's, K's, V's dequantisation
+ * factors), optional.
  */
 static void fp8_row(const double* qd, const double* kd, const double* vd, int64_t lo, int64_t n_keys, int64_t t,
                     int H, int h, int D, double scale, double* ot, double* lse_out) {
   const double* qr = qd + (t * H + h) * (int64_t)D;
+  double* s = (double*)malloc(sizeof(double) * (size_t)(n_keys > 0 ? n_keys : 1));
+  double m = -INFINITY;
+  for (int64_t j = 0; j < n_keys; ++j) {
+    const double* kr = kd + ((lo + j) * H + h) * (int64_t)D;
+    double dot = 0.0;
+    for (int d = 0; d < D; ++d) dot += qr[d] * kr[d];
+    s[j] = scale * dot;
+    if (s[j] > m) m = s[j];
+  }
+  double den = 0.0;
+  for (int d = 0; d < D; ++d) ot[d] = 0.0;
+  for (int64_t j = 0; j < n_keys; ++j) {
+    const double pj = exp(s[j] - m);
+    const double pq = e4m3_value(e4m3_code((float)pj));
+    den += pj;
+    const double* vr = vd + ((lo + j) * H + h) * (int64_t)D;
+    for (int d = 0; d < D; ++d) ot[d] += pq * vr[d];
+  }
+  for (int d = 0; d < D; ++d) ot[d] /= den;
+  if (lse_out) *lse_out = m + log(den);
+  free(s);
+}
+
+/*
+ * The same FP8 attention accumulated the way a streaming (online-softmax)
+ * implementation does it: NOT the definition above but the rounding schedule
+ * of such an implementation, kept as a second, tighter check on one. Per
+ * row, over key blocks of kblock keys counted from the request's first token,
+ * in order, with u = s / ln 2 (log2 units):
+ *   - the running maximum m is set by the first block and afterwards moves
+ *     only when a block's maximum exceeds it by more than threshold; the sums
+ *     are then scaled by 2^(m_old - m_new);
+ *   - each key adds p = 2^(u - m) to the denominator l and e4m3(p) * v~ to
+ *     the numerator (p <= 2^threshold);
+ *   - o = numerator / l and lse = (m + log2 l) ln 2.
+ * With threshold = 0 and one block per request this is the definition; any
+ * other schedule rounds each p against a smaller maximum, which changes each
+ * numerator term by at most one e4m3 step.
+ */
+static void fp8_row_online(const double* qd, const double* kd, const double* vd, int64_t lo, int64_t n_keys,
+                           int64_t t, int H, int h, int D, double scale, int kblock, double threshold, double* ot,
+                           double* lse_out) {
+  const double* qr = qd + (t * H + h) * (int64_t)D;
   double* num = (double*)calloc((size_t)D, sizeof(double));
+  double* ublock = (double*)malloc(sizeof(double) * (size_t)kblock);
   double mrun = -INFINITY, den = 0.0;
-  for (int64_t b0 = 0; b0 < n_keys; b0 += 128) {
-    const int64_t b1 = b0 + 128 < n_keys ? b0 + 128 : n_keys;
-    double ublock[128];
+  for (int64_t b0 = 0; b0 < n_keys; b0 += kblock) {
+    const int64_t b1 = b0 + kblock < n_keys ? b0 + kblock : n_keys;
     double bmax = -INFINITY;
     for (int64_t j = b0; j < b1; ++j) {
       const double* kr = kd + ((lo + j) * H + h) * (int64_t)D;
@@ -438,7 +488,7 @@ static void fp8_row(const double* qd, const double* kd, const double* vd, int64_
     }
     if (b0 == 0) {
       mrun = bmax;
-    } else if (bmax > mrun + 8.0) {
+    } else if (bmax > mrun + threshold) {
       const double alpha = exp2(mrun - bmax);
       den *= alpha;
       for (int d = 0; d < D; ++d) num[d] *= alpha;
@@ -454,13 +504,18 @@ static void fp8_row(const double* qd, const double* kd, const double* vd, int64_
   }
   for (int d = 0; d < D; ++d) ot[d] = num[d] / den;
   if (lse_out) *lse_out = (mrun + log2(den)) * log(2.0);
+  free(ublock);
   free(num);
 }
 
-int oracle_varlen_attn_fp8(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
-                           const int32_t* cu, int B, int64_t T, int H, int D, double scale, const int32_t* rows,
-                           int64_t nrows, double* o, double* lse, float* deq_out) {
+/* Both FP8 attentions: online == 0 the definition, else the online schedule
+ * with (kblock, threshold). */
+static int fp8_attention(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
+                         const int32_t* cu, int B, int64_t T, int H, int D, double scale, int online, int kblock,
+                         double threshold, const int32_t* rows, int64_t nrows, double* o, double* lse,
+                         float* deq_out) {
   if (check_cu(cu, B, T) || H <= 0 || D <= 0) return -1;
+  if (online && (kblock <= 0 || !(threshold >= 0.0))) return -1;
   const int64_t n = T * (int64_t)H * D;
   uint8_t* c8 = (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
   float* dq = (float*)malloc(sizeof(float) * (size_t)H * 3);
@@ -484,8 +539,13 @@ int oracle_varlen_attn_fp8(const void* q, const void* k, const void* v, int in_k
         const int64_t t = rows ? rows[r] : r;
         const int seg = (t >= 0 && t < T) ? segment_of(cu, B, t) : -1;
         if (seg < 0) { ++bad; continue; }
-        fp8_row(xd[0], xd[1], xd[2], cu[seg], (int64_t)cu[seg + 1] - cu[seg], t, H, h, D, scale,
-                o + (r * H + h) * (int64_t)D, lse ? &lse[r * H + h] : NULL);
+        const int64_t lo = cu[seg], n_keys = (int64_t)cu[seg + 1] - cu[seg];
+        double* ot = o + (r * H + h) * (int64_t)D;
+        double* lt = lse ? &lse[r * H + h] : NULL;
+        if (online)
+          fp8_row_online(xd[0], xd[1], xd[2], lo, n_keys, t, H, h, D, scale, kblock, threshold, ot, lt);
+        else
+          fp8_row(xd[0], xd[1], xd[2], lo, n_keys, t, H, h, D, scale, ot, lt);
       }
     }
     if (bad) rc = -1;
@@ -495,6 +555,20 @@ int oracle_varlen_attn_fp8(const void* q, const void* k, const void* v, int in_k
   free(c8);
   free(dq);
   return rc;
+}
+
+int oracle_varlen_attn_fp8(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
+                           const int32_t* cu, int B, int64_t T, int H, int D, double scale, const int32_t* rows,
+                           int64_t nrows, double* o, double* lse, float* deq_out) {
+  return fp8_attention(q, k, v, in_kind, stride_t, cu, B, T, H, D, scale, 0, 0, 0.0, rows, nrows, o, lse, deq_out);
+}
+
+int oracle_varlen_attn_fp8_online(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
+                                  const int32_t* cu, int B, int64_t T, int H, int D, double scale, int kblock,
+                                  double threshold, const int32_t* rows, int64_t nrows, double* o, double* lse,
+                                  float* deq_out) {
+  return fp8_attention(q, k, v, in_kind, stride_t, cu, B, T, H, D, scale, 1, kblock, threshold, rows, nrows, o, lse,
+                       deq_out);
 }
 
 /* e4m3 codes of a float32 array (the conversion alone, for its pins). */
@@ -507,9 +581,10 @@ void oracle_e4m3_codes(const float* x, int64_t n, uint8_t* codes) {
  * P x V work of unimportant blocks (first page, bullet on TRTLLM_ATTN SAGE and
  * Skip-Softmax; second page, section "System-wide optimizations in
  * vLLM-Omni", bullet "Sparse & quantized attention"). The pages name the idea
- * only. The reading taken:
- *   - a block is 32 consecutive query rows x 128 consecutive keys of one
- *     request and head, both counted from the request's first token; key
+ * only, not a block size. The reading taken, for a block geometry given by
+ * the caller:
+ *   - a block is qrows consecutive query rows x kblock consecutive keys of
+ *     one request and head, both counted from the request's first token; key
  *     blocks are visited in increasing order;
  *   - with u(r,k) = s(r,k) / ln 2 (the score s includes the softmax scale),
  *     key block j >= 1 is skipped for query block b when every row r of b
@@ -519,22 +594,21 @@ void oracle_e4m3_codes(const float* x, int64_t n, uint8_t* codes) {
  *   - a skipped block contributes nothing: o_r = sum_kept e^(s-m) v /
  *     sum_kept e^(s-m) with m the maximum over kept keys, lse_r = m + ln(sum).
  * A very large tau skips nothing and gives oracle_varlen_attn's result.
- * rows: tokens to output (NULL = all T); each row's whole 32-row block is
+ * rows: tokens to output (NULL = all T); each row's whole query block is
  * evaluated to take that block's decisions. counts (nullable, filled only
- * when rows == NULL): counts[0] = skipped (32-row block, head, key block)
- * triples; counts[1] = skipped (128-row tile, head, key block) triples, a
- * 128-row tile (also counted from the request's first token) skipping a key
- * block when all of its 32-row blocks inside the request do.
+ * when rows == NULL): counts[0] = skipped (query block, head, key block)
+ * triples; counts[1] = skipped (tile, head, key block) triples, a tile being
+ * tile_rows consecutive query rows (a multiple of qrows, also counted from the
+ * request's first token) that skips a key block when all of its query blocks
+ * inside the request do.
  */
-#define ORACLE_SKIP_QROWS 32
-#define ORACLE_SKIP_KEYS 128
-#define ORACLE_SKIP_TILE 128
 
 /* Keep flags of the key blocks of query block [r0, r1) (rows of one request
- * starting at lo, n_keys keys), head h. keep: [ceil(n_keys / 128)]. */
+ * starting at lo, n_keys keys), head h. keep: [ceil(n_keys / kblock)]. */
 static void skip_block_flags(const void* q, const void* k, int in_kind, int64_t stride_t, int64_t lo, int64_t n_keys,
-                             int64_t r0, int64_t r1, int h, int D, double scale, double tau, unsigned char* keep) {
-  const int64_t nkb = (n_keys + ORACLE_SKIP_KEYS - 1) / ORACLE_SKIP_KEYS;
+                             int64_t r0, int64_t r1, int h, int D, double scale, double tau, int kblock,
+                             unsigned char* keep) {
+  const int64_t nkb = (n_keys + kblock - 1) / kblock;
   const int64_t nr = r1 - r0;
   double* tmax = (double*)malloc(sizeof(double) * (size_t)(nr * nkb));
   double* qt = (double*)malloc(sizeof(double) * (size_t)D);
@@ -547,7 +621,7 @@ static void skip_block_flags(const void* q, const void* k, int in_kind, int64_t 
       const int64_t key_at = (lo + j) * stride_t + (int64_t)h * D;
       for (int d = 0; d < D; ++d) dot += qt[d] * load(k, in_kind, key_at + d);
       const double u = scale * dot / log(2.0);
-      double* tm = &tmax[i * nkb + j / ORACLE_SKIP_KEYS];
+      double* tm = &tmax[i * nkb + j / kblock];
       if (u > *tm) *tm = u;
     }
   }
@@ -567,14 +641,14 @@ static void skip_block_flags(const void* q, const void* k, int in_kind, int64_t 
 
 /* Output row t (of request lo, n_keys), head h, over the kept key blocks. */
 static void skip_row_output(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t, int64_t lo,
-                            int64_t n_keys, int64_t t, int h, int D, double scale, const unsigned char* keep, double* ot,
-                            double* lse_out) {
+                            int64_t n_keys, int64_t t, int h, int D, double scale, int kblock, const unsigned char* keep,
+                            double* ot, double* lse_out) {
   double* sc = (double*)malloc(sizeof(double) * (size_t)n_keys);
   double* qt = (double*)malloc(sizeof(double) * (size_t)D);
   for (int d = 0; d < D; ++d) qt[d] = load(q, in_kind, t * stride_t + (int64_t)h * D + d);
   double m = -INFINITY;
   for (int64_t j = 0; j < n_keys; ++j) {
-    if (!keep[j / ORACLE_SKIP_KEYS]) continue;
+    if (!keep[j / kblock]) continue;
     double dot = 0.0;
     const int64_t key_at = (lo + j) * stride_t + (int64_t)h * D;
     for (int d = 0; d < D; ++d) dot += qt[d] * load(k, in_kind, key_at + d);
@@ -584,7 +658,7 @@ static void skip_row_output(const void* q, const void* k, const void* v, int in_
   double mass = 0.0;
   for (int d = 0; d < D; ++d) ot[d] = 0.0;
   for (int64_t j = 0; j < n_keys; ++j) {
-    if (!keep[j / ORACLE_SKIP_KEYS]) continue;
+    if (!keep[j / kblock]) continue;
     const double pj = exp(sc[j] - m);
     mass += pj;
     const int64_t val_at = (lo + j) * stride_t + (int64_t)h * D;
@@ -598,8 +672,10 @@ static void skip_row_output(const void* q, const void* k, const void* v, int in_
 
 int oracle_varlen_attn_skip(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
                             const int32_t* cu, int B, int64_t T, int H, int D, double scale, double tau,
-                            const int32_t* rows, int64_t nrows, double* o, double* lse, int64_t* counts) {
+                            int qrows, int kblock, int tile_rows, const int32_t* rows, int64_t nrows, double* o,
+                            double* lse, int64_t* counts) {
   if (check_cu(cu, B, T) || H <= 0 || D <= 0 || isnan(tau)) return -1;
+  if (qrows <= 0 || kblock <= 0 || tile_rows <= 0 || tile_rows % qrows) return -1;
   if (rows != NULL) {
     int64_t bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) collapse(2) reduction(+ : bad)
@@ -609,12 +685,12 @@ int oracle_varlen_attn_skip(const void* q, const void* k, const void* v, int in_
         const int seg = (t >= 0 && t < T) ? segment_of(cu, B, t) : -1;
         if (seg < 0) { ++bad; continue; }
         const int64_t lo = cu[seg], n_keys = (int64_t)cu[seg + 1] - (int64_t)cu[seg];
-        const int64_t r0 = lo + ((t - lo) / ORACLE_SKIP_QROWS) * ORACLE_SKIP_QROWS;
-        const int64_t r1 = r0 + ORACLE_SKIP_QROWS < lo + n_keys ? r0 + ORACLE_SKIP_QROWS : lo + n_keys;
-        unsigned char* keep = (unsigned char*)malloc((size_t)((n_keys + ORACLE_SKIP_KEYS - 1) / ORACLE_SKIP_KEYS));
-        skip_block_flags(q, k, in_kind, stride_t, lo, n_keys, r0, r1, h, D, scale, tau, keep);
-        skip_row_output(q, k, v, in_kind, stride_t, lo, n_keys, t, h, D, scale, keep, o + (r * H + h) * (int64_t)D,
-                        lse ? &lse[r * H + h] : NULL);
+        const int64_t r0 = lo + ((t - lo) / qrows) * qrows;
+        const int64_t r1 = r0 + qrows < lo + n_keys ? r0 + qrows : lo + n_keys;
+        unsigned char* keep = (unsigned char*)malloc((size_t)((n_keys + kblock - 1) / kblock));
+        skip_block_flags(q, k, in_kind, stride_t, lo, n_keys, r0, r1, h, D, scale, tau, kblock, keep);
+        skip_row_output(q, k, v, in_kind, stride_t, lo, n_keys, t, h, D, scale, kblock, keep,
+                        o + (r * H + h) * (int64_t)D, lse ? &lse[r * H + h] : NULL);
         free(keep);
       }
     }
@@ -624,24 +700,24 @@ int oracle_varlen_attn_skip(const void* q, const void* k, const void* v, int in_
   for (int seg = 0; seg < B; ++seg) {
     const int64_t lo = cu[seg], n_keys = (int64_t)cu[seg + 1] - (int64_t)cu[seg];
     if (n_keys == 0) continue;
-    const int64_t nqb = (n_keys + ORACLE_SKIP_QROWS - 1) / ORACLE_SKIP_QROWS;
-    const int64_t nkb = (n_keys + ORACLE_SKIP_KEYS - 1) / ORACLE_SKIP_KEYS;
+    const int64_t nqb = (n_keys + qrows - 1) / qrows;
+    const int64_t nkb = (n_keys + kblock - 1) / kblock;
     unsigned char* keep = (unsigned char*)malloc((size_t)(H * nqb * nkb));
 #pragma omp parallel for schedule(dynamic, 1) collapse(2) reduction(+ : n_block)
     for (int64_t b = 0; b < nqb; ++b) {
       for (int h = 0; h < H; ++h) {
-        const int64_t r0 = lo + b * ORACLE_SKIP_QROWS;
-        const int64_t r1 = r0 + ORACLE_SKIP_QROWS < lo + n_keys ? r0 + ORACLE_SKIP_QROWS : lo + n_keys;
+        const int64_t r0 = lo + b * qrows;
+        const int64_t r1 = r0 + qrows < lo + n_keys ? r0 + qrows : lo + n_keys;
         unsigned char* kp = keep + ((int64_t)h * nqb + b) * nkb;
-        skip_block_flags(q, k, in_kind, stride_t, lo, n_keys, r0, r1, h, D, scale, tau, kp);
+        skip_block_flags(q, k, in_kind, stride_t, lo, n_keys, r0, r1, h, D, scale, tau, kblock, kp);
         for (int64_t t = r0; t < r1; ++t)
-          skip_row_output(q, k, v, in_kind, stride_t, lo, n_keys, t, h, D, scale, kp, o + (t * H + h) * (int64_t)D,
-                          lse ? &lse[t * H + h] : NULL);
+          skip_row_output(q, k, v, in_kind, stride_t, lo, n_keys, t, h, D, scale, kblock, kp,
+                          o + (t * H + h) * (int64_t)D, lse ? &lse[t * H + h] : NULL);
         for (int64_t jb = 0; jb < nkb; ++jb) n_block += !kp[jb];
       }
     }
-    /* a 128-row tile skips key block jb when each of its 32-row blocks inside the request does */
-    const int64_t per_tile = ORACLE_SKIP_TILE / ORACLE_SKIP_QROWS;
+    /* a tile skips key block jb when each of its query blocks inside the request does */
+    const int64_t per_tile = tile_rows / qrows;
     for (int h = 0; h < H; ++h)
       for (int64_t tb = 0; tb * per_tile < nqb; ++tb)
         for (int64_t jb = 0; jb < nkb; ++jb) {

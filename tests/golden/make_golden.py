@@ -32,9 +32,11 @@ def summarise(a):
 def variants(w, p, a):
     """The widened rows on the same configuration: three-axis RoPE (the
     200-token request laid out as a 2 x 10 x 10 grid, sections 8 / 12 / 12),
-    the full-width norm, block skipping at tau = 4 on block-scaled inputs,
-    attention with FP8 Q, K and with FP8 Q, K, V, P, and the three linear
-    layers with their fused epilogues."""
+    the full-width norm, block skipping at tau = 4 on block-scaled inputs
+    (blocks of 16 query rows x 64 keys, tiles of 64 rows), attention with FP8
+    Q, K and with FP8 Q, K, V, P (the definition, and the online schedule with
+    blocks of 64 keys and threshold 4), and the three linear layers with their
+    fused epilogues."""
     out = {}
     scale = 1.0 / math.sqrt(w.D)
     y = oracle.qk_norm_rope_3axis(p["q"], p["w_q"], w.positions3(video_grid=(2, 10, 10)), (8, 12, 12), w.eps,
@@ -43,7 +45,8 @@ def variants(w, p, a):
     y = oracle.qk_fullc_norm_rope(p["q"], wl.fullc_weights(w)["w_q"], p["pos"], w.eps, w.rope_base)
     out["q_fullc_norm_rope"] = {"summary": summarise(y), "head0": [y[r, 0, :8].tolist() for r in ROWS]}
     b = wl.block_scaled_attention_inputs(w)
-    o, lse, counts = oracle.varlen_attn_skip(b["q"], b["k"], b["v"], b["cu_seqlens"], scale, 4.0)
+    o, lse, counts = oracle.varlen_attn_skip(b["q"], b["k"], b["v"], b["cu_seqlens"], scale, 4.0, block=(16, 64),
+                                             tile_rows=64)
     out["attn_skip_tau4"] = {"summary": summarise(o), "lse_summary": summarise(lse), "counts": list(counts),
                              "head0": [o[r, 0, :8].tolist() for r in ROWS]}
     o, lse, _, _, deq = oracle.varlen_attn_fp8qk(a["q"], a["k"], a["v"], a["cu_seqlens"], scale)
@@ -52,6 +55,10 @@ def variants(w, p, a):
     o, lse, deq = oracle.varlen_attn_fp8(a["q"], a["k"], a["v"], a["cu_seqlens"], scale)
     out["attn_fp8"] = {"summary": summarise(o), "lse_summary": summarise(lse), "deq": deq.tolist(),
                        "head0": [o[r, 0, :8].tolist() for r in ROWS]}
+    o, lse, deq = oracle.varlen_attn_fp8_online(a["q"], a["k"], a["v"], a["cu_seqlens"], scale, kblock=64,
+                                                threshold=4.0)
+    out["attn_fp8_online_64_4"] = {"summary": summarise(o), "lse_summary": summarise(lse), "deq": deq.tolist(),
+                                   "head0": [o[r, 0, :8].tolist() for r in ROWS]}
     for name in ("o_proj", "w1", "w2"):
         d = wl.linear_inputs(w, name)
         if name == "w1":

@@ -136,20 +136,30 @@ def test_fp8_with_block_skipping_is_skipping_on_the_dequantised_inputs():
     cu = np.array([0, 400, T], np.int32)
     scale = 1.0 / math.sqrt(D)
     counts = []
-    o, lse, q8, k8, deq = oracle.varlen_attn_fp8qk(q, k, v, cu, scale, tau=6.0, counts_out=counts)
+    o, lse, q8, k8, deq = oracle.varlen_attn_fp8qk(q, k, v, cu, scale, tau=6.0, skip_block=(16, 64),
+                                                   skip_tile_rows=64, counts_out=counts)
     qd = _decode(q8) * deq[None, :H, None]
     kd = _decode(k8) * deq[None, H:, None]
-    os_, ls, cs = oracle.varlen_attn_skip(qd, kd, v, cu, scale, 6.0)
+    os_, ls, cs = oracle.varlen_attn_skip(qd, kd, v, cu, scale, 6.0, block=(16, 64), tile_rows=64)
     assert counts == [cs] and cs[0] > 0
     assert np.array_equal(o, os_) and np.array_equal(lse, ls)
     o_inf, _, _, _, _ = oracle.varlen_attn_fp8qk(q, k, v, cu, scale)
     on, _, _, _, _ = oracle.varlen_attn_fp8qk(q, k, v, cu, scale, tau=math.inf)
     assert np.array_equal(o_inf, on)
+    with pytest.raises(ValueError):
+        oracle.varlen_attn_fp8qk(q, k, v, cu, scale, tau=6.0)  # a finite tau needs the block geometry
 
 
 # ---------------------------------------------------------------- Q, K, V and P in FP8
+#
+# The definition: p_j = exp(s_j - m) against the row's exact maximum m,
+# e4m3(p_j) in the numerator, p_j in the denominator. The online schedule
+# (oracle.varlen_attn_fp8_online) rounds each p against the running maximum
+# of a streaming implementation instead; it is pinned separately below, and
+# against the definition by the bound that follows from e4m3's step.
 
-def _one_row_case(k_vals, v_vals, scale):
+
+def _one_row_case(k_vals, v_vals, scale, online=None):
     """One request, one head, D = 1, q = 1.75: keys k_vals, values v_vals.
     Every tensor's amax is 1.75 = 448 * 2^-8, so its scale is exactly 2^-8
     and values that are e4m3 codes times 2^-8 quantise exactly."""
@@ -157,7 +167,11 @@ def _one_row_case(k_vals, v_vals, scale):
     q = np.full((L, 1, 1), 1.75)
     k = np.array(k_vals, np.float64).reshape(L, 1, 1)
     v = np.array(v_vals, np.float64).reshape(L, 1, 1)
-    o, lse, _ = oracle.varlen_attn_fp8(q, k, v, np.array([0, L], np.int32), scale)
+    cu = np.array([0, L], np.int32)
+    if online is None:
+        o, lse, _ = oracle.varlen_attn_fp8(q, k, v, cu, scale)
+    else:
+        o, lse, _ = oracle.varlen_attn_fp8_online(q, k, v, cu, scale, kblock=online[0], threshold=online[1])
     return o[0, 0, 0], lse[0, 0]
 
 
@@ -171,18 +185,26 @@ def test_fp8_p_rounds_in_the_numerator_only():
     assert abs(lse - (0.6 + math.log2(1.0 + p2)) * math.log(2.0)) <= 1e-12
 
 
-def test_fp8_running_maximum_moves_only_beyond_eight():
-    # 128 keys with k = 0 (block 0, u = 0), then one key with k = 1.75
-    # (block 1) whose u is 5.3: within 8 of the maximum, so m stays 0,
-    # p = 2^5.3 = 39.40 and e4m3 rounds it to 40; values 0 then 1.75
-    k = [0.0] * 128 + [1.75]
-    o, _ = _one_row_case(k, [0.0] * 128 + [1.75], 5.3 * math.log(2.0) / 1.75 ** 2)
-    assert abs(o - 1.75 * 40.0 / (128.0 + 2.0 ** 5.3)) <= 1e-12
-    # u = 9.3 is beyond 8: m moves to 9.3, block 0's sums scale by 2^-9.3 and
-    # the new key has p = 1 exactly; block-0 values 0.5
-    o, _ = _one_row_case(k, [0.5] * 128 + [1.75], 9.3 * math.log(2.0) / 1.75 ** 2)
-    a = 2.0 ** -9.3
-    assert abs(o - (128 * 0.5 * a + 1.75) / (128 * a + 1.0)) <= 1e-12
+def test_fp8_p_is_rounded_against_the_rows_exact_maximum():
+    # keys 0 and 1.75 at scale 5.3 ln 2 / 1.75^2: u = (0, 5.3); the maximum is
+    # the second key, so p = (2^-5.3, 1) and e4m3(2^-5.3 = 0.025383) =
+    # 1.625 * 2^-6 = 0.025390625. Rounding against the first key instead would
+    # give p = (1, 2^5.3 -> 40): a different numerator.
+    o, lse = _one_row_case([0.0, 1.75], [1.75, -1.75], 5.3 * math.log(2.0) / 1.75 ** 2)
+    p1 = 2.0 ** -5.3
+    assert abs(o - 1.75 * (0.025390625 - 1.0) / (p1 + 1.0)) <= 1e-12
+    assert abs(lse - (5.3 + math.log2(1.0 + p1)) * math.log(2.0)) <= 1e-12
+
+
+def test_fp8_small_probabilities_round_on_the_subnormal_grid():
+    # keys 1.75, 0.75, 0 at scale 7.5 ln 2 / 1.75: u = (13.125, 5.625, 0), so
+    # p = (1, 2^-7.5, 2^-13.125). Below 2^-6 e4m3 steps by 2^-9: 2^-7.5 =
+    # 2.83 * 2^-9 rounds to 3 * 2^-9 and 2^-13.125 (0.11 steps) to 0, while the
+    # denominator keeps all three; values 0.5, 1.75, -1.75
+    o, lse = _one_row_case([1.75, 0.75, 0.0], [0.5, 1.75, -1.75], 7.5 * math.log(2.0) / 1.75)
+    den = 1.0 + 2.0 ** -7.5 + 2.0 ** -13.125
+    assert abs(o - (0.5 + 3 * 2.0 ** -9 * 1.75) / den) <= 1e-12
+    assert abs(lse - (13.125 + math.log2(den)) * math.log(2.0)) <= 1e-12
 
 
 def test_fp8_is_exact_on_representable_inputs():
@@ -209,16 +231,109 @@ def test_fp8_is_exact_on_representable_inputs():
     assert np.max(np.abs(o - ob)) <= 1e-12 and np.max(np.abs(lse - lb)) <= 1e-12
 
 
+def _dequantised(q, k, v):
+    return [_decode(c) * d[None, :, None] for c, d in (oracle.quantize_e4m3(x) for x in (q, k, v))]
+
+
+def _row_weights(qd, kd, cu, scale, t, h):
+    """Exact-max probabilities p_j of row t, head h over its request."""
+    i = int(np.searchsorted(cu, t, side="right") - 1)
+    s = scale * (kd[cu[i]:cu[i + 1], h] @ qd[t, h])
+    return np.exp(s - s.max()), int(cu[i]), int(cu[i + 1])
+
+
 def test_fp8_error_bound_against_exact_p():
-    # P's rounding moves each numerator term by at most 2^-4 of itself, so O
-    # moves by at most 2^-4 max|V~| from the attention with exact P on the
-    # same dequantised Q, K, V
+    # e4m3 rounds p <= 1 to within 2^-4 p in its normal range and within 2^-10
+    # below it, so every element of O lies within
+    # sum_j max(2^-4 p_j, 2^-10) |v_j| / sum_j p_j of the attention with exact P
+    # on the same dequantised Q, K, V
     g = np.random.default_rng(9)
     T, H, D = 500, 2, 32
     q, k, v = (g.standard_normal((T, H, D)) for _ in range(3))
     cu = np.array([0, 130, 500], np.int32)
     scale = 1.0 / math.sqrt(D)
-    o, _, deq = oracle.varlen_attn_fp8(q, k, v, cu, scale)
-    dec = [_decode(oracle.quantize_e4m3(x)[0]) * oracle.quantize_e4m3(x)[1][None, :, None] for x in (q, k, v)]
-    ob, _ = padded_masked_attention(dec[0], dec[1], dec[2], cu, scale)
-    assert 0 < np.max(np.abs(o - ob)) <= 2.0 ** -4 * np.abs(dec[2]).max()
+    o, _, _ = oracle.varlen_attn_fp8(q, k, v, cu, scale)
+    qd, kd, vd = _dequantised(q, k, v)
+    ob, _ = padded_masked_attention(qd, kd, vd, cu, scale)
+    assert np.max(np.abs(o - ob)) > 0
+    for t in range(0, T, 7):
+        for h in range(H):
+            p, lo, hi = _row_weights(qd, kd, cu, scale, t, h)
+            bound = (np.maximum(2.0 ** -4 * p, 2.0 ** -10)[:, None] * np.abs(vd[lo:hi, h])).sum(0) / p.sum()
+            assert np.all(np.abs(o[t, h] - ob[t, h]) <= bound * (1 + 1e-9) + 1e-15)
+
+
+def test_fp8_sampled_rows_equal_full_evaluation():
+    g = np.random.default_rng(10)
+    T, H, D = 300, 2, 16
+    q, k, v = (g.standard_normal((T, H, D)) for _ in range(3))
+    cu = np.array([0, 17, 300], np.int32)
+    o, lse, _ = oracle.varlen_attn_fp8(q, k, v, cu, 0.25)
+    rows = np.array([0, 16, 17, 150, 299], np.int32)
+    o2, l2, _ = oracle.varlen_attn_fp8(q, k, v, cu, 0.25, rows=rows)
+    assert np.array_equal(o2, o[rows]) and np.array_equal(l2, lse[rows])
+
+
+# ----------------------------------------------- the online schedule of the same FP8 attention
+
+@pytest.mark.parametrize("kblock, threshold", [(128, 8.0), (64, 4.0)])
+def test_online_running_maximum_moves_only_beyond_the_threshold(kblock, threshold):
+    # kblock keys with k = 0 (block 0, u = 0), then one key with k = 1.75
+    # (block 1) whose u is threshold - 2.7: within the threshold, so m stays
+    # 0 and p = 2^u is rounded as it is (2^5.3 = 39.40 -> 40, 2^1.3 = 2.462 ->
+    # 2.5); values 0 then 1.75
+    u = threshold - 2.7
+    k = [0.0] * kblock + [1.75]
+    o, _ = _one_row_case(k, [0.0] * kblock + [1.75], u * math.log(2.0) / 1.75 ** 2, online=(kblock, threshold))
+    rounded = {8.0: 40.0, 4.0: 2.5}[threshold]
+    assert abs(o - 1.75 * rounded / (kblock + 2.0 ** u)) <= 1e-12
+    # u = threshold + 1.3 is beyond it: m moves, block 0's sums scale by 2^-u
+    # and the new key has p = 1 exactly; block-0 values 0.5
+    u = threshold + 1.3
+    o, _ = _one_row_case(k, [0.5] * kblock + [1.75], u * math.log(2.0) / 1.75 ** 2, online=(kblock, threshold))
+    a = 2.0 ** -u
+    assert abs(o - (kblock * 0.5 * a + 1.75) / (kblock * a + 1.0)) <= 1e-12
+
+
+def test_online_with_one_block_per_request_is_the_definition():
+    g = np.random.default_rng(12)
+    T, H, D = 400, 2, 32
+    q, k, v = (g.standard_normal((T, H, D)) * 2 for _ in range(3))
+    cu = np.array([0, 150, 400], np.int32)
+    o, lse, d = oracle.varlen_attn_fp8(q, k, v, cu, 0.2)
+    for threshold in (0.0, 8.0):
+        o2, l2, d2 = oracle.varlen_attn_fp8_online(q, k, v, cu, 0.2, kblock=256, threshold=threshold)
+        assert np.array_equal(d, d2)
+        assert np.max(np.abs(o - o2)) <= 1e-12 and np.max(np.abs(lse - l2)) <= 1e-12
+
+
+@pytest.mark.parametrize("kblock, threshold", [(128, 8.0), (32, 2.0)])
+def test_online_schedule_against_the_definition_bound(kblock, threshold):
+    # each p is rounded against a maximum that is never above the row's: both
+    # roundings lie within max(2^-4 p, 2^-10) of p (in units of the row's
+    # maximum), so they differ by at most max(2^-3 p, 2^-9); with P in the
+    # numerator only, O differs by at most sum_j max(2^-3 p_j, 2^-9) |v_j| / l.
+    # The lse is the same sum either way.
+    g = np.random.default_rng(13)
+    T, H, D = 600, 2, 32
+    q, k, v = (g.standard_normal((T, H, D)) for _ in range(3))
+    k[300:, :, :] *= 2.0  # later keys score higher: the running maximum lags
+    cu = np.array([0, 90, 600], np.int32)
+    scale = 1.0 / math.sqrt(D)
+    o, lse, _ = oracle.varlen_attn_fp8(q, k, v, cu, scale)
+    o2, l2, _ = oracle.varlen_attn_fp8_online(q, k, v, cu, scale, kblock=kblock, threshold=threshold)
+    assert np.max(np.abs(o - o2)) > 0 and np.max(np.abs(lse - l2)) <= 1e-12
+    qd, kd, vd = _dequantised(q, k, v)
+    for t in range(0, T, 5):
+        for h in range(H):
+            p, lo, hi = _row_weights(qd, kd, cu, scale, t, h)
+            bound = (np.maximum(2.0 ** -3 * p, 2.0 ** -9)[:, None] * np.abs(vd[lo:hi, h])).sum(0) / p.sum()
+            assert np.all(np.abs(o[t, h] - o2[t, h]) <= bound * (1 + 1e-9) + 1e-15)
+
+
+def test_online_schedule_arguments_are_validated():
+    x = np.zeros((4, 1, 8))
+    cu = np.array([0, 4], np.int32)
+    for kb, th in [(0, 8.0), (128, -1.0), (128, float("nan"))]:
+        with pytest.raises(ValueError):
+            oracle.varlen_attn_fp8_online(x, x, x, cu, 1.0, kblock=kb, threshold=th)

@@ -59,12 +59,15 @@ def test_oracle_variants_match_stored_tiny_config_outputs():
     _summary_close(y, g["q_fullc_norm_rope"]["summary"])
     np.testing.assert_allclose([y[r, 0, :8] for r in rows], g["q_fullc_norm_rope"]["head0"], atol=1e-12)
     b = wl.block_scaled_attention_inputs(w)
-    o, lse, counts = oracle.varlen_attn_skip(b["q"], b["k"], b["v"], b["cu_seqlens"], scale, 4.0)
+    o, lse, counts = oracle.varlen_attn_skip(b["q"], b["k"], b["v"], b["cu_seqlens"], scale, 4.0, block=(16, 64),
+                                             tile_rows=64)
     assert list(counts) == g["attn_skip_tau4"]["counts"]
     _summary_close(o, g["attn_skip_tau4"]["summary"])
     _summary_close(lse, g["attn_skip_tau4"]["lse_summary"])
     np.testing.assert_allclose([o[r, 0, :8] for r in rows], g["attn_skip_tau4"]["head0"], atol=1e-12)
-    for key, fn in (("attn_fp8qk", oracle.varlen_attn_fp8qk), ("attn_fp8", oracle.varlen_attn_fp8)):
+    online = lambda *x: oracle.varlen_attn_fp8_online(*x, kblock=64, threshold=4.0)
+    for key, fn in (("attn_fp8qk", oracle.varlen_attn_fp8qk), ("attn_fp8", oracle.varlen_attn_fp8),
+                    ("attn_fp8_online_64_4", online)):
         res = fn(a["q"], a["k"], a["v"], a["cu_seqlens"], scale)
         o, lse, deq = res[0], res[1], res[-1]
         assert np.array_equal(np.asarray(deq, np.float32), np.asarray(g[key]["deq"], np.float32))

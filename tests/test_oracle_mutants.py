@@ -51,7 +51,9 @@ MUTANTS = {
     "fullc_mean_over_one_head": ("ms /= (double)width;", "ms /= (double)D;"),
     "fullc_weight_of_first_head": ("* inv * load(w, w_kind, (int64_t)h * D + d);", "* inv * load(w, w_kind, d);"),
     "skip_first_row_decides": ("for (int64_t i = 0; i < nr && skip; ++i) {", "for (int64_t i = 0; i < 1 && skip; ++i) {"),
-    "skip_query_block_64": ("#define ORACLE_SKIP_QROWS 32", "#define ORACLE_SKIP_QROWS 64"),
+    "skip_key_block_doubled": ("double* tm = &tmax[i * nkb + j / kblock];", "double* tm = &tmax[i * nkb + j / (2 * kblock)];"),
+    "skip_sampled_row_block_doubled": ("const int64_t r0 = lo + ((t - lo) / qrows) * qrows;",
+                                       "const int64_t r0 = lo + ((t - lo) / (2 * qrows)) * (2 * qrows);"),
     "skip_threshold_sign": ("if (!(tmax[i * nkb + jb] < M - tau)) skip = 0;", "if (!(tmax[i * nkb + jb] < M + tau)) skip = 0;"),
     "skip_natural_log_units": ("const double u = scale * dot / log(2.0);", "const double u = scale * dot;"),
     "e4m3_ties_away_from_zero": ("const double r = rint(a / quantum) * quantum;",
@@ -63,12 +65,17 @@ MUTANTS = {
                                 "    for (int64_t t = 0; t < 1; ++t)\n      for (int d = 0; d < D; ++d) {\n        const float v = (float)fabs("),
     "fp8_range_240": ("const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;",
                       "const float inv = amax > 0.0f ? 240.0f / amax : 1.0f;"),
-    "fp8_lazy_threshold_zero": ("} else if (bmax > mrun + 8.0) {", "} else if (bmax > mrun) {"),
-    "fp8_p_not_quantised": ("const double pq = e4m3_value(e4m3_code((float)pj));", "const double pq = pj;"),
-    "fp8_denominator_quantised": ("      den += pj;\n", "      den += pq;\n"),
-    "fp8_numerator_not_rescaled": ("      for (int d = 0; d < D; ++d) num[d] *= alpha;\n", ""),
+    "fp8_p_not_quantised": ("\n    const double pq = e4m3_value(e4m3_code((float)pj));", "\n    const double pq = pj;"),
+    "fp8_denominator_quantised": ("\n    den += pj;\n", "\n    den += pq;\n"),
+    "fp8_reference_first_key": ("    s[j] = scale * dot;\n    if (s[j] > m) m = s[j];",
+                                "    s[j] = scale * dot;\n    if (j == 0) m = s[j];"),
     "fp8_v_with_q_scale": ("xd[i][e] = e4m3_value(c8[e]) * (double)dq[(int64_t)i * H + (e / D) % H];",
                            "xd[i][e] = e4m3_value(c8[e]) * (double)dq[(e / D) % H];"),
+    "fp8_online_threshold_zero": ("} else if (bmax > mrun + threshold) {", "} else if (bmax > mrun) {"),
+    "fp8_online_p_not_quantised": ("\n      const double pq = e4m3_value(e4m3_code((float)pj));",
+                                   "\n      const double pq = pj;"),
+    "fp8_online_denominator_quantised": ("\n      den += pj;\n", "\n      den += pq;\n"),
+    "fp8_online_numerator_not_rescaled": ("      for (int d = 0; d < D; ++d) num[d] *= alpha;\n", ""),
     "linear_w_transposed": ("load(w, in_kind, (int64_t)n * K + k)", "load(w, in_kind, (int64_t)k * N + n)"),
     "linear_gate_of_first_request": ("(double)gate_res[(int64_t)seg * N + n] * y", "(double)gate_res[n] * y"),
     "linear_residual_sign": ("load(x, in_kind, t * N + n) + (double)gate_res", "load(x, in_kind, t * N + n) - (double)gate_res"),

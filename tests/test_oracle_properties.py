@@ -45,7 +45,7 @@ def test_skip_with_huge_threshold_equals_bruteforce(lens, H, D, seed):
     T = sum(lens)
     q, k, v = (g.standard_normal((T, H, D)) * 3 for _ in range(3))
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
-    o, lse, counts = oracle.varlen_attn_skip(q, k, v, cu, 0.3, 1e30)
+    o, lse, counts = oracle.varlen_attn_skip(q, k, v, cu, 0.3, 1e30, block=(16, 64), tile_rows=64)
     ob, lb = padded_masked_attention(q, k, v, cu, 0.3)
     assert counts == (0, 0)
     assert np.max(np.abs(o - ob)) <= 1e-11 and np.max(np.abs(lse - lb)) <= 1e-11
