@@ -409,11 +409,14 @@ PQK_API int pqk_linear_swiglu(const void* a, int64_t a_stride_t, const void* w1,
 PQK_API int pqk_get_device_status(void* stream);
 
 /*
- * pqk_set_wait_timeout_ns -- upper bound, in nanoseconds, on every wait of
- * the attention and linear-layer pipelines (default 1e9). A wait that runs out records
- * PQK_ERR_TIMEOUT, its thread block stops issuing work, waits (again
- * bounded) for its copies in flight, frees its tensor memory and exits.
- * Values <= 0 restore the default. Affects calls enqueued afterwards.
+ * pqk_set_wait_timeout_ns -- upper bound, in nanoseconds, on every pipeline
+ * wait of the attention and linear-layer kernels (default 1e9). A wait that
+ * runs out records PQK_ERR_TIMEOUT and its thread block stops issuing work;
+ * once all of the block's roles have stopped it waits for the copies and
+ * MMAs it still has in flight (a fixed bound of 2 s, independent of this
+ * setting), frees its tensor memory and exits. Values <= 0 restore the
+ * default; others are clamped to [1e3, 1e10] (1 us .. 10 s). Process-wide;
+ * affects calls enqueued afterwards.
  */
 PQK_API void pqk_set_wait_timeout_ns(int64_t ns);
 

@@ -38,8 +38,10 @@
 // A rows and W columns in L2.
 //
 // Every wait is bounded (the library's timeout); a wait that runs out raises
-// the block's abort flag and the device status word, in-flight copies and
-// MMAs are drained, and the tensor memory is freed before the kernel ends.
+// the block's abort flag and the device status word and every role stops
+// issuing work. Once all roles have stopped (a block barrier), the copies and
+// MMAs still in flight are drained with waits bounded by kDrainTimeoutNs,
+// not by the caller's timeout, and only then is the tensor memory freed.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -194,11 +196,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const int n_tiles_total = p.m_tiles * p.n_tiles;
+  uint32_t loads = 0;  // stage copies issued by the producer thread, for the drain
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t& it = loads;
       bool ok = true;
       for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
         const TileCoord tc = tile_coord(tile, p.m_tiles, p.n_tiles);
@@ -218,15 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++it;
         }
       }
-      if (!ok) {
-        raise_abort(abort_flag, p.status);
-        // drain: the last kStages loads may still be in flight
-        const uint32_t first = it > static_cast<uint32_t>(kStages) ? it - kStages : 0;
-        for (uint32_t idx = first; idx < it; ++idx) {
-          const volatile int no_abort = 0;
-          mbar_wait(full(idx % kStages), (idx / kStages) & 1, &no_abort, p.timeout_ns);
-        }
-      }
+      if (!ok) raise_abort(abort_flag, p.status);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer
@@ -259,14 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_commit(acc_full(acc));
       }
-      if (!ok) {
-        raise_abort(abort_flag, p.status);
-        // every MMA issued so far must complete before the tensor memory is
-        // released: the drain barrier completes once they have
-        const volatile int no_abort = 0;
-        tc_commit(drain);
-        mbar_wait(drain, 0, &no_abort, p.timeout_ns);
-      }
+      if (!ok) raise_abort(abort_flag, p.status);
     }
   } else {
     // ------------------------------------------------ epilogue warps 2-5
@@ -363,6 +351,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before_sync();
   __syncthreads();
+  // Every role has stopped, so the abort flag is final. On an abort, wait for
+  // the copies and MMAs still in flight before the memory is freed.
+  if (*abort_flag) {
+    if (warp == kProducerWarp && lane == 0) {
+      // copy idx was issued only after copy idx - kStages had landed: the
+      // last kStages copies are the ones that can be outstanding
+      const uint32_t first = loads > static_cast<uint32_t>(kStages) ? loads - kStages : 0;
+      for (uint32_t idx = first; idx < loads; ++idx) mbar_drain_wait(full(idx % kStages), (idx / kStages) & 1);
+    } else if (warp == kMmaWarp && lane == 0) {
+      // completes once every MMA this thread issued has
+      tc_commit(drain);
+      mbar_drain_wait(drain, 0);
+    }
+    __syncthreads();
+  }
   tc_fence_after_sync();
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }

@@ -96,7 +96,10 @@ const char* pqk_status_string(int status) {
 
 const char* pqk_version(void) { return "0.1.0"; }
 
-void pqk_set_wait_timeout_ns(int64_t ns) { g_timeout_ns.store(ns > 0 ? ns : 1000000000LL); }
+void pqk_set_wait_timeout_ns(int64_t ns) {
+  constexpr int64_t kDefault = 1000000000LL, kMin = 1000LL, kMax = 10000000000LL;
+  g_timeout_ns.store(ns <= 0 ? kDefault : (ns < kMin ? kMin : (ns > kMax ? kMax : ns)));
+}
 
 int pqk_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride_t,
                      int64_t k_stride_t, const void* q_weight, const void* k_weight, const int32_t* pos, int64_t T,

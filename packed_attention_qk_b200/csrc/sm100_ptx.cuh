@@ -71,6 +71,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // Hard cap on polls of one wait, on top of the time limit.
 constexpr uint32_t kMaxPolls = 1u << 26;
 
+// Bound of the waits that drain an aborting block: copies and MMAs already
+// in flight into its shared and tensor memory must land before the block
+// frees them and exits, whatever pipeline timeout the caller chose. They
+// finish within microseconds on a working GPU; the bound only keeps a broken
+// one from spinning forever.
+constexpr long long kDrainTimeoutNs = 2000000000LL;
+
 // Waits for the phase of `bar` with parity `parity` to complete. Returns
 // false (without completing) when the block's abort flag is raised or when
 // `timeout_ns` of global time or kMaxPolls polls have passed; the caller
@@ -86,6 +93,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const v
       if ((long long)(global_timer_ns() - t0) > timeout_ns || polls >= kMaxPolls) return false;
     }
   }
+}
+
+// Drain wait: the phase with parity `parity` of `bar`, bounded by
+// kDrainTimeoutNs and not by the block's abort flag.
+__device__ __forceinline__ bool mbar_drain_wait(uint32_t bar, uint32_t parity) {
+  const volatile int no_abort = 0;
+  return mbar_wait(bar, parity, &no_abort, kDrainTimeoutNs);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -38,9 +38,13 @@
 // maximum is only raised (and O, l rescaled) when the tile maximum exceeds
 // it by more than 2^8, which keeps every probability <= 256 and makes
 // rescales rare after the first tiles.
-// Every wait is bounded (pqk::mbar_wait); a wait that runs out raises the
-// block's abort flag and the device status word, and the block drains its
-// copies and MMAs in flight (bounded again), frees tensor memory and exits.
+// Every wait is bounded (pqk::mbar_wait, the caller's timeout); a wait that
+// runs out raises the block's abort flag and the device status word, and
+// every role stops issuing work. Once all roles have stopped (a block
+// barrier), the producer waits for every copy it issued that no one consumed
+// and the MMA thread for every MMA it issued (a commit on a barrier used only
+// for that), both bounded by kDrainTimeoutNs rather than the caller's
+// timeout; only then is the tensor memory freed and the block exits.
 //
 // Two compile-time variants of the same pipeline:
 //   kSkip  block skipping ("Skip-Softmax", first page, bullet on TRTLLM_ATTN
@@ -92,8 +96,8 @@ struct Layout {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  // barriers: kv_full[S], kv_empty[S], q_full, q_empty, s_full[2], p_full[2], o_done[2]
-  static constexpr int kNumBars = 2 * kStages + 8;
+  // barriers: kv_full[S], kv_empty[S], q_full, q_empty, s_full[2], p_full[2], o_done[2], drain
+  static constexpr int kNumBars = 2 * kStages + 9;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
   // block-skip votes: one byte per softmax warp, [group][tile parity][warp]
@@ -364,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto s_full = [&](int i) { return q_full + 16 + 8u * i; };
   auto p_full = [&](int i) { return q_full + 32 + 8u * i; };
   auto o_done = [&](int i) { return q_full + 48 + 8u * i; };
+  const uint32_t drain = q_full + 64;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
   volatile uint8_t* votes = smem + L::kVoteOff;
@@ -380,6 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(p_full(i), kBM);
       mbar_init(o_done(i), 1);
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -397,12 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const int n_work = p.sched[0];
+  // copies issued by the producer thread (K/V stages, Q tile pairs), for the drain
+  uint32_t load_idx = 0;
+  uint32_t q_loads = 0;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t load_idx = 0;
-      uint32_t q_loads = 0;
       int wt = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
@@ -440,19 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) {
-        raise_abort(abort_flag, p.status);
-        // drain: the last kStages loads and the last Q load may still be in flight
-        const uint32_t first = load_idx > static_cast<uint32_t>(L::kStages) ? load_idx - L::kStages : 0;
-        for (uint32_t idx = first; idx < load_idx; ++idx) {
-          const volatile int no_abort = 0;
-          mbar_wait(kv_full(idx % L::kStages), (idx / L::kStages) & 1, &no_abort, p.timeout_ns);
-        }
-        if (q_loads > 0) {
-          const volatile int no_abort = 0;
-          mbar_wait(q_full, (q_loads - 1) & 1, &no_abort, p.timeout_ns);
-        }
-      }
+      if (!ok) raise_abort(abort_flag, p.status);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer
@@ -587,17 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (kSkip && p.skip_counts != nullptr && pv_skips != 0) atomicAdd(&p.skip_counts[1], pv_skips);
-      if (!ok) {
-        raise_abort(abort_flag, p.status);
-        // every MMA issued by this thread must complete before the tensor
-        // memory is released: a fresh commit on o_done(0) completes its next
-        // phase (phase wt, or wt + 1 if this tile's commit was already made)
-        // once all of them are done
-        const volatile int no_abort = 0;
-        tc_commit(o_done(0));
-        mbar_wait(o_done(0), wt & 1, &no_abort, p.timeout_ns);
-        mbar_wait(o_done(0), (wt + 1) & 1, &no_abort, p.timeout_ns);
-      }
+      if (!ok) raise_abort(abort_flag, p.status);
     }
   } else {
     // ------------------------------------------------ softmax groups
@@ -711,6 +696,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before_sync();
   __syncthreads();
+  // Every role has stopped, so the abort flag is final. On an abort, copies
+  // and MMAs may still be in flight into this block's shared and tensor
+  // memory: wait for all of them before the memory is freed.
+  if (*abort_flag) {
+    if (warp == kProducerWarp && lane == 0) {
+      // the producer issued K/V copy idx only after copy idx - kStages had
+      // landed, so the last kStages copies (and the last Q pair) are the
+      // ones that can be outstanding; each is the newest phase of its stage
+      const uint32_t first = load_idx > static_cast<uint32_t>(L::kStages) ? load_idx - L::kStages : 0;
+      for (uint32_t idx = first; idx < load_idx; ++idx)
+        mbar_drain_wait(kv_full(idx % L::kStages), (idx / L::kStages) & 1);
+      if (q_loads > 0) mbar_drain_wait(q_full, (q_loads - 1) & 1);
+    } else if (warp == kMmaWarp && lane == 0) {
+      // a commit on the drain barrier completes once every MMA this thread
+      // issued has (and with them the arrivals of their own commits)
+      tc_commit(drain);
+      mbar_drain_wait(drain, 0);
+    }
+    __syncthreads();
+  }
   tc_fence_after_sync();
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }

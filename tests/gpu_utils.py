@@ -20,6 +20,12 @@ ATTN_MAX_ABS = 2e-2
 ATTN_REL_L2 = 1e-2
 LSE_MAX_ABS = 1e-3
 
+# The attention kernel's block-skipping geometry: a decision covers one
+# softmax warp's 32 query rows x one K/V tile of 128 keys, and a P x V
+# product (the second count) one 128-row query tile.
+SKIP_BLOCK = (32, 128)
+SKIP_TILE_ROWS = 128
+
 
 def torch_cuda():
     torch = pytest.importorskip("torch")

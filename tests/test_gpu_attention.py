@@ -112,6 +112,33 @@ def test_four_request_batch_sampled(outliers):
     check(x, w.H, w.D, rows=wl.sample_rows(w, 64), what=f"4 requests outliers={outliers}")
 
 
+def _tail_rows(w, per_segment):
+    """Seeded sample rows plus, in every request, the rows of its last
+    (ragged) 128-row tile and the first rows after each 256-row boundary of
+    the last two tiles."""
+    rows = set(int(r) for r in wl.sample_rows(w, per_segment))
+    cu = w.cu_seqlens()
+    for i in range(len(cu) - 1):
+        lo, hi = int(cu[i]), int(cu[i + 1])
+        if hi == lo:
+            continue
+        last = lo + ((hi - lo - 1) // 128) * 128
+        rows.update(range(last, hi, 7))
+        rows.update((hi - 1, hi - 2, max(lo, last - 1)))
+    return np.array(sorted(rows), np.int32)
+
+
+@pytest.mark.parametrize("config", [3, 4])
+def test_peaked_full_size_sampled_with_ragged_tails(config):
+    # Q x 8 at the full-size configurations: O is close to single V rows, so
+    # the unit-scale bound applies; the sample covers every request's ragged
+    # last tile
+    w = wl.config(config)
+    x = wl.attention_inputs(w)
+    x["q"] = wl.f32_to_bf16_bits(wl.bf16_bits_to_f32(x["q"]) * np.float32(8.0))
+    check(x, w.H, w.D, rows=_tail_rows(w, 32), what=f"peaked Q x 8, configuration {config}", peaked=True)
+
+
 def test_strided_fused_qkv_and_output_canaries():
     torch = torch_cuda()
     lens = [300, 45]

@@ -20,7 +20,8 @@ import pytest
 from oracle import oracle
 from packed_attention_qk_b200 import pqk
 from packed_attention_qk_b200 import workloads as wl
-from tests.gpu_utils import LSE_MAX_ABS, assert_attention, bf16_to_f64, max_abs, to_dev, to_dev_bf16, torch_cuda
+from tests.gpu_utils import (LSE_MAX_ABS, SKIP_BLOCK, SKIP_TILE_ROWS, assert_attention, bf16_to_f64, max_abs, to_dev,
+                             to_dev_bf16, torch_cuda)
 
 pytestmark = pytest.mark.gpu
 
@@ -98,7 +99,8 @@ def test_block_scaled_matches_oracle_and_counts(lens, H, D, seed, tau):
     scale = 1.0 / math.sqrt(D)
     assert decision_margins(x, tau, scale) >= MARGIN
     o, lse, counts = run_skip(x, tau, scale)
-    ro, rl, rc = oracle.varlen_attn_skip(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, tau)
+    ro, rl, rc = oracle.varlen_attn_skip(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, tau, block=SKIP_BLOCK,
+                                        tile_rows=SKIP_TILE_ROWS)
     assert rc[0] > 0, "the case must drop some blocks"
     assert counts == rc
     assert_attention(bf16_to_f64(o), ro, f"{lens} H{H} D{D} tau {tau}", peaked=True)
@@ -130,7 +132,8 @@ def test_local_inputs_sampled_rows():
     assert counts[0] > 0
     o = bf16_to_f64(o)[rows]
     lse = lse.cpu().numpy().astype(np.float64).T[rows]
-    ro, rl, _ = oracle.varlen_attn_skip(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, tau, rows=rows)
+    ro, rl, _ = oracle.varlen_attn_skip(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, tau, block=SKIP_BLOCK,
+                                       tile_rows=SKIP_TILE_ROWS, rows=rows)
     q, k = wl.bf16_bits_to_f64(x["q"]), wl.bf16_bits_to_f64(x["k"])
     vmax = float(np.abs(wl.bf16_bits_to_f64(x["v"])).max())
     n_clear = 0
@@ -161,7 +164,8 @@ def test_local_inputs_58048_tokens_sampled_rows():
     o, lse, counts = run_skip(x, tau, scale)
     assert counts[0] > 0
     o = bf16_to_f64(o)[rows]
-    ro, rl, _ = oracle.varlen_attn_skip(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, tau, rows=rows)
+    ro, rl, _ = oracle.varlen_attn_skip(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, tau, block=SKIP_BLOCK,
+                                       tile_rows=SKIP_TILE_ROWS, rows=rows)
     q, k = wl.bf16_bits_to_f64(x["q"]), wl.bf16_bits_to_f64(x["k"])
     vmax = float(np.abs(wl.bf16_bits_to_f64(x["v"])).max())
     n_clear = 0

@@ -16,8 +16,8 @@ import pytest
 from oracle import oracle
 from packed_attention_qk_b200 import pqk
 from packed_attention_qk_b200 import workloads as wl
-from tests.gpu_utils import (LSE_MAX_ABS, assert_attention, bf16_to_f64, max_abs, rel_l2, to_dev, to_dev_bf16,
-                             torch_cuda)
+from tests.gpu_utils import (ATTN_MAX_ABS, ATTN_REL_L2, ELEM_UNIT_MAX, LSE_MAX_ABS, SKIP_BLOCK, SKIP_TILE_ROWS,
+                             assert_attention, bf16_to_f64, max_abs, rel_l2, to_dev, to_dev_bf16, torch_cuda)
 
 pytestmark = pytest.mark.gpu
 
@@ -149,6 +149,7 @@ def test_fp8_with_block_skipping_matches_oracle_and_counts(tau):
     scale = 1.0 / math.sqrt(128)
     counts = []
     ro, rl, q8r, k8r, deqr = oracle.varlen_attn_fp8qk(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, tau=tau,
+                                                      skip_block=SKIP_BLOCK, skip_tile_rows=SKIP_TILE_ROWS,
                                                       counts_out=counts)
     H = w.H
     dec = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
@@ -190,35 +191,92 @@ def _full_fp8_gpu(x, scale):
     return o, lse, v8, deq
 
 
-def _check_full_fp8(x, scale, what, rows=None):
-    """Element-wise against the oracle, each row allowed, beyond the attention
-    tolerance, one e4m3 step (2^-4 relative) of its largest-weight key: the
-    kernel rounds fp32 probabilities, the oracle float64 ones, so a value
-    lying on an e4m3 rounding boundary may round differently."""
-    o, lse, v8, deq = _full_fp8_gpu(x, scale)
-    ro, rl, rdeq = oracle.varlen_attn_fp8(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, rows=rows)
-    T, H, D = x["q"].shape
-    assert np.array_equal(deq.cpu().numpy(), rdeq)
-    sel = np.arange(T) if rows is None else rows
-    g = bf16_to_f64(o)[sel]
-    assert rel_l2(g, ro) <= 1e-2, what
-    # largest softmax weight per (row, head), from the dequantised Q, K
-    q8, k8, _ = _quantise_gpu(x)
-    dq = deq.cpu().numpy().astype(np.float64)
+# The whole-FP8 kernel is an online softmax over K/V tiles of 128 keys whose
+# running maximum (log2 units) is set by the first tile and moves only when a
+# tile's maximum exceeds it by more than 8: its rounding schedule for P.
+KERNEL_KBLOCK, KERNEL_THRESHOLD = 128, 8.0
+
+
+def _decode(c):
     import torch
-    dec = lambda c: torch.from_numpy(c.cpu().numpy()).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
-    qd, kd = dec(q8) * dq[None, :H, None], dec(k8) * dq[None, H:2 * H, None]
-    vmax = float(np.abs(dec(v8)).max() * dq[2 * H:].max())
+    return torch.from_numpy(np.ascontiguousarray(c)).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+
+
+def _e4m3_quantum(p):
+    """Spacing of the e4m3 grid at p > 0: 2^(e - 3) in the normal range, 2^-9 below 2^-6."""
+    e = np.floor(np.log2(np.maximum(p, 2.0 ** -6)))
+    return np.exp2(e - 3)
+
+
+def _row_terms(qd, kd, scale, lo, hi, t, h):
+    """For row t, head h over keys [lo, hi): the probabilities p_j against
+    the row's exact maximum, and c_j = 2^(M - m_j), where m_j is the kernel's
+    running maximum when key j's tile is visited (c_j >= 1)."""
+    u = scale * (kd[lo:hi, h] @ qd[t, h]) / math.log(2.0)
+    M = u.max()
+    m_at = np.empty_like(u)
+    m = -np.inf
+    for b0 in range(0, hi - lo, KERNEL_KBLOCK):
+        bmax = u[b0:b0 + KERNEL_KBLOCK].max()
+        if b0 == 0 or bmax > m + KERNEL_THRESHOLD:
+            m = bmax
+        m_at[b0:b0 + KERNEL_KBLOCK] = m
+    return np.exp2(u - M), np.exp2(M - m_at)
+
+
+def _check_full_fp8(x, scale, what, rows=None, peaked=False):
+    """Element-wise against the oracle, twice.
+
+    (1) The definition (oracle.varlen_attn_fp8: each probability p_j <= 1
+    rounded to e4m3 against its row's exact maximum, the denominator
+    unrounded). The kernel rounds each p against a running maximum that is
+    never above the row's; e4m3 puts both roundings within max(2^-4 p_j,
+    2^-10) of p_j (in units of the row's maximum), so each numerator term
+    differs by at most max(2^-3 p_j, 2^-9) |v~_j| and each output element by
+    at most the sum of those over the row's keys, divided by sum_j p_j. The
+    test allows that row's sum plus the attention tolerance.
+
+    (2) The kernel's own rounding schedule (oracle.varlen_attn_fp8_online with
+    128-key blocks and threshold 8): the attention tolerances (relative L2 <=
+    1e-2 over all elements; per element the max-abs bound, or on peaked
+    inputs the unit-scale bound) plus, per row, one e4m3 step of each key
+    whose probability lies within 2^-10 (relative) of an e4m3 rounding
+    midpoint: the kernel rounds fp32 probabilities and the oracle float64
+    ones, so only those keys can round differently."""
+    o, lse, v8, deq = _full_fp8_gpu(x, scale)
+    T, H, D = x["q"].shape
+    sel = np.arange(T) if rows is None else rows
+    rd, rld, rdeq = oracle.varlen_attn_fp8(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, rows=rows)
+    rs, rls, _ = oracle.varlen_attn_fp8_online(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, kblock=KERNEL_KBLOCK,
+                                               threshold=KERNEL_THRESHOLD, rows=rows)
+    assert np.array_equal(deq.cpu().numpy(), rdeq)
+    g = bf16_to_f64(o)[sel]
+    assert rel_l2(g, rs) <= ATTN_REL_L2, f"{what}: rel-L2 {rel_l2(g, rs):.3e} against the kernel's schedule"
+    qd, kd, vd = (_decode(c) * dq[None, :, None]
+                  for c, dq in (oracle.quantize_e4m3(x[n]) for n in ("q", "k", "v")))
     cu = x["cu_seqlens"]
     for n, t in enumerate(sel):
         i = int(np.searchsorted(cu, t, side="right") - 1)
         lo, hi = int(cu[i]), int(cu[i + 1])
         for h in range(H):
-            s = scale * (kd[lo:hi, h] @ qd[t, h])
-            wmax = float(np.exp(s - s.max()).max() / np.exp(s - s.max()).sum())
-            err = float(np.max(np.abs(g[n, h] - ro[n, h])))
-            assert err <= 2e-2 + 2.0 ** -3 * wmax * vmax, f"{what}: row {t} head {h} error {err:.3e}"
-    assert max_abs(lse.cpu().numpy().astype(np.float64).T[sel], rl) <= LSE_MAX_ABS
+            p, c = _row_terms(qd, kd, scale, lo, hi, t, h)
+            l = p.sum()
+            av = np.abs(vd[lo:hi, h])
+            # (1) the definition
+            bound = ATTN_MAX_ABS + (np.maximum(2.0 ** -3 * p, 2.0 ** -9)[:, None] * av).sum(0) / l
+            err = np.abs(g[n, h] - rd[n, h])
+            assert np.all(err <= bound), f"{what}: row {t} head {h}: {err.max():.3e} over the definition's bound"
+            # (2) the schedule: keys near a rounding midpoint, in the frame the kernel rounds in
+            ps = p * c
+            qn = _e4m3_quantum(ps)
+            frac = ps / qn - np.floor(ps / qn)
+            near = np.abs(frac - 0.5) * qn <= 2.0 ** -10 * ps
+            slack = (near[:, None] * (qn / c)[:, None] * av).sum(0) / l
+            err = np.abs(g[n, h] - rs[n, h])
+            tol = ELEM_UNIT_MAX * np.maximum(1.0, np.abs(rs[n, h])) if peaked else ATTN_MAX_ABS
+            assert np.all(err <= tol + slack), f"{what}: row {t} head {h}: {err.max():.3e} against the schedule"
+    assert max_abs(lse.cpu().numpy().astype(np.float64).T[sel], rls) <= LSE_MAX_ABS
+    assert max_abs(rls, rld) <= 1e-9  # the lse does not depend on P's rounding
 
 
 def test_v_quantisation_is_bitwise_the_oracle():
@@ -241,7 +299,7 @@ def test_full_fp8_attention_peaked():
     w = wl.custom([700, 1300], 2, 128, seed=44)
     x = wl.attention_inputs(w)
     x["q"] = wl.f32_to_bf16_bits(wl.bf16_bits_to_f32(x["q"]) * np.float32(8.0))
-    _check_full_fp8(x, 1.0 / math.sqrt(128), "full fp8 peaked")
+    _check_full_fp8(x, 1.0 / math.sqrt(128), "full fp8 peaked", peaked=True)
 
 
 def test_full_fp8_attention_16k_sampled_and_error_against_bf16():
