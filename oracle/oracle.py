@@ -61,11 +61,13 @@ def load(path: str):
     L.oracle_varlen_attn_fp8qk.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
                                            C.c_int, C.c_double, C.c_double, C.c_int, C.c_int, C.c_int, i32p,
                                            C.c_int64, f64p, f64p, C.POINTER(C.c_int64), u8p, u8p, f32p]
+    skip_args = [C.c_double, C.c_int, C.c_int, C.c_int]  # tau, query rows, keys, tile rows
     L.oracle_varlen_attn_fp8.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
-                                         C.c_int, C.c_double, i32p, C.c_int64, f64p, f64p, f32p]
+                                         C.c_int, C.c_double, *skip_args, i32p, C.c_int64, f64p, f64p,
+                                         C.POINTER(C.c_int64), f32p]
     L.oracle_varlen_attn_fp8_online.argtypes = [vp, vp, vp, C.c_int, C.c_int64, i32p, C.c_int, C.c_int64, C.c_int,
-                                                C.c_int, C.c_double, C.c_int, C.c_double, i32p, C.c_int64, f64p,
-                                                f64p, f32p]
+                                                C.c_int, C.c_double, C.c_int, C.c_double, *skip_args, i32p,
+                                                C.c_int64, f64p, f64p, C.POINTER(C.c_int64), f32p]
     L.oracle_linear_gated_residual.argtypes = [vp, C.c_int64, vp, vp, C.c_int, f32p, i32p, C.c_int, C.c_int64,
                                                C.c_int, C.c_int, i32p, C.c_int64, f64p]
     L.oracle_linear_swiglu.argtypes = [vp, C.c_int64, vp, C.c_int, C.c_int64, C.c_int, C.c_int, i32p, C.c_int64,
@@ -251,12 +253,7 @@ def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: n
     assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
     q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
-    if math.isinf(tau) and tau > 0:
-        qrows, kblock, tile_rows = 1, 1, 1
-    else:
-        if skip_block is None or skip_tile_rows is None:
-            raise ValueError("a finite tau needs the block geometry (skip_block, skip_tile_rows)")
-        (qrows, kblock), tile_rows = (int(b) for b in skip_block), int(skip_tile_rows)
+    tau, qrows, kblock, tile_rows = _skip_geometry(tau, skip_block, skip_tile_rows)
     r, n = _rows(rows)
     n = n if r is not None else T
     o = np.empty((n, H, D), np.float64)
@@ -266,7 +263,7 @@ def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: n
     deq = np.empty(2 * H, np.float32)
     counts = np.zeros(2, np.int64)
     rc = lib().oracle_varlen_attn_fp8qk(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32),
-                                        int(cu.shape[0]) - 1, T, H, D, scale, float(tau), qrows, kblock, tile_rows,
+                                        int(cu.shape[0]) - 1, T, H, D, scale, tau, qrows, kblock, tile_rows,
                                         _ptr(r, C.c_int32), n if r is not None else 0, _ptr(o, C.c_double),
                                         _ptr(lse, C.c_double), _ptr(counts, C.c_int64), _ptr(q8, C.c_uint8),
                                         _ptr(k8, C.c_uint8), _ptr(deq, C.c_float))
@@ -277,7 +274,18 @@ def varlen_attn_fp8qk(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: n
     return o, lse, q8, k8, deq
 
 
-def _fp8_call(fn, name, q, k, v, cu_seqlens, scale, rows, want_lse, extra):
+def _skip_geometry(tau, skip_block, skip_tile_rows):
+    """(tau, query rows, keys, tile rows) for the C calls; the geometry is
+    unused (and not needed) for an infinite tau."""
+    if math.isinf(tau) and tau > 0:
+        return float(tau), 1, 1, 1
+    if skip_block is None or skip_tile_rows is None:
+        raise ValueError("a finite tau needs the block geometry (skip_block, skip_tile_rows)")
+    qrows, kblock = (int(b) for b in skip_block)
+    return float(tau), qrows, kblock, int(skip_tile_rows)
+
+
+def _fp8_call(fn, name, q, k, v, cu_seqlens, scale, rows, want_lse, extra, skip, counts_out):
     T, H, D = q.shape
     assert k.shape == q.shape == v.shape and q.dtype == k.dtype == v.dtype
     q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
@@ -287,31 +295,41 @@ def _fp8_call(fn, name, q, k, v, cu_seqlens, scale, rows, want_lse, extra):
     o = np.empty((n, H, D), np.float64)
     lse = np.empty((n, H), np.float64) if want_lse else None
     deq = np.empty(3 * H, np.float32)
+    counts = np.zeros(2, np.int64)
     rc = fn(_ptr(q), _ptr(k), _ptr(v), _kind(q), H * D, _ptr(cu, C.c_int32), int(cu.shape[0]) - 1, T, H, D, scale,
-            *extra, _ptr(r, C.c_int32), n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
-            _ptr(deq, C.c_float))
+            *extra, *skip, _ptr(r, C.c_int32), n if r is not None else 0, _ptr(o, C.c_double), _ptr(lse, C.c_double),
+            _ptr(counts, C.c_int64), _ptr(deq, C.c_float))
     if rc:
         raise ValueError(f"{name}: invalid arguments")
+    if counts_out is not None and not (math.isinf(skip[0]) and skip[0] > 0):
+        counts_out.append(tuple(int(c) for c in counts))
     return o, lse, deq
 
 
 def varlen_attn_fp8(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, rows=None,
-                    want_lse: bool = True):
+                    want_lse: bool = True, tau: float = math.inf, skip_block=None, skip_tile_rows=None,
+                    counts_out: list | None = None):
     """Attention with Q, K, V and P in FP8 e4m3, P rounded against each row's
-    exact maximum (oracle_varlen_attn_fp8). Returns (o [nrows, H, D], lse
-    [nrows, H] or None, deq [3H])."""
+    exact maximum (oracle_varlen_attn_fp8); with a finite tau, key blocks are
+    skipped by the rule of varlen_attn_skip on the dequantised Q, K (geometry
+    skip_block = (query rows, keys), skip_tile_rows; the counts of all T rows
+    appended to counts_out). Returns (o [nrows, H, D], lse [nrows, H] or
+    None, deq [3H])."""
     return _fp8_call(lib().oracle_varlen_attn_fp8, "oracle_varlen_attn_fp8", q, k, v, cu_seqlens, scale, rows,
-                     want_lse, ())
+                     want_lse, (), _skip_geometry(tau, skip_block, skip_tile_rows), counts_out)
 
 
 def varlen_attn_fp8_online(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, scale: float, *,
-                           kblock: int, threshold: float, rows=None, want_lse: bool = True):
+                           kblock: int, threshold: float, rows=None, want_lse: bool = True, tau: float = math.inf,
+                           skip_block=None, skip_tile_rows=None, counts_out: list | None = None):
     """The same FP8 attention in the rounding order of an online softmax over
     blocks of kblock keys whose running maximum moves only past threshold
     (log2 units): a streaming implementation's schedule, not the definition
-    (oracle_varlen_attn_fp8_online). Returns (o, lse or None, deq [3H])."""
-    return _fp8_call(lib().oracle_varlen_attn_fp8_online, "oracle_varlen_attn_fp8_online", q, k, v, cu_seqlens, scale,
-                     rows, want_lse, (int(kblock), float(threshold)))
+    (oracle_varlen_attn_fp8_online). Block skipping as in varlen_attn_fp8.
+    Returns (o, lse or None, deq [3H])."""
+    return _fp8_call(lib().oracle_varlen_attn_fp8_online, "oracle_varlen_attn_fp8_online", q, k, v, cu_seqlens,
+                     scale, rows, want_lse, (int(kblock), float(threshold)),
+                     _skip_geometry(tau, skip_block, skip_tile_rows), counts_out)
 
 
 def modulate_swiglu(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, gate_res: np.ndarray,

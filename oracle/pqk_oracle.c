@@ -363,6 +363,10 @@ int oracle_varlen_attn_skip(const void* q, const void* k, const void* v, int in_
                             const int32_t* cu, int B, int64_t T, int H, int D, double scale, double tau,
                             int qrows, int kblock, int tile_rows, const int32_t* rows, int64_t nrows, double* o,
                             double* lse, int64_t* counts);
+static void skip_block_flags(const void* q, const void* k, int in_kind, int64_t stride_t, int64_t lo, int64_t n_keys,
+                             int64_t r0, int64_t r1, int h, int D, double scale, double tau, int kblock,
+                             unsigned char* keep);
+static int64_t skip_tile_count(const unsigned char* keep, int H, int64_t nqb, int64_t nkb, int64_t per_tile);
 
 /*
  * Attention with Q and K quantised to e4m3 per head (oracle_quantize_e4m3)
@@ -426,13 +430,19 @@ int oracle_varlen_attn_fp8qk(const void* q, const void* k, const void* v, int in
  * e4m3(p) is the code nearest to p taken as a float (oracle_e4m3_codes),
  * read back as its value. deq_out: [3H] (Q's, K's, V's dequantisation
  * factors), optional.
+ * With a finite tau the key blocks that the block-skipping rule of
+ * oracle_varlen_attn_skip drops (decided on the scores of Q~, K~ with the
+ * caller's geometry) are left out of every sum and of the maximum, and
+ * counts (nullable) receives that rule's two counts for all T rows.
  */
 static void fp8_row(const double* qd, const double* kd, const double* vd, int64_t lo, int64_t n_keys, int64_t t,
-                    int H, int h, int D, double scale, double* ot, double* lse_out) {
+                    int H, int h, int D, double scale, const unsigned char* keep, int kblock, double* ot,
+                    double* lse_out) {
   const double* qr = qd + (t * H + h) * (int64_t)D;
   double* s = (double*)malloc(sizeof(double) * (size_t)(n_keys > 0 ? n_keys : 1));
   double m = -INFINITY;
   for (int64_t j = 0; j < n_keys; ++j) {
+    if (keep && !keep[j / kblock]) continue;
     const double* kr = kd + ((lo + j) * H + h) * (int64_t)D;
     double dot = 0.0;
     for (int d = 0; d < D; ++d) dot += qr[d] * kr[d];
@@ -442,6 +452,7 @@ static void fp8_row(const double* qd, const double* kd, const double* vd, int64_
   double den = 0.0;
   for (int d = 0; d < D; ++d) ot[d] = 0.0;
   for (int64_t j = 0; j < n_keys; ++j) {
+    if (keep && !keep[j / kblock]) continue;
     const double pj = exp(s[j] - m);
     const double pq = e4m3_value(e4m3_code((float)pj));
     den += pj;
@@ -467,24 +478,25 @@ static void fp8_row(const double* qd, const double* kd, const double* vd, int64_
  *   - o = numerator / l and lse = (m + log2 l) ln 2.
  * With threshold = 0 and one block per request this is the definition; any
  * other schedule rounds each p against a smaller maximum, which changes each
- * numerator term by at most one e4m3 step.
+ * numerator term by at most one e4m3 step. With block skipping (a finite
+ * tau) dropped keys take no part: a block's maximum is over its kept keys.
  */
 static void fp8_row_online(const double* qd, const double* kd, const double* vd, int64_t lo, int64_t n_keys,
-                           int64_t t, int H, int h, int D, double scale, int kblock, double threshold, double* ot,
-                           double* lse_out) {
+                           int64_t t, int H, int h, int D, double scale, int kblock, double threshold,
+                           const unsigned char* keep, int skip_kblock, double* ot, double* lse_out) {
   const double* qr = qd + (t * H + h) * (int64_t)D;
   double* num = (double*)calloc((size_t)D, sizeof(double));
   double* ublock = (double*)malloc(sizeof(double) * (size_t)kblock);
   double mrun = -INFINITY, den = 0.0;
   for (int64_t b0 = 0; b0 < n_keys; b0 += kblock) {
     const int64_t b1 = b0 + kblock < n_keys ? b0 + kblock : n_keys;
-    double bmax = -INFINITY;
+    double bmax = -INFINITY;  /* over the block's kept keys */
     for (int64_t j = b0; j < b1; ++j) {
       const double* kr = kd + ((lo + j) * H + h) * (int64_t)D;
       double dot = 0.0;
       for (int d = 0; d < D; ++d) dot += qr[d] * kr[d];
       ublock[j - b0] = scale * dot / log(2.0);
-      if (ublock[j - b0] > bmax) bmax = ublock[j - b0];
+      if ((!keep || keep[j / skip_kblock]) && ublock[j - b0] > bmax) bmax = ublock[j - b0];
     }
     if (b0 == 0) {
       mrun = bmax;
@@ -495,6 +507,7 @@ static void fp8_row_online(const double* qd, const double* kd, const double* vd,
       mrun = bmax;
     }
     for (int64_t j = b0; j < b1; ++j) {
+      if (keep && !keep[j / skip_kblock]) continue;
       const double pj = exp2(ublock[j - b0] - mrun);
       const double pq = e4m3_value(e4m3_code((float)pj));
       den += pj;
@@ -509,13 +522,18 @@ static void fp8_row_online(const double* qd, const double* kd, const double* vd,
 }
 
 /* Both FP8 attentions: online == 0 the definition, else the online schedule
- * with (kblock, threshold). */
+ * with (kblock, threshold); a finite tau adds block skipping with the
+ * geometry (skip_qrows, skip_kblock, skip_tile_rows). */
 static int fp8_attention(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
                          const int32_t* cu, int B, int64_t T, int H, int D, double scale, int online, int kblock,
-                         double threshold, const int32_t* rows, int64_t nrows, double* o, double* lse,
+                         double threshold, double tau, int skip_qrows, int skip_kblock, int skip_tile_rows,
+                         const int32_t* rows, int64_t nrows, double* o, double* lse, int64_t* counts,
                          float* deq_out) {
-  if (check_cu(cu, B, T) || H <= 0 || D <= 0) return -1;
+  if (check_cu(cu, B, T) || H <= 0 || D <= 0 || isnan(tau)) return -1;
   if (online && (kblock <= 0 || !(threshold >= 0.0))) return -1;
+  const int skipping = !(isinf(tau) && tau > 0);
+  if (skipping && (skip_qrows <= 0 || skip_kblock <= 0 || skip_tile_rows <= 0 || skip_tile_rows % skip_qrows))
+    return -1;
   const int64_t n = T * (int64_t)H * D;
   uint8_t* c8 = (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
   float* dq = (float*)malloc(sizeof(float) * (size_t)H * 3);
@@ -530,6 +548,34 @@ static int fp8_attention(const void* q, const void* k, const void* v, int in_kin
       for (int64_t e = 0; e < n; ++e) xd[i][e] = e4m3_value(c8[e]) * (double)dq[(int64_t)i * H + (e / D) % H];
     }
   }
+  /* skip decisions per (request, head, query block), on the dequantised Q, K */
+  unsigned char** keep = NULL;
+  if (!rc && skipping) {
+    keep = (unsigned char**)calloc((size_t)(B > 0 ? B : 1), sizeof(unsigned char*));
+    int64_t n_block = 0, n_tile = 0;
+    for (int seg = 0; seg < B; ++seg) {
+      const int64_t lo = cu[seg], n_keys = (int64_t)cu[seg + 1] - cu[seg];
+      if (n_keys == 0) continue;
+      const int64_t nqb = (n_keys + skip_qrows - 1) / skip_qrows, nkb = (n_keys + skip_kblock - 1) / skip_kblock;
+      keep[seg] = (unsigned char*)malloc((size_t)(H * nqb * nkb));
+#pragma omp parallel for schedule(dynamic, 1) collapse(2) reduction(+ : n_block)
+      for (int64_t b = 0; b < nqb; ++b) {
+        for (int h = 0; h < H; ++h) {
+          const int64_t r0 = lo + b * skip_qrows;
+          const int64_t r1 = r0 + skip_qrows < lo + n_keys ? r0 + skip_qrows : lo + n_keys;
+          unsigned char* kp = keep[seg] + ((int64_t)h * nqb + b) * nkb;
+          skip_block_flags(xd[0], xd[1], ORACLE_IN_F64, (int64_t)H * D, lo, n_keys, r0, r1, h, D, scale, tau,
+                           skip_kblock, kp);
+          for (int64_t jb = 0; jb < nkb; ++jb) n_block += !kp[jb];
+        }
+      }
+      n_tile += skip_tile_count(keep[seg], H, nqb, nkb, skip_tile_rows / skip_qrows);
+    }
+    if (counts) {
+      counts[0] = n_block;
+      counts[1] = n_tile;
+    }
+  }
   if (!rc) {
     const int64_t nr = rows ? nrows : T;
     int64_t bad = 0;
@@ -540,15 +586,25 @@ static int fp8_attention(const void* q, const void* k, const void* v, int in_kin
         const int seg = (t >= 0 && t < T) ? segment_of(cu, B, t) : -1;
         if (seg < 0) { ++bad; continue; }
         const int64_t lo = cu[seg], n_keys = (int64_t)cu[seg + 1] - cu[seg];
+        const unsigned char* kp = NULL;
+        if (keep) {
+          const int64_t nqb = (n_keys + skip_qrows - 1) / skip_qrows, nkb = (n_keys + skip_kblock - 1) / skip_kblock;
+          kp = keep[seg] + ((int64_t)h * nqb + (t - lo) / skip_qrows) * nkb;
+        }
         double* ot = o + (r * H + h) * (int64_t)D;
         double* lt = lse ? &lse[r * H + h] : NULL;
         if (online)
-          fp8_row_online(xd[0], xd[1], xd[2], lo, n_keys, t, H, h, D, scale, kblock, threshold, ot, lt);
+          fp8_row_online(xd[0], xd[1], xd[2], lo, n_keys, t, H, h, D, scale, kblock, threshold, kp, skip_kblock, ot,
+                         lt);
         else
-          fp8_row(xd[0], xd[1], xd[2], lo, n_keys, t, H, h, D, scale, ot, lt);
+          fp8_row(xd[0], xd[1], xd[2], lo, n_keys, t, H, h, D, scale, kp, skip_kblock, ot, lt);
       }
     }
     if (bad) rc = -1;
+  }
+  if (keep) {
+    for (int seg = 0; seg < B; ++seg) free(keep[seg]);
+    free(keep);
   }
   if (deq_out) memcpy(deq_out, dq, sizeof(float) * (size_t)H * 3);
   for (int i = 0; i < 3; ++i) free(xd[i]);
@@ -558,17 +614,20 @@ static int fp8_attention(const void* q, const void* k, const void* v, int in_kin
 }
 
 int oracle_varlen_attn_fp8(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
-                           const int32_t* cu, int B, int64_t T, int H, int D, double scale, const int32_t* rows,
-                           int64_t nrows, double* o, double* lse, float* deq_out) {
-  return fp8_attention(q, k, v, in_kind, stride_t, cu, B, T, H, D, scale, 0, 0, 0.0, rows, nrows, o, lse, deq_out);
+                           const int32_t* cu, int B, int64_t T, int H, int D, double scale, double tau, int qrows,
+                           int kblock, int tile_rows, const int32_t* rows, int64_t nrows, double* o, double* lse,
+                           int64_t* counts, float* deq_out) {
+  return fp8_attention(q, k, v, in_kind, stride_t, cu, B, T, H, D, scale, 0, 0, 0.0, tau, qrows, kblock, tile_rows,
+                       rows, nrows, o, lse, counts, deq_out);
 }
 
 int oracle_varlen_attn_fp8_online(const void* q, const void* k, const void* v, int in_kind, int64_t stride_t,
                                   const int32_t* cu, int B, int64_t T, int H, int D, double scale, int kblock,
-                                  double threshold, const int32_t* rows, int64_t nrows, double* o, double* lse,
+                                  double threshold, double tau, int qrows, int skip_kblock, int tile_rows,
+                                  const int32_t* rows, int64_t nrows, double* o, double* lse, int64_t* counts,
                                   float* deq_out) {
-  return fp8_attention(q, k, v, in_kind, stride_t, cu, B, T, H, D, scale, 1, kblock, threshold, rows, nrows, o, lse,
-                       deq_out);
+  return fp8_attention(q, k, v, in_kind, stride_t, cu, B, T, H, D, scale, 1, kblock, threshold, tau, qrows,
+                       skip_kblock, tile_rows, rows, nrows, o, lse, counts, deq_out);
 }
 
 /* e4m3 codes of a float32 array (the conversion alone, for its pins). */
@@ -602,6 +661,22 @@ void oracle_e4m3_codes(const float* x, int64_t n, uint8_t* codes) {
  * request's first token) that skips a key block when all of its query blocks
  * inside the request do.
  */
+
+/* Number of (tile, head, key block) triples in which every query block of
+ * the tile (per_tile consecutive query blocks of one request) drops the key
+ * block. keep: [H][nqb][nkb] flags of one request. */
+static int64_t skip_tile_count(const unsigned char* keep, int H, int64_t nqb, int64_t nkb, int64_t per_tile) {
+  int64_t n_tile = 0;
+  for (int h = 0; h < H; ++h)
+    for (int64_t tb = 0; tb * per_tile < nqb; ++tb)
+      for (int64_t jb = 0; jb < nkb; ++jb) {
+        int all = 1;
+        for (int64_t b = tb * per_tile; b < (tb + 1) * per_tile && b < nqb; ++b)
+          if (keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;
+        n_tile += all;
+      }
+  return n_tile;
+}
 
 /* Keep flags of the key blocks of query block [r0, r1) (rows of one request
  * starting at lo, n_keys keys), head h. keep: [ceil(n_keys / kblock)]. */
@@ -717,15 +792,7 @@ int oracle_varlen_attn_skip(const void* q, const void* k, const void* v, int in_
       }
     }
     /* a tile skips key block jb when each of its query blocks inside the request does */
-    const int64_t per_tile = tile_rows / qrows;
-    for (int h = 0; h < H; ++h)
-      for (int64_t tb = 0; tb * per_tile < nqb; ++tb)
-        for (int64_t jb = 0; jb < nkb; ++jb) {
-          int all = 1;
-          for (int64_t b = tb * per_tile; b < (tb + 1) * per_tile && b < nqb; ++b)
-            if (keep[((int64_t)h * nqb + b) * nkb + jb]) all = 0;
-          n_tile += all;
-        }
+    n_tile += skip_tile_count(keep, H, nqb, nkb, tile_rows / qrows);
     free(keep);
   }
   if (counts) {

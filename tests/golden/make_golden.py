@@ -34,9 +34,10 @@ def variants(w, p, a):
     200-token request laid out as a 2 x 10 x 10 grid, sections 8 / 12 / 12),
     the full-width norm, block skipping at tau = 4 on block-scaled inputs
     (blocks of 16 query rows x 64 keys, tiles of 64 rows), attention with FP8
-    Q, K and with FP8 Q, K, V, P (the definition, and the online schedule with
-    blocks of 64 keys and threshold 4), and the three linear layers with their
-    fused epilogues."""
+    Q, K and with FP8 Q, K, V, P (the definition, the online schedule with
+    blocks of 64 keys and threshold 4, and the definition with block skipping
+    at tau = 4 on the block-scaled inputs), and the three linear layers with
+    their fused epilogues."""
     out = {}
     scale = 1.0 / math.sqrt(w.D)
     y = oracle.qk_norm_rope_3axis(p["q"], p["w_q"], w.positions3(video_grid=(2, 10, 10)), (8, 12, 12), w.eps,
@@ -59,6 +60,11 @@ def variants(w, p, a):
                                                 threshold=4.0)
     out["attn_fp8_online_64_4"] = {"summary": summarise(o), "lse_summary": summarise(lse), "deq": deq.tolist(),
                                    "head0": [o[r, 0, :8].tolist() for r in ROWS]}
+    counts = []
+    o, lse, deq = oracle.varlen_attn_fp8(b["q"], b["k"], b["v"], b["cu_seqlens"], scale, tau=4.0, skip_block=(16, 64),
+                                         skip_tile_rows=64, counts_out=counts)
+    out["attn_fp8_skip_tau4"] = {"summary": summarise(o), "lse_summary": summarise(lse), "counts": list(counts[0]),
+                                 "head0": [o[r, 0, :8].tolist() for r in ROWS]}
     for name in ("o_proj", "w1", "w2"):
         d = wl.linear_inputs(w, name)
         if name == "w1":

@@ -337,3 +337,109 @@ def test_online_schedule_arguments_are_validated():
     for kb, th in [(0, 8.0), (128, -1.0), (128, float("nan"))]:
         with pytest.raises(ValueError):
             oracle.varlen_attn_fp8_online(x, x, x, cu, 1.0, kblock=kb, threshold=th)
+
+
+# ----------------------------------------------- FP8 P with block skipping (Skip-Softmax)
+
+def _skip_case(kb, qr, seed=0):
+    """One request of four key blocks of kb keys, one head, D = 16: queries
+    close to +a*u, keys of blocks 0 and 2 close to -a*u (block 2 is dropped,
+    block 0 never is), except query row qr + 5, which points at -u, so its
+    query block keeps block 2. Dimension 15 is zero everywhere but in token
+    0, which holds every tensor's absolute maximum there: removing block 2's
+    tokens leaves all three quantisation scales unchanged."""
+    L, D, a = 4 * kb, 16, 6.0
+    g = np.random.default_rng(seed)
+    u = np.zeros(D)
+    u[0] = 1.0
+    q = a * u + 0.1 * g.standard_normal((L, D))
+    k = 0.3 * g.standard_normal((L, D))
+    k[2 * kb:3 * kb] -= a * u
+    k[0:kb] -= a * u
+    q[qr + 5] = -a * u + 0.1 * g.standard_normal(D)
+    v = g.standard_normal((L, D))
+    for x in (q, k, v):
+        x[:, 15] = 0.0
+        x[0, 15] = 20.0
+    return q[:, None, :], k[:, None, :], v[:, None, :], np.array([0, L], np.int32), 1.0 / math.sqrt(D)
+
+
+@pytest.mark.parametrize("geom", [(16, 64, 64), (32, 128, 128)])
+def test_fp8_skipping_is_the_definition_over_the_kept_keys(geom):
+    # rows whose query block drops key block 2 equal the FP8 attention of the
+    # same sequence with block 2's tokens removed; rows of the query block
+    # that keeps it equal the FP8 attention of the whole sequence; the counts
+    # are the forced ones, and the same as the FP8 Q K^T composition's
+    qr, kb, tile = geom
+    q, k, v, cu, scale = _skip_case(kb, qr)
+    L = q.shape[0]
+    counts = []
+    o, lse, _ = oracle.varlen_attn_fp8(q, k, v, cu, scale, tau=10.0, skip_block=(qr, kb), skip_tile_rows=tile,
+                                       counts_out=counts)
+    assert counts == [(L // qr - 1, math.ceil(L / tile) - 1)]
+    qk_counts = []
+    oracle.varlen_attn_fp8qk(q, k, v, cu, scale, tau=10.0, skip_block=(qr, kb), skip_tile_rows=tile,
+                             counts_out=qk_counts)
+    assert qk_counts == counts
+    full, full_lse, _ = oracle.varlen_attn_fp8(q, k, v, cu, scale)
+    keep = np.r_[0:2 * kb, 3 * kb:L]
+    red, red_lse, _ = oracle.varlen_attn_fp8(q[keep], k[keep], v[keep], np.array([0, len(keep)], np.int32), scale)
+    pos_in_red = {int(t): i for i, t in enumerate(keep)}
+    for t in range(L):
+        if qr <= t < 2 * qr:
+            ref, ref_lse = full[t], full_lse[t]
+        elif t in pos_in_red:
+            ref, ref_lse = red[pos_in_red[t]], red_lse[pos_in_red[t]]
+        else:
+            continue  # a row of block 2 itself: its own request has no reduced counterpart
+        np.testing.assert_allclose(o[t], ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[t], ref_lse, rtol=0, atol=1e-12)
+    # row qr + 5 attends mostly to block 2: dropping it would change its output
+    assert np.max(np.abs(full[qr + 5] - red[pos_in_red[qr + 5]])) > 1e-3
+
+
+@pytest.mark.parametrize("geom", [(16, 64, 64), (32, 128, 128)])
+def test_fp8_online_skipping_is_the_online_schedule_over_the_kept_keys(geom):
+    # the online schedule with blocks of kb keys: dropping the whole block 2
+    # leaves the same blocks as removing its tokens
+    qr, kb, tile = geom
+    q, k, v, cu, scale = _skip_case(kb, qr, seed=1)
+    L = q.shape[0]
+    counts = []
+    o, lse, _ = oracle.varlen_attn_fp8_online(q, k, v, cu, scale, kblock=kb, threshold=8.0, tau=10.0,
+                                              skip_block=(qr, kb), skip_tile_rows=tile, counts_out=counts)
+    assert counts == [(L // qr - 1, math.ceil(L / tile) - 1)]
+    full, _, _ = oracle.varlen_attn_fp8_online(q, k, v, cu, scale, kblock=kb, threshold=8.0)
+    keep = np.r_[0:2 * kb, 3 * kb:L]
+    red, _, _ = oracle.varlen_attn_fp8_online(q[keep], k[keep], v[keep], np.array([0, len(keep)], np.int32), scale,
+                                              kblock=kb, threshold=8.0)
+    pos_in_red = {int(t): i for i, t in enumerate(keep)}
+    for t in range(L):
+        if qr <= t < 2 * qr:
+            np.testing.assert_allclose(o[t], full[t], rtol=0, atol=1e-12)
+        elif t in pos_in_red:
+            np.testing.assert_allclose(o[t], red[pos_in_red[t]], rtol=0, atol=1e-12)
+
+
+def test_fp8_huge_threshold_skips_nothing():
+    g = np.random.default_rng(14)
+    T, H, D = 700, 2, 32
+    q, k, v = (g.standard_normal((T, H, D)) * 2 for _ in range(3))
+    cu = np.array([0, 300, 300, 700], np.int32)
+    for fn, kw in ((oracle.varlen_attn_fp8, {}), (oracle.varlen_attn_fp8_online, {"kblock": 128, "threshold": 8.0})):
+        counts = []
+        o, lse, _ = fn(q, k, v, cu, 0.2, tau=1e30, skip_block=(32, 128), skip_tile_rows=128, counts_out=counts, **kw)
+        o0, l0, _ = fn(q, k, v, cu, 0.2, **kw)
+        assert counts == [(0, 0)]
+        assert np.array_equal(o, o0) and np.array_equal(lse, l0)
+    with pytest.raises(ValueError):
+        oracle.varlen_attn_fp8(q, k, v, cu, 0.2, tau=4.0)  # a finite tau needs the block geometry
+
+
+def test_fp8_skipping_sampled_rows_equal_full_evaluation():
+    q, k, v, cu, scale = _skip_case(64, 16, seed=2)
+    o, lse, _ = oracle.varlen_attn_fp8(q, k, v, cu, scale, tau=10.0, skip_block=(16, 64), skip_tile_rows=64)
+    rows = np.array([0, 15, 16, 21, 31, 32, 150, 255], np.int32)
+    o2, l2, _ = oracle.varlen_attn_fp8(q, k, v, cu, scale, tau=10.0, skip_block=(16, 64), skip_tile_rows=64,
+                                       rows=rows)
+    assert np.array_equal(o2, o[rows]) and np.array_equal(l2, lse[rows])

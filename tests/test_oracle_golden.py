@@ -74,6 +74,13 @@ def test_oracle_variants_match_stored_tiny_config_outputs():
         _summary_close(o, g[key]["summary"])
         _summary_close(lse, g[key]["lse_summary"])
         np.testing.assert_allclose([o[r, 0, :8] for r in rows], g[key]["head0"], atol=1e-12)
+    counts = []
+    o, lse, _ = oracle.varlen_attn_fp8(b["q"], b["k"], b["v"], b["cu_seqlens"], scale, tau=4.0, skip_block=(16, 64),
+                                       skip_tile_rows=64, counts_out=counts)
+    assert list(counts[0]) == g["attn_fp8_skip_tau4"]["counts"]
+    _summary_close(o, g["attn_fp8_skip_tau4"]["summary"])
+    _summary_close(lse, g["attn_fp8_skip_tau4"]["lse_summary"])
+    np.testing.assert_allclose([o[r, 0, :8] for r in rows], g["attn_fp8_skip_tau4"]["head0"], atol=1e-12)
     for name in ("o_proj", "w1", "w2"):
         d = wl.linear_inputs(w, name)
         if name == "w1":

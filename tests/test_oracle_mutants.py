@@ -76,6 +76,8 @@ MUTANTS = {
                                    "\n      const double pq = pj;"),
     "fp8_online_denominator_quantised": ("\n      den += pj;\n", "\n      den += pq;\n"),
     "fp8_online_numerator_not_rescaled": ("      for (int d = 0; d < D; ++d) num[d] *= alpha;\n", ""),
+    "fp8_skip_dropped_keys_summed": ("    if (keep && !keep[j / kblock]) continue;\n    const double pj", "    const double pj"),
+    "fp8_online_dropped_keys_summed": ("      if (keep && !keep[j / skip_kblock]) continue;\n", ""),
     "linear_w_transposed": ("load(w, in_kind, (int64_t)n * K + k)", "load(w, in_kind, (int64_t)k * N + n)"),
     "linear_gate_of_first_request": ("(double)gate_res[(int64_t)seg * N + n] * y", "(double)gate_res[n] * y"),
     "linear_residual_sign": ("load(x, in_kind, t * N + n) + (double)gate_res", "load(x, in_kind, t * N + n) - (double)gate_res"),
