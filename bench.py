@@ -23,7 +23,10 @@ vs skipping vs FP8 Q K^T with and without skipping); the FP8 Q K^T attention
 on the step's inputs (``--no-fp8`` leaves it out); the block's three linear
 layers with the gated residual or SwiGLU in the GEMM epilogue, on the step's
 own activations, against cuBLAS plus torch epilogues (``linear_epilogue``;
-``--no-linear`` leaves it out); and, with ``--graph``,
+``--no-linear`` leaves it out); the two HBM-bound kernels on the 40-head
+bandwidth-sweep shapes at 4,096 and 58,048 tokens with an L2 flush between
+launches (``bandwidth_sweep_40_heads``; ``--no-bw-sweep`` leaves it out); and,
+with ``--graph``,
 the step replayed as a CUDA graph (``graph_ms_per_step``). ``--config N``
 selects another configuration, ``--sweep`` the HBM bandwidth sweep,
 ``--linear-sweep`` the fused-epilogue linear layers on a range of shapes.
@@ -77,6 +80,8 @@ def parse():
                          "widths (one JSON line per shape) instead of the step")
     ap.add_argument("--no-linear", action="store_true",
                     help="leave out the linear layers with the fused epilogues (gated residual, SwiGLU)")
+    ap.add_argument("--no-bw-sweep", action="store_true",
+                    help="leave out the HBM-bound kernels on the 40-head sweep shapes at 4,096 and 58,048 tokens")
     ap.add_argument("--graph", action="store_true",
                     help="also time the block call captured once in a CUDA graph and replayed (graph_ms_per_step)")
     ap.add_argument("--skip-tau", type=float, default=8.0,
@@ -292,6 +297,78 @@ def time_linear_layers(w, d, o, pk, pk_kind, reps=3):
                 "weights": "random-init N(0, 1/in) bf16"})
     del w_o, w1, w2, out_c, out_f
     return res
+
+
+def time_bandwidth_sweep(w_step, dev, pk, pk_kind, tokens=(4096, 58048), reps=10):
+    """The two HBM-bound kernels on the 40-head bandwidth-sweep shapes (Q, K
+    [T, 40, 128]; modulation + SwiGLU with hidden 5,120 and FFN 13,824, no
+    residual branch) at the given token counts: one launch at a time, a
+    256 MB write between launches to flush L2 (the 4,096-token working set is
+    close to its 126 MB), followed by a 256 MB read that evicts the written
+    lines (their write-back would otherwise compete with the kernel), median
+    of ``reps`` launches after two warm-up ones.
+    Inputs are drawn on the device with the sweep's distributions (torch's
+    CUDA generator, seeded per token count) to keep the multi-GB tensors off
+    the host; the kernels' time does not depend on the values."""
+    import torch
+    from packed_attention_qk_b200 import pqk
+    from packed_attention_qk_b200 import workloads as wl
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clean = torch.ones(64 << 20, dtype=torch.int32, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def timed(fn):
+        ts = []
+        for i in range(2 + reps):
+            # write 256 MB (more than the L2), then read another 256 MB so that
+            # the written lines are evicted before the kernel starts rather
+            # than written back while it runs
+            flush.fill_(i & 0xFF)
+            clean.sum()
+            ev[0].record()
+            fn()
+            ev[1].record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                ts.append(ev[0].elapsed_time(ev[1]))
+        return statistics.median(ts)
+
+    out = {}
+    for T in tokens:
+        w = wl.config(5, T)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(w.seed * 1000003 + T)
+        bf = lambda *shape: torch.randn(*shape, generator=gen, device=dev).to(torch.bfloat16)
+        q, k = bf(T, w.H, w.D), bf(T, w.H, w.D)
+        wq = (torch.rand(w.D, generator=gen, device=dev) + 0.5).to(torch.bfloat16)
+        wk = (torch.rand(w.D, generator=gen, device=dev) + 0.5).to(torch.bfloat16)
+        pos = torch.arange(T, dtype=torch.int32, device=dev)
+        qo, ko = torch.empty_like(q), torch.empty_like(k)
+        pro_ms = timed(lambda: pqk.qk_norm_rope(q, k, wq, wk, pos, eps=w.eps, rope_base=w.rope_base, q_out=qo,
+                                                k_out=ko))
+        del q, k, qo, ko
+        x = bf(T, w.C)
+        gate, up = bf(T, w.F), bf(T, w.F)
+        shift = torch.randn(1, w.C, generator=gen, device=dev) * 0.1
+        scale = torch.randn(1, w.C, generator=gen, device=dev) * 0.1
+        cu = torch.tensor([0, T], dtype=torch.int32, device=dev)
+        h, act = torch.empty_like(x), torch.empty_like(gate)
+        epi_ms = timed(lambda: pqk.modulate_swiglu(x, shift, scale, cu, gate=gate, up=up, eps=w.eps, h=h, act=act))
+        del x, gate, up, h, act
+        if pqk.get_device_status() != 0:
+            raise RuntimeError("device status set during the bandwidth sweep")
+        pro_gbs = w.prologue_bytes() / (pro_ms * 1e-3) / 1e9
+        epi_gbs = w.epilogue_bytes() / (epi_ms * 1e-3) / 1e9
+        out[str(T)] = {"qk_norm_rope_us": pro_ms * 1e3, "qk_norm_rope_gbs": pro_gbs,
+                       "qk_norm_rope_frac_hbm": pro_gbs / pk["hbm_gbs"],
+                       "modulate_swiglu_us": epi_ms * 1e3, "modulate_swiglu_gbs": epi_gbs,
+                       "modulate_swiglu_frac_hbm": epi_gbs / pk["hbm_gbs"]}
+    del flush, clean
+    torch.cuda.empty_cache()
+    out["shapes"] = "qk_norm_rope: Q, K [T, 40, 128]; modulate_swiglu: hidden 5,120, FFN 13,824, no branch"
+    out["peak"] = f"{pk_kind} HBM {pk['hbm_gbs']:.1f} GB/s"
+    out["l2"] = "between launches 256 MB written, then another 256 MB read (the L2 holds no dirty lines at the start)"
+    return out
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -601,6 +678,9 @@ def run_ours(args, w):
     if not args.no_linear and w.H * w.D == w.C:
         lin = time_linear_layers(w, d, o, pk, pk_kind)
 
+    # the HBM half of the metric on the bandwidth-sweep shapes (40 heads)
+    bw = None if args.no_bw_sweep else time_bandwidth_sweep(w, dev, pk, pk_kind)
+
     # e2e through host buffers: every step copies all of its inputs from
     # pinned host memory to the device (H2D stream), runs the three C-ABI
     # calls (compute stream) and copies its outputs x', h, act back to pinned
@@ -701,7 +781,8 @@ def run_ours(args, w):
                     "qk_norm_rope_back_to_back_us": rope1_b2b_us,
                     "qk_fullc_norm_rope_us": fullc_us, "qk_fullc_norm_rope_gbs": fullc_gbs,
                     "qk_fullc_norm_rope_frac_hbm": fullc_gbs / pk["hbm_gbs"],
-                    "varlen_attn_skip": skip, "varlen_attn_fp8qk": fp8, "linear_epilogue": lin},
+                    "varlen_attn_skip": skip, "varlen_attn_fp8qk": fp8, "linear_epilogue": lin,
+                    "bandwidth_sweep_40_heads": bw},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * K,
@@ -747,12 +828,14 @@ def run_linear_sweep(args):
 def run_sweep(args):
     """The HBM-bound kernels alone on the sweep shapes, one launch at a time
     with a 256 MB L2 flush in between (the 4,096-token working set is close
-    to the 126 MB L2), median of the timed launches."""
+    to the 126 MB L2: 256 MB written, then 256 MB read, so no dirty lines are
+    written back during the kernel), median of the timed launches."""
     import torch
     from packed_attention_qk_b200 import pqk
     from packed_attention_qk_b200 import workloads as wl
     dev = torch.device("cuda", 0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clean = torch.ones(64 << 20, dtype=torch.int32, device=dev)
     pk, pk_kind = peaks()
 
     def dev16(bits):
@@ -762,6 +845,7 @@ def run_sweep(args):
         ts = []
         for i in range(args.warmup + reps):
             flush.fill_(i & 0xFF)
+            clean.sum()  # evicts the written lines before the kernel starts
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fn()

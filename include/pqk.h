@@ -38,6 +38,10 @@
  *     compute entry point on a device queries and caches device attributes
  *     and kernel settings; make it before capturing. pqk_get_device_status
  *     synchronizes and must not be captured.
+ *   - Per-device state (the status word's device address, cached device
+ *     attributes) is looked up once per device and kept for the life of its
+ *     CUDA context: do not use the library on a device after destroying and
+ *     recreating its context (cudaDeviceReset).
  */
 #ifndef PQK_H
 #define PQK_H
@@ -307,9 +311,12 @@ PQK_API int pqk_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* 
  * workspace. B may be at most 4096; a larger B returns PQK_ERR_WORKSPACE.
  * The first call on a device looks up the array's device address (a CUDA
  * runtime query, no allocation); make that first call before capturing a
- * stream. Every call uses the same array, so calls whose work overlaps on
- * the GPU (e.g. on different streams) race and must be serialised by the
- * caller; each call rewrites the whole schedule it reads, so nothing needs
+ * stream. The address is kept for the life of the device's CUDA context: a
+ * caller that destroys and recreates the context (cudaDeviceReset) must not
+ * call this entry point on that device afterwards. Every call uses the same
+ * array, so calls whose work overlaps on the GPU (e.g. on different streams)
+ * race and must be serialised by the caller; each call rewrites the whole
+ * schedule it reads and resets the tile-claim counter in it, so nothing needs
  * to be cleared between calls.
  */
 PQK_API int pqk_varlen_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,

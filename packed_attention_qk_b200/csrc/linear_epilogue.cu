@@ -1,47 +1,51 @@
-// linear_epilogue.cu -- persistent tcgen05 GEMM out = epilogue(A W^T) for
-// the linear layers around the DiT block's fused operators, with the
-// residual connection or SwiGLU done in the GEMM's epilogue instead of a
-// separate pass over the GEMM's output (the pages fuse "residual
-// connections" and SwiGLU into fewer launches: "FastH3 在八卡 B300 上实现完整
-// MP4 生成快于播放时长", section "融合 DiT 算子"; "MiniMax H3 FastH3 real-time
-// serving with vLLM-Omni", bullet "Fused DiT operators"):
+// linear_epilogue.cu -- persistent tcgen05 GEMM on CTA pairs,
+// out = epilogue(A W^T), for the linear layers around the DiT block's fused
+// operators, with the residual connection or SwiGLU done in the GEMM's
+// epilogue instead of a separate pass over the GEMM's output (the pages fuse
+// "residual connections" and SwiGLU into fewer launches: "FastH3 在八卡 B300 上
+// 实现完整 MP4 生成快于播放时长", section "融合 DiT 算子"; "MiniMax H3 FastH3
+// real-time serving with vLLM-Omni", bullet "Fused DiT operators"):
 //
 //   kEpiGatedResidual  out[t, n] = x[t, n] + gate_res[s(t), n] * (A W^T)[t, n]
-//                      (output projection after attention, W2 after SwiGLU)
 //   kEpiSwiglu         out[t, f] = silu((A W_gate^T)[t, f]) * (A W_up^T)[t, f]
-//                      (W1; W_gate = the first F rows of W1, W_up the last F)
 //   kEpiNone           out = A W^T
 //
 // A: [T, K] bf16 (token stride a_stride), W: [N, K] bf16 (out x in). fp32
 // accumulation in tensor memory, epilogue arithmetic in fp32, bf16 output
 // rounded to nearest even.
 //
-// Structure (one CTA per SM, persistent over 128 x 256 accumulator tiles):
-//   warp 0      TMA producer: per K block of 64, the A box (128 tokens x 64)
-//               and two W boxes (2 x 128 rows x 64) into a 4-stage ring of
-//               48 KB stages, 128-byte swizzled, K-major.
-//   warp 1      allocates 512 tensor-memory columns (two 256-column fp32
-//               accumulators) and issues tcgen05.mma M=128 N=256 K=16 (four
-//               per stage) from one thread; commits free the stage, and the
-//               last K block of a tile commits the accumulator to the
-//               epilogue.
-//   warps 2-5   epilogue: each thread owns one token row (tensor-memory lane)
-//               of the tile, reads its accumulator columns 32 at a time, adds
-//               the gated residual or applies SwiGLU and stores 16-byte
-//               chunks; then releases the accumulator. The two accumulators
-//               let the epilogue of one tile run under the main loop of the
-//               next.
-// The W boxes of a SwiGLU tile are the gate rows f0..f0+127 and the up rows
-// F+f0..F+f0+127, so one N = 256 MMA computes both halves of 128 outputs.
-// Rows past T or N read as zeros (TMA bounds) and are not stored. Tiles are
-// rastered in groups of 16 M tiles so that concurrently running CTAs share
-// A rows and W columns in L2.
+// Two CTAs of a cluster work on one 256-token x 256-column accumulator tile
+// (tcgen05 cta_group::2, M = 256): each CTA loads its 128 A rows and 128 of
+// the 256 W rows per K block of 64 into its own 6-stage ring (32 KB stages),
+// the even CTA's single MMA thread drives both SMs' tensor cores, and each
+// CTA's tensor memory holds its 128 rows of the tile in one of two
+// 256-column accumulators.
+//   warp 0      TMA producer in each CTA; copies complete on the even CTA's
+//               stage barrier, where only the even CTA posts the stage's
+//               bytes and then lets the odd CTA's producer load its halves.
+//   warp 1      allocates the tensor memory of the pair; in the even CTA
+//               issues the MMAs and commits stage releases and finished
+//               accumulators to its own barriers.
+//   warps 2-5   epilogue in each CTA: 32 token rows per warp, 32 columns of
+//               the accumulator at a time, the gated residual or SwiGLU, 16-
+//               byte stores; one release per warp to the even CTA's MMA
+//               thread. The even CTA passes "accumulator ready" on to the odd
+//               CTA.
+// Hand-offs between the two CTAs are plain remote mbarrier arrives, one CTA
+// signalling the other. A SwiGLU tile's W halves are 128 gate rows (even
+// CTA) and the same 128 up rows (odd CTA). Rows past T or N and columns past
+// K read as zeros and are not stored.
 //
 // Every wait is bounded (the library's timeout); a wait that runs out raises
-// the block's abort flag and the device status word and every role stops
-// issuing work. Once all roles have stopped (a block barrier), the copies and
-// MMAs still in flight are drained with waits bounded by kDrainTimeoutNs,
-// not by the caller's timeout, and only then is the tensor memory freed.
+// the abort flag of both CTAs and the device status word, and every role of
+// the pair stops issuing work. After a cluster barrier (when both flags are
+// final) the even CTA waits for the stages it posted that may still be
+// loading (their barriers complete only once both CTAs' copies have landed:
+// the odd CTA copies into a stage only after the even one posted it) and for
+// every MMA it issued, with waits bounded by kDrainTimeoutNs rather than the
+// caller's timeout; a second cluster barrier keeps the odd CTA, whose copies
+// signal the even CTA's barriers, from exiting before that, and both free
+// the pair's tensor memory.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -54,18 +58,16 @@
 namespace pqk {
 namespace {
 
-constexpr int kBM = 128;         // tokens per tile (one tensor-memory lane each)
-constexpr int kBK = 64;          // K per stage: one 128-byte swizzle row of bf16
-constexpr int kBoxRows = 128;    // W rows per TMA box
-constexpr int kAccCols = 256;    // fp32 accumulator columns per tile = MMA N
-constexpr int kStages = 4;
+constexpr int kBM = 128;       // token rows per CTA (pair: 256)
+constexpr int kBK = 64;        // K per stage: one 128-byte swizzle row of bf16
+constexpr int kBoxRows = 128;  // W rows per CTA and stage
+constexpr int kAccCols = 256;  // fp32 accumulator columns per tile = MMA N
+constexpr int kStages = 6;
 constexpr int kThreads = 192;
-constexpr int kProducerWarp = 0;
-constexpr int kMmaWarp = 1;
-constexpr int kGroupM = 16;      // tile raster: M tiles per group
-constexpr uint32_t kABytes = kBM * kBK * 2;              // 16 KB
-constexpr uint32_t kBBytes = 2 * kBoxRows * kBK * 2;     // 32 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr int kGroupM = 8;     // raster: pair M tiles per group
+constexpr uint32_t kABytes = kBM * kBK * 2;        // 16 KB
+constexpr uint32_t kBBytes = kBoxRows * kBK * 2;   // 16 KB
+constexpr uint32_t kPairStageBytes = 2 * (kABytes + kBBytes);
 
 struct Layout {
   static constexpr int kAOff = 0;
@@ -78,10 +80,9 @@ struct Layout {
   static constexpr int kBytes = kAbortOff + 4;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
   static_assert(kAlloc <= 232448, "shared memory budget");
-  static_assert(kBOff % 1024 == 0 && kBBytes % 1024 == 0 && kABytes % 1024 == 0, "swizzle atoms 1024-aligned");
 };
 
-struct LinearParams {
+struct Params {
   __nv_bfloat16* out;
   int64_t out_stride;
   const __nv_bfloat16* x;   // gated residual input [T, N]
@@ -92,20 +93,81 @@ struct LinearParams {
   int64_t T;
   int N;                    // output columns (F for SwiGLU)
   int n_kb;                 // K blocks of 64
-  int m_tiles;
+  int m_pairs;              // 256-token tiles
   int n_tiles;
   int* status;
   long long timeout_ns;
 };
 
+__device__ __forceinline__ uint32_t ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t nclusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// the same shared-memory variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t in_cta(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void st_remote_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mma_bf16_ss_pair(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t desc_hi,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      ".reg .b64 da, db;\n"
+      "setp.ne.b32 p, %5, 0;\n"
+      "mov.b64 da, {%1, %3};\n"
+      "mov.b64 db, {%2, %3};\n"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %4, {%6, %6, %6, %6, %6, %6, %6, %6}, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(desc_hi), "r"(idesc), "r"(accumulate), "r"(0u)
+      : "memory");
+}
+
 struct TileCoord {
   int m;
   int n;
 };
-
-// Tile i of the raster: groups of kGroupM M tiles, and inside a group the
-// M tile varies fastest, so the CTAs that run together cover a few W column
-// blocks of a 16-tile band of A.
 __device__ __forceinline__ TileCoord tile_coord(int i, int m_tiles, int n_tiles) {
   const int group_tiles = kGroupM * n_tiles;
   const int g = i / group_tiles;
@@ -118,12 +180,6 @@ __device__ __forceinline__ TileCoord tile_coord(int i, int m_tiles, int n_tiles)
   return c;
 }
 
-__device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* status) {
-  *abort_flag = 1;
-  atomicCAS(status, 0, kStatusTimeout);
-}
-
-// Request s with cu[s] <= t < cu[s+1] (the last such s when requests are empty).
 __device__ __forceinline__ int request_of(const int32_t* cu, int B, int64_t t) {
   int lo = 0, hi = B - 1;
   while (lo < hi) {
@@ -132,24 +188,19 @@ __device__ __forceinline__ int request_of(const int32_t* cu, int B, int64_t t) {
   }
   return lo;
 }
-
 __device__ __forceinline__ uint4 ld_nc16(const void* p) {
   uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
   return v;
 }
-
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 template <int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
-    linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
-                  const __grid_constant__ CUtensorMap tm_b1, const LinearParams p) {
+    linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
+                       const __grid_constant__ CUtensorMap tm_b1, const Params p) {
   using L = Layout;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
@@ -158,6 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = ctarank();
+  const bool even = rank == 0;
   const uint32_t a_smem = base + L::kAOff;
   const uint32_t b_smem = base + L::kBOff;
   const uint32_t bar0 = base + L::kBarOff;
@@ -168,6 +221,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t drain = bar0 + 8u * (2 * kStages + 4);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
+  const uint32_t peer_abort = in_cta(base + L::kAbortOff, rank ^ 1u);
+  auto raise_abort = [&]() {
+    *abort_flag = 1;
+    st_remote_u32(peer_abort, 1u);
+    atomicCAS(p.status, 0, kStatusTimeout);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -176,64 +235,73 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full(i), 1);
-      mbar_init(acc_empty(i), 128);
+      mbar_init(acc_empty(i), 2 * 4);  // one arrive per epilogue warp of each CTA
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
-    tmem_alloc(base + L::kTmemSlotOff, 512);
-    tmem_relinquish();
+  if (warp == 1) {
+    tmem_alloc_pair(base + L::kTmemSlotOff, 512);
+    tmem_relinquish_pair();
   }
-  if (warp == kProducerWarp && lane == 0) {
+  if (warp == 0 && lane == 0) {
     prefetch_tensor_map(&tm_a);
     prefetch_tensor_map(&tm_b0);
     prefetch_tensor_map(&tm_b1);
   }
   tc_fence_before_sync();
-  __syncthreads();
+  __syncwarp();
+  cluster_sync_all();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int n_tiles_total = p.m_tiles * p.n_tiles;
-  uint32_t loads = 0;  // stage copies issued by the producer thread, for the drain
+  const int total = p.m_pairs * p.n_tiles;
+  const int pair = static_cast<int>(cluster_x());
+  const int npairs = static_cast<int>(nclusters_x());
+  uint32_t loads = 0;  // stages this CTA's producer loaded into, for the drain
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------ TMA producer
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       uint32_t& it = loads;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
-        const TileCoord tc = tile_coord(tile, p.m_tiles, p.n_tiles);
-        // W rows of the tile's two boxes: 256 consecutive output columns, or
-        // the same 128 rows of the gate and the up halves
-        const int r0 = kEpi == kEpiSwiglu ? tc.n * kBoxRows : tc.n * kAccCols;
-        const int r1 = kEpi == kEpiSwiglu ? tc.n * kBoxRows : tc.n * kAccCols + kBoxRows;
-        const CUtensorMap* m1 = kEpi == kEpiSwiglu ? &tm_b1 : &tm_b0;
+      const CUtensorMap* mb = (kEpi == kEpiSwiglu && !even) ? &tm_b1 : &tm_b0;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        const TileCoord tc = tile_coord(tile, p.m_pairs, p.n_tiles);
+        const int arow = tc.m * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int brow = kEpi == kEpiSwiglu ? tc.n * kBoxRows : tc.n * kAccCols + static_cast<int>(rank) * kBoxRows;
         for (int kb = 0; kb < p.n_kb; ++kb) {
           const int s = it % kStages;
           const uint32_t round = it / kStages;
-          if (round > 0 && !(ok = mbar_wait(empty(s), (round - 1) & 1, abort_flag, p.timeout_ns))) break;
-          mbar_arrive_expect_tx(full(s), kStageBytes);
-          tma_load_2d(a_smem + s * kABytes, &tm_a, full(s), kb * kBK, tc.m * kBM);
-          tma_load_2d(b_smem + s * kBBytes, &tm_b0, full(s), kb * kBK, r0);
-          tma_load_2d(b_smem + s * kBBytes + kBBytes / 2, m1, full(s), kb * kBK, r1);
+          if (even) {
+            // the MMAs that read this stage in both CTAs are complete; post the
+            // stage's bytes, then let the odd CTA's producer load its halves
+            // (so no copy of it completes before the count it belongs to)
+            if (round > 0 && !(ok = mbar_wait(empty(s), (round - 1) & 1, abort_flag, p.timeout_ns))) break;
+            mbar_arrive_expect_tx(full(s), kPairStageBytes);
+            arrive_remote(in_cta(empty(s), 1));
+          } else {
+            if (!(ok = mbar_wait(empty(s), round & 1, abort_flag, p.timeout_ns))) break;
+          }
+          const uint32_t bar = in_cta(full(s), 0);
+          tma_load_2d_pair(a_smem + s * kABytes, &tm_a, bar, kb * kBK, arow);
+          tma_load_2d_pair(b_smem + s * kBBytes, mb, bar, kb * kBK, brow);
           ++it;
         }
       }
-      if (!ok) raise_abort(abort_flag, p.status);
+      if (!ok) raise_abort();
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kAccCols, false);
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && even) {
+      constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kBM, kAccCols, false);
       constexpr uint32_t kDescHi = smem_desc_hi_sw128(1024);
       const uint32_t a_lo = smem_desc_lo(a_smem, 16);
       const uint32_t b_lo = smem_desc_lo(b_smem, 16);
       uint32_t it = 0;
       int tcount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++tcount) {
+      for (int tile = pair; tile < total && ok; tile += npairs, ++tcount) {
         const int acc = tcount & 1;
         const uint32_t use = static_cast<uint32_t>(tcount >> 1);
         if (use > 0 && !(ok = mbar_wait(acc_empty(acc), (use - 1) & 1, abort_flag, p.timeout_ns))) break;
@@ -243,33 +311,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = it % kStages;
           if (!(ok = mbar_wait(full(s), (it / kStages) & 1, abort_flag, p.timeout_ns))) break;
           tc_fence_after_sync();
-          // K steps of 16 (32 bytes inside the 128-byte swizzled row)
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
-            mma_bf16_ss_w(d, a_lo + s * (kABytes >> 4) + 2 * k, b_lo + s * (kBBytes >> 4) + 2 * k, kDescHi, kIdesc,
-                          (kb > 0 || k > 0) ? 1u : 0u);
-          tc_commit(empty(s));
+            mma_bf16_ss_pair(d, a_lo + s * (kABytes >> 4) + 2 * k, b_lo + s * (kBBytes >> 4) + 2 * k, kDescHi, kIdesc,
+                             (kb > 0 || k > 0) ? 1u : 0u);
+          tc_commit_pair(empty(s));
           ++it;
         }
         if (!ok) break;
-        tc_commit(acc_full(acc));
+        tc_commit_pair(acc_full(acc));
       }
-      if (!ok) raise_abort(abort_flag, p.status);
+      if (!ok) raise_abort();
     }
   } else {
-    // ------------------------------------------------ epilogue warps 2-5
-    const int quarter = warp & 3;  // tensor-memory lanes 32 * quarter .. + 31
+    // ------------------------------------------------ epilogue warps 2-5 (both CTAs)
+    const int quarter = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     int tcount = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++tcount) {
-      const TileCoord tc = tile_coord(tile, p.m_tiles, p.n_tiles);
+    for (int tile = pair; tile < total; tile += npairs, ++tcount) {
+      const TileCoord tc = tile_coord(tile, p.m_pairs, p.n_tiles);
       const int acc = tcount & 1;
       const uint32_t use = static_cast<uint32_t>(tcount >> 1);
       ok = __all_sync(0xffffffffu, mbar_wait(acc_full(acc), use & 1, abort_flag, p.timeout_ns));
       if (!ok) break;
+      // the even CTA's MMAs wrote both CTAs' accumulators: tell the odd CTA
+      if (even && warp == 2 && lane == 0) arrive_remote(in_cta(acc_full(acc), 1));
       tc_fence_after_sync();
-      const int64_t row = static_cast<int64_t>(tc.m) * kBM + quarter * 32 + lane;
+      const int64_t row = static_cast<int64_t>(tc.m) * 2 * kBM + rank * kBM + quarter * 32 + lane;
       const bool row_ok = row < p.T;
       const uint32_t t_acc = tmem + lane_off + static_cast<uint32_t>(acc * kAccCols);
       __nv_bfloat16* dst = p.out + (row_ok ? row : 0) * p.out_stride;
@@ -344,30 +413,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before_sync();
-      mbar_arrive(acc_empty(acc));
+      __syncwarp();
+      // release the accumulator to the even CTA's MMA issuer (both CTAs' warps count)
+      if (lane == 0) arrive_remote(in_cta(acc_empty(acc), 0));
     }
-    if (!ok) raise_abort(abort_flag, p.status);
+    if (!ok) raise_abort();
   }
 
   tc_fence_before_sync();
-  __syncthreads();
-  // Every role has stopped, so the abort flag is final. On an abort, wait for
-  // the copies and MMAs still in flight before the memory is freed.
+  __syncwarp();
+  cluster_sync_all();  // no CTA frees its tensor memory or exits while its pair still works
+  // Every role of both CTAs has stopped: the abort flags are final and the
+  // same in both CTAs. On an abort, wait for what may still be in flight.
   if (*abort_flag) {
-    if (warp == kProducerWarp && lane == 0) {
-      // copy idx was issued only after copy idx - kStages had landed: the
-      // last kStages copies are the ones that can be outstanding
+    if (even && warp == 0 && lane == 0) {
+      // stage idx was posted only after stage idx - kStages had landed in
+      // both CTAs: the last kStages posted stages are the ones outstanding
       const uint32_t first = loads > static_cast<uint32_t>(kStages) ? loads - kStages : 0;
       for (uint32_t idx = first; idx < loads; ++idx) mbar_drain_wait(full(idx % kStages), (idx / kStages) & 1);
-    } else if (warp == kMmaWarp && lane == 0) {
-      // completes once every MMA this thread issued has
-      tc_commit(drain);
+    } else if (even && warp == 1 && lane == 0) {
+      // completes once every MMA of the pair has
+      tc_commit_pair(drain);
       mbar_drain_wait(drain, 0);
     }
-    __syncthreads();
+    __syncwarp();
+    cluster_sync_all();
   }
   tc_fence_after_sync();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  if (warp == 1) tmem_dealloc_pair(tmem, 512);
 }
 
 // ------------------------------------------------------------ host side
@@ -403,27 +476,46 @@ bool make_rows_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Per device and epilogue: the shared-memory attribute is set and the number
+// of CTA pairs that can be resident at once is queried on the first call
+// (which must precede any stream capture), so that the persistent grid never
+// leaves a pair waiting for a second wave.
 template <int kEpi>
-bool set_smem_attr() {
-  static int done[64] = {0};
+int resident_pairs(cudaLaunchConfig_t* cfg) {
+  static int pairs[64] = {0};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (!done[dev]) {
-    if (cudaFuncSetAttribute(linear_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout::kAlloc) !=
-        cudaSuccess)
-      return false;
-    done[dev] = 1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (pairs[dev] == 0) {
+    if (cudaFuncSetAttribute(linear_pair_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Layout::kAlloc) != cudaSuccess)
+      return -1;
+    int n = 0;
+    cfg->gridDim = dim3(2, 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&n, linear_pair_kernel<kEpi>, cfg) != cudaSuccess || n < 1) return -1;
+    pairs[dev] = n;
   }
-  return true;
+  return pairs[dev];
 }
 
 template <int kEpi>
-int launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const LinearParams& p,
-           cudaStream_t stream, int num_sms) {
-  if (!set_smem_attr<kEpi>()) return -1;
-  const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  linear_kernel<kEpi><<<grid, kThreads, Layout::kAlloc, stream>>>(ta, tb0, tb1, p);
+int launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const Params& p,
+           cudaStream_t stream) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Layout::kAlloc;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int max_pairs = resident_pairs<kEpi>(&cfg);
+  if (max_pairs < 1) return -1;
+  const int tiles = p.m_pairs * p.n_tiles;
+  cfg.gridDim = dim3(2 * (tiles < max_pairs ? tiles : max_pairs), 1, 1);
+  if (cudaLaunchKernelEx(&cfg, linear_pair_kernel<kEpi>, ta, tb0, tb1, p) != cudaSuccess) return -1;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -432,12 +524,13 @@ int launch(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1
 int launch_linear(int epi, const void* a, int64_t a_stride, const void* w, const void* x, int64_t x_stride,
                   const float* gate_res, const int32_t* cu, int B, void* out, int64_t out_stride, int64_t T, int K,
                   int N, int* status, long long timeout_ns, cudaStream_t stream, int num_sms) {
+  (void)num_sms;
   CUtensorMap ta, tb0, tb1;
   const bool swiglu = epi == kEpiSwiglu;
   bool ok = make_rows_map(&ta, a, T, K, a_stride, kBM);
   if (swiglu) {
-    // W1 [2N, K]: gate rows [0, N), up rows [N, 2N), each its own map so that
-    // the last tile's rows past N read as zeros rather than the other half
+    // W1 [2N, K]: gate rows [0, N) for the even CTA, up rows [N, 2N) for the
+    // odd one, each its own map so that rows past N read as zeros
     ok = ok && make_rows_map(&tb0, w, N, K, K, kBoxRows) &&
          make_rows_map(&tb1, static_cast<const __nv_bfloat16*>(w) + static_cast<int64_t>(N) * K, N, K, K, kBoxRows);
   } else {
@@ -445,7 +538,7 @@ int launch_linear(int epi, const void* a, int64_t a_stride, const void* w, const
     tb1 = tb0;
   }
   if (!ok) return -2;
-  LinearParams p;
+  Params p;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.out_stride = out_stride;
   p.x = static_cast<const __nv_bfloat16*>(x);
@@ -456,13 +549,13 @@ int launch_linear(int epi, const void* a, int64_t a_stride, const void* w, const
   p.T = T;
   p.N = N;
   p.n_kb = (K + kBK - 1) / kBK;
-  p.m_tiles = static_cast<int>((T + kBM - 1) / kBM);
+  p.m_pairs = static_cast<int>((T + 2 * kBM - 1) / (2 * kBM));
   p.n_tiles = swiglu ? (N + kBoxRows - 1) / kBoxRows : (N + kAccCols - 1) / kAccCols;
   p.status = status;
   p.timeout_ns = timeout_ns;
-  if (epi == kEpiGatedResidual) return launch<kEpiGatedResidual>(ta, tb0, tb1, p, stream, num_sms);
-  if (swiglu) return launch<kEpiSwiglu>(ta, tb0, tb1, p, stream, num_sms);
-  return launch<kEpiNone>(ta, tb0, tb1, p, stream, num_sms);
+  if (epi == kEpiGatedResidual) return launch<kEpiGatedResidual>(ta, tb0, tb1, p, stream);
+  if (swiglu) return launch<kEpiSwiglu>(ta, tb0, tb1, p, stream);
+  return launch<kEpiNone>(ta, tb0, tb1, p, stream);
 }
 
 }  // namespace pqk

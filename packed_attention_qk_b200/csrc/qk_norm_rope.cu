@@ -19,6 +19,12 @@
 // K) with one weight per element: a first pass of the warp over the token's
 // rows sums the squares (full-warp reduction), the second pass re-reads the
 // rows (now in cache), normalises, rotates and stores.
+// Few tokens: with about one token per resident warp the slowest warps take
+// two tokens while most take one, and the launch ends at the tail. The
+// launcher then splits each token's 2*H rows into n_split tasks of
+// rows_per_task rows (a warp task is a (token, row range) pair; every task
+// forms its own cos/sin), chosen so that each warp gets several tasks; with
+// enough tokens n_split is 1 and a task is a whole token.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -48,6 +54,8 @@ struct QkParams {
   float eps;
   double log2_base;
   int style;
+  int n_split;        // tasks per token (1: the whole token)
+  int rows_per_task;  // rows of the token's 2H a task covers (2H when n_split is 1)
 };
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
@@ -107,10 +115,14 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
   // per-head weights ([D], shared by all heads) stay in registers
   const uint4 wq_raw = kFullWidth ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(p.wq + chunk * 8);
   const uint4 wk_raw = kFullWidth ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(p.wk + chunk * 8);
-  const int rows = 2 * p.H;
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + threadIdx.x / 32; t < p.T;
-       t += warps_total) {
+  const int64_t n_tasks = p.T * p.n_split;
+  for (int64_t task = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + threadIdx.x / 32; task < n_tasks;
+       task += warps_total) {
+    const int64_t t = p.n_split == 1 ? task : task / p.n_split;
+    // this task's rows [r_lo, rows) of the token's 2H (Q heads, then K heads)
+    const int r_lo = p.n_split == 1 ? 0 : static_cast<int>(task % p.n_split) * p.rows_per_task;
+    const int rows = min(2 * p.H, r_lo + p.rows_per_task);
     int32_t pos3[3];
     if constexpr (kThreeAxis) {
       pos3[0] = p.pos[3 * t];
@@ -134,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
     float inv_q = 0.f, inv_k = 0.f;
     if constexpr (kFullWidth) {
       float ssq_q = 0.f, ssq_k = 0.f;
-      for (int r0 = 0; r0 < rows; r0 += kRowsPerStep * kUnroll) {
+      for (int r0 = r_lo; r0 < rows; r0 += kRowsPerStep * kUnroll) {
         uint4 raw[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
@@ -166,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
       inv_q = rsqrtf(ssq_q * inv_width + p.eps);
       inv_k = rsqrtf(ssq_k * inv_width + p.eps);
     }
-    for (int r0 = 0; r0 < rows; r0 += kRowsPerStep * kUnroll) {
+    for (int r0 = r_lo; r0 < rows; r0 += kRowsPerStep * kUnroll) {
       uint4 raw[kUnroll];
       bool live[kUnroll];
 #pragma unroll
@@ -257,8 +269,25 @@ int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k
   p.log2_base = log2(static_cast<double>(rope_base));
   p.style = style;
   const int64_t warps_per_block = kThreads / 32;
-  const int64_t want = (T + warps_per_block - 1) / warps_per_block;
   const int64_t cap = static_cast<int64_t>(num_sms) * 3;
+  // split tokens into row ranges when there are fewer than kTasksPerWarp
+  // tokens per resident warp (not for the full-width norm, which needs all
+  // of a token's rows in one warp); ranges are whole warp steps of rows
+  constexpr int64_t kTasksPerWarp = 4;
+  const int rows = 2 * H;
+  const int step_rows = (32 / (D / 8)) * kUnroll;
+  const int64_t resident_warps = cap * warps_per_block;
+  int rows_per_task = rows;
+  if (!full_width && T < kTasksPerWarp * resident_warps) {
+    const int64_t want_split = (kTasksPerWarp * resident_warps + T - 1) / (T > 0 ? T : 1);
+    const int r = static_cast<int>(rows / want_split) / step_rows * step_rows;
+    rows_per_task = r > step_rows ? r : step_rows;
+    if (rows_per_task > rows) rows_per_task = rows;
+  }
+  p.rows_per_task = rows_per_task;
+  p.n_split = (rows + rows_per_task - 1) / rows_per_task;
+  const int64_t tasks = T * p.n_split;
+  const int64_t want = (tasks + warps_per_block - 1) / warps_per_block;
   const int grid = static_cast<int>(want < cap ? want : cap);
   const bool three = sections != nullptr;
   if (D == 128) {

@@ -87,11 +87,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const v
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t polls = 1;; ++polls) {
+    // try_wait may itself suspend for a system-defined time, so the time is
+    // checked after every unsuccessful try
     if (mbar_try_wait(bar, parity)) return true;
-    if ((polls & 31u) == 0u) {
-      if (*abort_flag) return false;
-      if ((long long)(global_timer_ns() - t0) > timeout_ns || polls >= kMaxPolls) return false;
-    }
+    if (*abort_flag) return false;
+    if ((long long)(global_timer_ns() - t0) > timeout_ns || polls >= kMaxPolls) return false;
   }
 }
 

@@ -12,8 +12,13 @@
 // 128-row query tiles Q0, Q1 that share every K/V tile. A one-block
 // schedule kernel turns cu_seqlens into a tile list (requests longest
 // first, then head, then query block, so that the CTAs running at the same
-// time read the same head's K/V from L2), and a persistent kernel with one
-// CTA per SM walks that list round-robin.
+// time read the same head's K/V from L2) and resets a claim counter; a
+// persistent kernel with one CTA per SM claims tiles from that list in
+// order with an atomic on the counter (each CTA's producer claims its next
+// tile when it is ready to load it and hands the index to the block's other
+// roles through shared memory), so a CTA that runs faster simply takes more
+// tiles. Each tile has exactly one owner and writes only its own rows, so the
+// result does not depend on which CTA computed what.
 //
 // CTA roles (320 threads):
 //   warps 0-3  softmax for Q0; thread r owns query row r (tensor-memory lane r)
@@ -87,6 +92,12 @@ constexpr float kRescaleThreshold = PQK_ATTN_RESCALE_LOG2;
 #endif
 constexpr bool kPacked = PQK_ATTN_PACKED != 0;
 constexpr int kSlabBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-byte swizzle width)
+// Ring of claimed work-tile indices in shared memory. The producer claims
+// tile wt + 1 only once the Q K^T products of tile wt are complete, and the
+// MMA thread starts tile wt + 1 only after the softmax warps have handed over
+// the last P of tile wt, so the producer is at most two tiles ahead of the
+// softmax warps: at most three slots are live.
+constexpr int kWorkSlots = 4;
 
 template <int D>
 struct Layout {
@@ -96,22 +107,31 @@ struct Layout {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  // barriers: kv_full[S], kv_empty[S], q_full, q_empty, s_full[2], p_full[2], o_done[2], drain
-  static constexpr int kNumBars = 2 * kStages + 9;
+  // barriers: kv_full[S], kv_empty[S], q_full, q_empty, s_full[2], p_full[2], o_done[2], drain,
+  // work_full[kWorkSlots]
+  static constexpr int kNumBars = 2 * kStages + 9 + kWorkSlots;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemSlotOff + 4;
   // block-skip votes: one byte per softmax warp, [group][tile parity][warp]
   static constexpr int kVoteOff = kAbortOff + 4;
-  static constexpr int kBytes = kVoteOff + 16;
+  // claimed work-tile indices, a ring of kWorkSlots (-1: no more work)
+  static constexpr int kWorkOff = kVoteOff + 16;
+  // the producer's copy counts (K/V stages, Q pairs), left for the drain
+  static constexpr int kLoadsOff = kWorkOff + 4 * kWorkSlots;
+  static constexpr int kBytes = kLoadsOff + 8;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
   static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256, kTmemO1 = 256 + D;
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
 // Schedule in the workspace (int32): [0] number of work tiles, [1] number of
-// requests B, then for the requests in schedule order r = 0..B-1:
-// tile_start[B+1] (prefix of tiles), seg_start[B], seg_len[B].
-__host__ __device__ constexpr size_t sched_words(int B) { return 2 + (B + 1) + 2 * static_cast<size_t>(B); }
+// requests B, [2] the claim counter (reset to 0 by the schedule kernel on
+// every call), [3] unused, then for the requests in schedule order r =
+// 0..B-1: tile_start[B+1] (prefix of tiles), seg_start[B], seg_len[B].
+constexpr int kSchedHeader = 4;
+__host__ __device__ constexpr size_t sched_words(int B) {
+  return kSchedHeader + (B + 1) + 2 * static_cast<size_t>(B);
+}
 
 struct AttnParams {
   __nv_bfloat16* o;
@@ -138,7 +158,7 @@ struct Work {
 
 __device__ __forceinline__ Work decode_work(const int32_t* sched, int H, int w) {
   const int B = sched[1];
-  const int32_t* tile_start = sched + 2;
+  const int32_t* tile_start = sched + kSchedHeader;
   const int32_t* seg_start = tile_start + B + 1;
   const int32_t* seg_len = seg_start + B;
   int lo = 0, hi = B - 1;  // last r with tile_start[r] <= w
@@ -163,13 +183,39 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int* statu
   atomicCAS(status, 0, kStatusTimeout);
 }
 
+// Drain of an aborting block (after its final barrier). Kept out of line:
+// inlined, the rarely run drain loops change the register allocation of the
+// softmax loop.
+// Producer: K/V copy idx was issued only after copy idx - n_stages had
+// landed, so the last n_stages copies (and the last Q pair) are the ones
+// that can be outstanding; each is the newest phase of its stage barrier
+// (stage s at bar_kv_full + 8 s).
+__device__ __noinline__ void drain_copies(uint32_t bar_kv_full, uint32_t bar_q_full, uint32_t n_stages,
+                                          uint32_t load_idx, uint32_t q_loads) {
+  const uint32_t first = load_idx > n_stages ? load_idx - n_stages : 0;
+  for (uint32_t idx = first; idx < load_idx; ++idx)
+    mbar_drain_wait(bar_kv_full + 8u * (idx % n_stages), (idx / n_stages) & 1);
+  if (q_loads > 0) mbar_drain_wait(bar_q_full, (q_loads - 1) & 1);
+}
+
+// MMA thread: a commit on the (otherwise unused) drain barrier completes
+// once every MMA this thread issued has, and with them the arrivals of their
+// own commits.
+__device__ __noinline__ void drain_mmas(uint32_t bar_drain) {
+  tc_commit(bar_drain);
+  mbar_drain_wait(bar_drain, 0);
+}
+
 // ------------------------------------------------------------ schedule
 
 constexpr int kSchedThreads = 1024;
 constexpr int kSortLimit = 8192;  // requests ordered longest first up to this B
+// dynamic shared memory of the schedule kernel: one 64-bit sort key per request
+constexpr int kSchedSmem = kSortLimit * 8;
 
 __global__ void __launch_bounds__(kSchedThreads) build_schedule_kernel(const int32_t* cu, int B, int64_t T, int H,
                                                                         int32_t* sched, int* status) {
+  extern __shared__ uint64_t sort_keys[];
   __shared__ int bad;
   __shared__ int32_t carry;
   if (threadIdx.x == 0) {
@@ -180,30 +226,55 @@ __global__ void __launch_bounds__(kSchedThreads) build_schedule_kernel(const int
   for (int i = threadIdx.x; i < B; i += kSchedThreads)
     if (cu[i + 1] < cu[i]) bad = 1;
   __syncthreads();
-  int32_t* tile_start = sched + 2;
+  int32_t* tile_start = sched + kSchedHeader;
   int32_t* seg_start = tile_start + B + 1;
   int32_t* seg_len = seg_start + B;
   if (bad) {
     if (threadIdx.x == 0) {
       sched[0] = 0;
       sched[1] = B;
+      sched[2] = 0;
       atomicCAS(status, 0, kStatusBadSeqlens);
     }
     return;
   }
-  // rank of request i: longer first, ties by index (identity order above kSortLimit)
-  for (int i = threadIdx.x; i < B; i += kSchedThreads) {
-    const int Li = cu[i + 1] - cu[i];
-    int rank = i;
-    if (B <= kSortLimit) {
-      rank = 0;
-      for (int j = 0; j < B; ++j) {
-        const int Lj = cu[j + 1] - cu[j];
-        rank += (Lj > Li) || (Lj == Li && j < i);
+  if (B <= kSortLimit) {
+    // requests longest first, ties by index: a bitonic sort of the keys
+    // (INT32_MAX - length) << 32 | index over the next power of two, padded
+    // with keys above every real one
+    int n = 1;
+    while (n < B) n <<= 1;
+    for (int i = threadIdx.x; i < n; i += kSchedThreads)
+      sort_keys[i] = i < B ? (static_cast<uint64_t>(static_cast<uint32_t>(INT32_MAX - (cu[i + 1] - cu[i]))) << 32) |
+                                 static_cast<uint32_t>(i)
+                           : ~0ull;
+    __syncthreads();
+    for (int k = 2; k <= n; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = threadIdx.x; i < n; i += kSchedThreads) {
+          const int partner = i ^ j;
+          if (partner > i) {
+            const uint64_t a = sort_keys[i], b = sort_keys[partner];
+            if ((a > b) == ((i & k) == 0)) {
+              sort_keys[i] = b;
+              sort_keys[partner] = a;
+            }
+          }
+        }
+        __syncthreads();
       }
     }
-    seg_start[rank] = cu[i];
-    seg_len[rank] = Li;
+    for (int r = threadIdx.x; r < B; r += kSchedThreads) {
+      const int i = static_cast<int>(sort_keys[r] & 0xffffffffu);
+      seg_start[r] = cu[i];
+      seg_len[r] = cu[i + 1] - cu[i];
+    }
+  } else {
+    // the given order
+    for (int i = threadIdx.x; i < B; i += kSchedThreads) {
+      seg_start[i] = cu[i];
+      seg_len[i] = cu[i + 1] - cu[i];
+    }
   }
   __syncthreads();
   // exclusive prefix of tiles per request in schedule order, one chunk of
@@ -231,6 +302,7 @@ __global__ void __launch_bounds__(kSchedThreads) build_schedule_kernel(const int
     tile_start[B] = carry;
     sched[0] = carry;
     sched[1] = B;
+    sched[2] = 0;  // claim counter
   }
 }
 
@@ -369,6 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto p_full = [&](int i) { return q_full + 32 + 8u * i; };
   auto o_done = [&](int i) { return q_full + 48 + 8u * i; };
   const uint32_t drain = q_full + 64;
+  auto work_full = [&](int i) { return q_full + 72 + 8u * i; };
+  volatile int* work_slot = reinterpret_cast<volatile int*>(smem + L::kWorkOff);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
   volatile uint8_t* votes = smem + L::kVoteOff;
@@ -386,6 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(o_done(i), 1);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < kWorkSlots; ++i) mbar_init(work_full(i), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -403,18 +478,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const int n_work = p.sched[0];
-  // copies issued by the producer thread (K/V stages, Q tile pairs), for the drain
-  uint32_t load_idx = 0;
-  uint32_t q_loads = 0;
+  int* claim_counter = const_cast<int*>(p.sched + 2);
+  // copies issued by the producer thread (K/V stages, Q tile pairs), kept in
+  // shared memory for the drain so that no other thread holds them
+  volatile uint32_t* loads_done = reinterpret_cast<volatile uint32_t*>(smem + L::kLoadsOff);
+  // The index of this block's work tile wt, published by the producer in
+  // slot wt % kWorkSlots (-1 once the list is exhausted); false when the
+  // block aborts first.
+  auto next_work = [&](int wt, int& w) {
+    if (!mbar_wait(work_full(wt % kWorkSlots), (wt / kWorkSlots) & 1, abort_flag, p.timeout_ns)) return false;
+    w = work_slot[wt % kWorkSlots];
+    return true;
+  };
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      int wt = 0;
+      uint32_t load_idx = 0;
+      uint32_t q_loads = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
-        const Work wk = decode_work(p.sched, p.H, w);
+      for (int wt = 0; ok; ++wt) {
+        // the Q tiles of the previous work tile are no longer needed: claim the next one
         if (wt > 0 && !(ok = mbar_wait(q_empty, (wt - 1) & 1, abort_flag, p.timeout_ns))) break;
+        const int claimed = atomicAdd(claim_counter, 1);
+        const int w = claimed < n_work ? claimed : -1;
+        work_slot[wt % kWorkSlots] = w;
+        mbar_arrive(work_full(wt % kWorkSlots));
+        if (w < 0) break;
+        const Work wk = decode_work(p.sched, p.H, w);
         mbar_arrive_expect_tx(q_full, 2 * kQKBytes);
         ++q_loads;
         for (int i = 0; i < 2; ++i) {
@@ -448,6 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) raise_abort(abort_flag, p.status);
+      loads_done[0] = load_idx;
+      loads_done[1] = q_loads;
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer
@@ -513,7 +606,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait_stage = [&](uint32_t idx) {
         return mbar_wait(kv_full(idx % L::kStages), (idx / L::kStages) & 1, abort_flag, p.timeout_ns);
       };
-      for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
+      for (;; ++wt) {
+        int w;
+        if (!(ok = next_work(wt, w)) || w < 0) break;
         const Work wk = decode_work(p.sched, p.H, w);
         const bool q1_in_request = wk.q0 + kBM < wk.seg_start + wk.seg_len;
         if (!(ok = mbar_wait(q_full, wt & 1, abort_flag, p.timeout_ns))) break;
@@ -595,7 +690,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int wt = 0;
     bool ok = true;
     unsigned long long warp_skips = 0;
-    for (int w = blockIdx.x; w < n_work && ok; w += gridDim.x, ++wt) {
+    for (;; ++wt) {
+      int w;
+      ok = __all_sync(0xffffffffu, next_work(wt, w));
+      if (!ok || w < 0) break;
       const Work wk = decode_work(p.sched, p.H, w);
       const int row = wk.q0 + grp * kBM + r;
       // log2-domain score factor; FP8 scores carry the two heads' dequantisation factors
@@ -700,20 +798,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // and MMAs may still be in flight into this block's shared and tensor
   // memory: wait for all of them before the memory is freed.
   if (*abort_flag) {
-    if (warp == kProducerWarp && lane == 0) {
-      // the producer issued K/V copy idx only after copy idx - kStages had
-      // landed, so the last kStages copies (and the last Q pair) are the
-      // ones that can be outstanding; each is the newest phase of its stage
-      const uint32_t first = load_idx > static_cast<uint32_t>(L::kStages) ? load_idx - L::kStages : 0;
-      for (uint32_t idx = first; idx < load_idx; ++idx)
-        mbar_drain_wait(kv_full(idx % L::kStages), (idx / L::kStages) & 1);
-      if (q_loads > 0) mbar_drain_wait(q_full, (q_loads - 1) & 1);
-    } else if (warp == kMmaWarp && lane == 0) {
-      // a commit on the drain barrier completes once every MMA this thread
-      // issued has (and with them the arrivals of their own commits)
-      tc_commit(drain);
-      mbar_drain_wait(drain, 0);
-    }
+    if (warp == kProducerWarp && lane == 0)
+      drain_copies(kv_full(0), q_full, L::kStages, loads_done[0], loads_done[1]);
+    else if (warp == kMmaWarp && lane == 0)
+      drain_mmas(drain);
     __syncthreads();
   }
   tc_fence_after_sync();
@@ -785,6 +873,19 @@ bool make_e4m3_map(CUtensorMap* map, const void* ptr, int64_t T, int H, int D, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool set_schedule_smem_attr() {
+  static int done[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(build_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSchedSmem) !=
+        cudaSuccess)
+      return false;
+    done[dev] = 1;
+  }
+  return true;
+}
+
 template <int D, bool kSkip, bool kFp8, bool kFp8Pv>
 bool set_smem_attr() {
   static int done[64] = {0};
@@ -815,7 +916,11 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
   const bool v_ok = fp8_pv ? make_e4m3_map(&tv, v, T, H, D, v_stride) : make_qkv_map(&tv, v, T, H, D, v_stride);
   if (!maps_ok || !v_ok) return -2;
   int32_t* sched = static_cast<int32_t*>(workspace);
-  build_schedule_kernel<<<1, kSchedThreads, 0, stream>>>(cu_seqlens, B, T, H, sched, status);
+  int sort_n = 1;
+  while (sort_n < B) sort_n <<= 1;
+  const size_t sched_smem = B <= kSortLimit ? static_cast<size_t>(sort_n) * 8 : 0;
+  if (sched_smem > 48 * 1024 && !set_schedule_smem_attr()) return -1;
+  build_schedule_kernel<<<1, kSchedThreads, sched_smem, stream>>>(cu_seqlens, B, T, H, sched, status);
   if (cudaGetLastError() != cudaSuccess) return -1;
   AttnParams p;
   p.o = static_cast<__nv_bfloat16*>(o);

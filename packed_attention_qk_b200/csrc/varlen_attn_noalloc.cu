@@ -14,8 +14,9 @@
 // Limits and sharing: the array holds the schedule of at most
 // kNoAllocMaxRequests requests; larger B is rejected. Every call uses the
 // same array and leaves its own schedule in it; the schedule kernel rewrites
-// every word the attention kernel reads before it reads it, so nothing has
-// to start at zero. Two calls whose work overlaps on the GPU (for example on
+// every word the attention kernel reads before it reads it, and resets the
+// one word that must start at zero (the counter the attention's blocks claim
+// work tiles with), so the previous call's contents never matter. Two calls whose work overlaps on the GPU (for example on
 // two streams) race on the array and may produce wrong output: serialise
 // them.
 #include <cuda_runtime.h>
@@ -29,9 +30,10 @@
 namespace {
 
 constexpr int kNoAllocMaxRequests = 4096;
-// words of the schedule for kNoAllocMaxRequests requests (3B + 3), rounded
-// up to 256 bytes like the workspace size query
-constexpr size_t kScratchWords = ((3 * static_cast<size_t>(kNoAllocMaxRequests) + 3) * 4 + 255) / 256 * 64;
+// words of the schedule for kNoAllocMaxRequests requests (3B + 5: a header
+// of 4 words, B + 1 tile offsets, 2B request words), rounded up to 256 bytes
+// like the workspace size query
+constexpr size_t kScratchWords = ((3 * static_cast<size_t>(kNoAllocMaxRequests) + 5) * 4 + 255) / 256 * 64;
 
 static __device__ __align__(256) int32_t g_noalloc_schedule[kScratchWords];
 

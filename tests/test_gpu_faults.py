@@ -100,12 +100,19 @@ def test_attention_pipeline_timeout_is_reported_drained_and_recovered():
 
 
 def test_linear_pipeline_timeout_is_reported_drained_and_recovered():
+    # K = 16,384: each output tile's main loop runs for tens of microseconds,
+    # so the epilogue's wait for a finished accumulator outlasts the 1 us bound
     torch = torch_cuda()
-    w = wl.config(2)                       # 4,096 tokens, hidden 2,048
-    d = wl.linear_inputs(w, "o_proj")
-    T, N = w.T, w.C
-    a, wt, x = to_dev_bf16(d["a"]), to_dev_bf16(d["w"]), to_dev_bf16(d["x"])
-    gr, cu = to_dev(d["gate_res"]), to_dev(d["cu_seqlens"])
+    g = np.random.default_rng(71)
+    lens, K, N = [1500, 0, 548], 16384, 2048
+    T = sum(lens)
+    a_bits = wl.f32_to_bf16_bits(g.standard_normal((T, K)).astype(np.float32))
+    w_bits = wl.f32_to_bf16_bits((g.standard_normal((N, K)) / np.sqrt(K)).astype(np.float32))
+    x_bits = wl.f32_to_bf16_bits(g.standard_normal((T, N)).astype(np.float32))
+    gate_res = (0.1 * g.standard_normal((len(lens), N))).astype(np.float32)
+    cu_np = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    a, wt, x = to_dev_bf16(a_bits), to_dev_bf16(w_bits), to_dev_bf16(x_bits)
+    gr, cu = to_dev(gate_res), to_dev(cu_np)
     out_full = torch.full((T + 16, N + 64), 7.0, dtype=torch.bfloat16, device="cuda")
     out = out_full[8:8 + T, :N]
     assert _runs_out(lambda: pqk.linear_gated_residual(a, wt, x=x, gate_res=gr, cu_seqlens=cu, out=out))
@@ -114,8 +121,9 @@ def test_linear_pipeline_timeout_is_reported_drained_and_recovered():
     y = pqk.linear_gated_residual(a, wt, x=x, gate_res=gr, cu_seqlens=cu)
     torch.cuda.synchronize()
     assert pqk.get_device_status() == 0
-    rows = wl.sample_rows(w, 64)
-    ref = oracle.linear_gated_residual(d["a"], d["w"], d["x"], d["gate_res"], d["cu_seqlens"], rows=rows)
+    rows = np.array(sorted({0, 1, 255, 256, 1499, 1500, 1501, 2047} | set(g.choice(T, 40, replace=False).tolist())),
+                    np.int32)
+    ref = oracle.linear_gated_residual(a_bits, w_bits, x_bits, gate_res, cu_np, rows=rows)
     assert_elementwise(bf16_to_f64(y)[rows], ref, "linear layer after a timed-out call")
 
 
