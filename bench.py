@@ -19,7 +19,8 @@ scaling, no collective on the data path.
 After the timed steps the same line also carries, under ``kernels``: the
 three-axis RoPE, back-to-back and full-width norm timings; the block-
 skipping attention on the local-attention stand-in (``--skip-tau``, plain
-vs skipping vs FP8 Q K^T with and without skipping); the FP8 Q K^T attention
+vs skipping vs FP8 Q K^T and the whole attention in FP8, each with and
+without skipping); the FP8 Q K^T attention
 on the step's inputs (``--no-fp8`` leaves it out); the block's three linear
 layers with the gated residual or SwiGLU in the GEMM epilogue, on the step's
 own activations, against cuBLAS plus torch epilogues (``linear_epilogue``;
@@ -606,15 +607,29 @@ def run_ours(args, w):
             fp8_plain()
             fp8_skip()
             torch.cuda.synchronize()
-            for name, fn in (("fp8", fp8_plain), ("fp8_skip", fp8_skip), ("fp8_2", fp8_plain),
-                             ("fp8_skip_2", fp8_skip)):
+            # the whole computation in FP8 (V and P too), without and with skipping
+            lv8, ldeq_v = pqk.quantize_e4m3(lv)
+            ldeq3 = torch.cat([deq, ldeq_v]).contiguous()
+            full_plain = lambda: pqk.varlen_attn_fwd_fp8(q8, k8, lv8, ldeq3, d["cu"], o=lo, workspace=o["ws"])
+            full_skip = lambda: pqk.varlen_attn_fwd_fp8(q8, k8, lv8, ldeq3, d["cu"], o=lo, workspace=o["ws"],
+                                                        skip_threshold_log2=args.skip_tau)
+            fp8_plain()
+            fp8_skip()
+            full_plain()
+            full_skip()
+            torch.cuda.synchronize()
+            for name, fn in (("fp8", fp8_plain), ("fp8_skip", fp8_skip), ("full", full_plain),
+                             ("full_skip", full_skip), ("fp8_2", fp8_plain), ("fp8_skip_2", fp8_skip),
+                             ("full_2", full_plain), ("full_skip_2", full_skip)):
                 ev3[0].record()
                 for _ in range(3):
                     fn()
                 ev3[1].record()
                 torch.cuda.synchronize()
                 fp8_times[name] = ev3[0].elapsed_time(ev3[1]) / 3
-            del q8, k8
+            if pqk.get_device_status() != 0:
+                raise RuntimeError("device status set during the FP8 block-skipping timing")
+            del q8, k8, lv8
         c = counts.cpu().tolist()
         n32 = sum(((L + 31) // 32) * ((L + 127) // 128) for L in w.seg_lens) * w.H
         n128 = sum(((L + 127) // 128) ** 2 for L in w.seg_lens) * w.H
@@ -628,7 +643,11 @@ def run_ours(args, w):
         if fp8_times:
             f_ms = min(fp8_times["fp8"], fp8_times["fp8_2"])
             fs_ms = min(fp8_times["fp8_skip"], fp8_times["fp8_skip_2"])
-            skip.update({"fp8qk_ms": f_ms, "fp8qk_skip_ms": fs_ms, "speedup_fp8qk_skip_vs_plain": plain_ms / fs_ms})
+            ff_ms = min(fp8_times["full"], fp8_times["full_2"])
+            ffs_ms = min(fp8_times["full_skip"], fp8_times["full_skip_2"])
+            skip.update({"fp8qk_ms": f_ms, "fp8qk_skip_ms": fs_ms, "speedup_fp8qk_skip_vs_plain": plain_ms / fs_ms,
+                         "full_fp8_ms": ff_ms, "full_fp8_skip_ms": ffs_ms,
+                         "speedup_full_fp8_skip_vs_plain": plain_ms / ffs_ms})
         del lq, lk, lv, lo, lx
 
     # FP8 Q K^T (the SAGE reading): the step's normalised Q, K quantised per

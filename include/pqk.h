@@ -278,23 +278,32 @@ PQK_API int pqk_quantize_e4m3(const void* x, int64_t x_stride_t, int64_t T, int 
 /*
  * pqk_varlen_attn_fwd_fp8 -- the whole attention computation in FP8 (SAGE
  * quantises the attention computation to FP8: first page, bullet on
- * TRTLLM_ATTN SAGE and Skip-Softmax). Q, K, V are e4m3 per head
- * (pqk_quantize_qk_e4m3, pqk_quantize_e4m3); S = Q K^T and O += P V both
- * run on the FP8 tensor cores. Per row, over key blocks of 128 keys counted
- * from the request's first token, with u = s / ln 2 (s from the dequantised
- * Q, K): the running maximum m (log2 units) is set by the first block and
- * moves only when a block's maximum exceeds it by more than 8, the sums then
- * scaling by 2^(m_old - m_new); each key adds p = 2^(u - m) <= 256 to the
- * denominator and e4m3(p) * V~ to the numerator; O = numerator / denominator
- * rounded to bf16, lse = (m + log2 denominator) ln 2.
+ * TRTLLM_ATTN SAGE and Skip-Softmax), optionally with block skipping
+ * (Skip-Softmax: the same bullet, and the second page's bullet "Sparse &
+ * quantized attention", which credits the two together). Q, K, V are e4m3
+ * per head (pqk_quantize_qk_e4m3, pqk_quantize_e4m3); S = Q K^T and
+ * O += P V both run on the FP8 tensor cores. With u = s / ln 2 (s from the
+ * dequantised Q, K), the probabilities are formed by an online softmax over
+ * key blocks of 128 keys counted from the request's first token: the
+ * running maximum m (log2 units) is set by the first block and moves only
+ * when a block's maximum exceeds it by more than 8, the sums then scaling by
+ * 2^(m_old - m_new); each key adds p = 2^(u - m) <= 256 to the denominator
+ * and e4m3(p) * V~ to the numerator; O = numerator / denominator rounded to
+ * bf16, lse = (m + log2 denominator) ln 2. Rounding p against the running
+ * maximum rather than the row's final one changes each numerator term by
+ * at most one e4m3 step (2^-3 of p, or 2^-9 below e4m3's normal range).
  *
  * q8, k8, v8  device e4m3 [T, H, D] bytes, contiguous, 16-byte aligned.
  * deq         device fp32 [3H]: Q's, K's, then V's dequantisation factors.
+ * skip_threshold_log2, skip_counts: block skipping as pqk_varlen_attn_fwd_skip,
+ *             decided on the FP8 scores; dropped keys take no part in the
+ *             sums or the maximum; +inf skips nothing (and counts nothing).
  * o, lse, cu_seqlens, workspace: as pqk_varlen_attn_fwd. D must be 128.
  */
 PQK_API int pqk_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* deq, void* o,
                             float* lse, int64_t o_stride_t, const int32_t* cu_seqlens, int B, int64_t T,
-                            int H, int D, float softmax_scale, void* workspace, size_t workspace_bytes,
+                            int H, int D, float softmax_scale, float skip_threshold_log2,
+                            unsigned long long* skip_counts, void* workspace, size_t workspace_bytes,
                             void* stream);
 
 /*

@@ -288,17 +288,19 @@ int pqk_quantize_e4m3(const void* x, int64_t x_stride_t, int64_t T, int H, int D
 
 int pqk_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* deq, void* o, float* lse,
                             int64_t o_stride_t, const int32_t* cu_seqlens, int B, int64_t T, int H, int D,
-                            float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+                            float softmax_scale, float skip_threshold_log2, unsigned long long* skip_counts,
+                            void* workspace, size_t workspace_bytes, void* stream) {
   if (B < 1 || T < 0 || H <= 0 || T > INT32_MAX - 512 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     return PQK_ERR_INVALID_ARG;
   if (!attn_tiles_fit(T, B, H)) return PQK_ERR_INVALID_ARG;
+  if (!(skip_threshold_log2 >= 0.f)) return PQK_ERR_INVALID_ARG;
   if (D != 128) return PQK_ERR_UNSUPPORTED;
   const int64_t row = static_cast<int64_t>(H) * D;
   if (o_stride_t < row) return PQK_ERR_INVALID_ARG;
   if (T == 0) return PQK_OK;
   if (!q8 || !k8 || !v8 || !deq || !o || !cu_seqlens) return PQK_ERR_INVALID_ARG;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || !aligned16(lse) ||
-      (reinterpret_cast<uintptr_t>(deq) % 4) || (o_stride_t % 8))
+      (reinterpret_cast<uintptr_t>(deq) % 4) || (o_stride_t % 8) || (reinterpret_cast<uintptr_t>(skip_counts) % 8))
     return PQK_ERR_MISALIGNED;
   if (workspace == nullptr || workspace_bytes < pqk_varlen_attn_workspace_size(B)) return PQK_ERR_WORKSPACE;
   if (!aligned16(workspace)) return PQK_ERR_MISALIGNED;
@@ -306,7 +308,8 @@ int pqk_varlen_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, cons
   if (int rc = check_device(&d)) return rc;
   const int rc = pqk::launch_varlen_attn(q8, k8, v8, o, lse, row, row, row, o_stride_t, cu_seqlens, B, T, H, D,
                                          softmax_scale, workspace, d->status, g_timeout_ns.load(),
-                                         static_cast<cudaStream_t>(stream), d->num_sms, false, 0.0f, nullptr, deq,
+                                         static_cast<cudaStream_t>(stream), d->num_sms,
+                                         std::isfinite(skip_threshold_log2), skip_threshold_log2, skip_counts, deq,
                                          true);
   return rc == 0 ? PQK_OK : (rc == -2 ? PQK_ERR_INVALID_ARG : PQK_ERR_CUDA);
 }

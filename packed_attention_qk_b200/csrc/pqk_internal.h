@@ -36,7 +36,7 @@ size_t attn_schedule_bytes(int B);
 // with Q, K given as e4m3 bytes ([T, H, D], strides in bytes) and deq their
 // [2H] per-head dequantisation factors (D = 128; skipping may be combined
 // with it). fp8_pv: V is e4m3 bytes too and P is rounded to e4m3 for P V
-// (deq then [3H], V's last; no skipping). Returns 0, or
+// (deq then [3H], V's last; skipping may be combined with it too). Returns 0, or
 // -1 when a CUDA call failed, -2 when the tensor maps could not be encoded.
 int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, float* lse, int64_t q_stride,
                        int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,

@@ -59,7 +59,10 @@
 //          O_i += P_i V_j when all four warps of the group voted so;
 //   kFp8   Q and K as e4m3 bytes (SAGE FP8): S_i = Q_i K^T from 16 KB tiles
 //          with kind::f8f6f4 MMAs, the heads' dequantisation factors folded
-//          into the softmax scale.
+//          into the softmax scale;
+//   kFp8Pv V as e4m3 bytes too and P rounded to e4m3 in tensor memory, so
+//          that O_i += P_i V_j runs on the FP8 tensor cores as well; it
+//          combines with kSkip (SAGE FP8 with Skip-Softmax).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -414,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using L = Layout<D>;
   static_assert(!kFp8 || D == 128, "FP8 Q K^T: one 128-byte swizzle row per token");
-  static_assert(!kFp8Pv || (kFp8 && !kSkip), "FP8 P V comes with FP8 Q K^T, without block skipping");
+  static_assert(!kFp8Pv || kFp8, "FP8 P V comes with FP8 Q K^T");
   // FP8 Q K^T: the MMA thread waits for the next V stage (loaded long ago)
   // while it waits for P1 anyway, and probes the next K stage there without
   // blocking (its copy may still be in flight), instead of waiting for both
@@ -721,11 +724,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) votes[(grp * 2 + (j & 1)) * 4 + (warp & 3)] = skip ? 1 : 0;
           if (skip) {
             if (__any_sync(0xffffffffu, in_request) && lane == 0) ++warp_skips;
-            // P = 0 for these rows (the product still runs if another warp keeps the tile)
-            uint32_t zero[64];
+            // P = 0 for these rows (the product still runs if another warp
+            // keeps the tile): 64 columns of bf16 pairs, or 32 of e4m3 quads
+            if constexpr (kFp8Pv) {
+              uint32_t zero[32];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) zero[c] = 0u;
-            tmem_st_x64(t_s, zero);
+              for (int c = 0; c < 32; ++c) zero[c] = 0u;
+              tmem_st_x32(t_s, zero);
+            } else {
+              uint32_t zero[64];
+#pragma unroll
+              for (int c = 0; c < 64; ++c) zero[c] = 0u;
+              tmem_st_x64(t_s, zero);
+            }
             tc_fence_before_sync();
             mbar_arrive(p_full(grp));
             continue;
@@ -744,15 +755,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tile j completed after them): rescale it before P_j V_j. Tensor-
         // memory loads and stores are warp-collective (.sync.aligned), so
         // the whole warp takes this path when any of its rows needs it, the
-        // other rows with alpha = 1.
+        // other rows with alpha = 1. Eight columns at a time in a rolled
+        // loop: the 128 scores are live here, and wider chunks push the
+        // kernel past its register budget (spills in every variant).
         if (__any_sync(0xffffffffu, need_rescale)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 8) {
+            uint32_t ov[8];
+            tmem_ld_x8(t_o + c0, ov);
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t ov[32];
-            tmem_ld_x32(t_o + c0, ov);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-            tmem_st_x32(t_o + c0, ov);
+            for (int c = 0; c < 8; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+            tmem_st_x8(t_o + c0, ov);
           }
         }
         l += exp_tile_store<kFp8Pv>(s, sl2, -m, t_s);
@@ -938,10 +951,14 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
   // upper bound of work tiles: every request adds at most one partial block
   const int64_t max_work = static_cast<int64_t>(H) * ((T + kRowsPerWork - 1) / kRowsPerWork + B);
   const int grid = static_cast<int>(max_work < num_sms ? max_work : num_sms);
-  if (fp8_pv) {
-    if (D != 128 || deq == nullptr || skip) return -1;
+  if (fp8_pv && !skip) {
+    if (D != 128 || deq == nullptr) return -1;
     if (!set_smem_attr<128, false, true, true>()) return -1;
     attn_fwd_kernel<128, false, true, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+  } else if (fp8_pv) {
+    if (D != 128 || deq == nullptr) return -1;
+    if (!set_smem_attr<128, true, true, true>()) return -1;
+    attn_fwd_kernel<128, true, true, true><<<grid, kThreads, Layout<128>::kAlloc, stream>>>(tq, tk, tv, p);
   } else if (deq != nullptr && !skip) {
     if (D != 128) return -1;
     if (!set_smem_attr<128, false, true, false>()) return -1;

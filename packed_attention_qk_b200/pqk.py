@@ -72,7 +72,8 @@ def lib(path: str | None = None) -> C.CDLL:
     L.pqk_varlen_attn_fwd_fp8qk.restype = i32
     L.pqk_quantize_e4m3.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp]
     L.pqk_quantize_e4m3.restype = i32
-    L.pqk_varlen_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, i32, i64, i32, i32, f32, vp, sz, vp]
+    L.pqk_varlen_attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i64, vp, i32, i64, i32, i32, f32, f32, vp, vp, sz,
+                                          vp]
     L.pqk_varlen_attn_fwd_fp8.restype = i32
     L.pqk_varlen_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, i64, i32, i32, f32,
                                               vp]
@@ -289,10 +290,12 @@ def quantize_e4m3(x, *, x8=None, scales=None, stream=None):
 
 
 def varlen_attn_fwd_fp8(q8, k8, v8, deq, cu_seqlens, *, softmax_scale: float | None = None, o=None, lse=None,
-                        workspace=None, want_lse: bool = False, stream=None):
+                        workspace=None, want_lse: bool = False, skip_threshold_log2: float = math.inf,
+                        skip_counts=None, stream=None):
     """The attention with Q K^T and P V on the FP8 tensor cores: q8, k8, v8
-    e4m3 bytes [T, H, D]; deq fp32 [3H] (Q's, K's, V's factors). Returns
-    (o bf16 [T, H, D], lse or None)."""
+    e4m3 bytes [T, H, D]; deq fp32 [3H] (Q's, K's, V's factors). A finite
+    skip_threshold_log2 adds block skipping (skip_counts as in
+    varlen_attn_fwd_skip). Returns (o bf16 [T, H, D], lse or None)."""
     import torch
     T, H, D = q8.shape
     B = cu_seqlens.shape[0] - 1
@@ -306,9 +309,12 @@ def varlen_attn_fwd_fp8(q8, k8, v8, deq, cu_seqlens, *, softmax_scale: float | N
     for t in (q8, k8, v8):
         assert t.is_contiguous() and tuple(t.shape) == (T, H, D)
     assert deq.is_contiguous() and deq.numel() >= 3 * H
+    if skip_counts is not None:
+        assert skip_counts.dtype == torch.int64 and skip_counts.numel() >= 2 and skip_counts.is_contiguous()
     _check("pqk_varlen_attn_fwd_fp8", lib().pqk_varlen_attn_fwd_fp8(
         _ptr(q8), _ptr(k8), _ptr(v8), _ptr(deq), _ptr(o), _ptr(lse), _token_stride(o, 3), _ptr(cu_seqlens), B, T, H,
-        D, scale, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+        D, scale, float(skip_threshold_log2), _ptr(skip_counts), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
     return o, lse
 
 

@@ -153,7 +153,8 @@ def test_attention_rejects_more_work_tiles_than_32_bits_count(L):
                                       8.0, None, A, 4096, None) == ERR_INVALID
     assert L.pqk_varlen_attn_fwd_fp8qk(A, A, A, A, A, None, H * 128, H * 128, A, 1, T, H, 128, 0.1,
                                        float("inf"), None, A, 4096, None) == ERR_INVALID
-    assert L.pqk_varlen_attn_fwd_fp8(A, A, A, A, A, None, H * 128, A, 1, T, H, 128, 0.1, A, 4096, None) == ERR_INVALID
+    assert L.pqk_varlen_attn_fwd_fp8(A, A, A, A, A, None, H * 128, A, 1, T, H, 128, 0.1, float("inf"), None, A, 4096,
+                                     None) == ERR_INVALID
     # (the no-allocation entry looks up its device array first and then forwards to pqk_varlen_attn_fwd, so the
     # same check applies to it on a GPU; without one it stops at the lookup)
 
@@ -250,16 +251,20 @@ def test_quantize_e4m3_and_fp8_attention_host_errors(L):
     assert L.pqk_quantize_e4m3(A, 1024, 16, 8, 128, A, None, None) == ERR_INVALID
 
     def call(**kw):
-        a = dict(q8=A, k8=A, v8=A, deq=A, o=A, lse=None, os_=1024, cu=A, B=2, T=512, H=8, D=128, scale=0.088, ws=A,
-                 wsb=4096)
+        a = dict(q8=A, k8=A, v8=A, deq=A, o=A, lse=None, os_=1024, cu=A, B=2, T=512, H=8, D=128, scale=0.088,
+                 tau=float("inf"), counts=None, ws=A, wsb=4096)
         a.update(kw)
         return L.pqk_varlen_attn_fwd_fp8(a["q8"], a["k8"], a["v8"], a["deq"], a["o"], a["lse"], a["os_"], a["cu"],
-                                         a["B"], a["T"], a["H"], a["D"], a["scale"], a["ws"], a["wsb"], None)
+                                         a["B"], a["T"], a["H"], a["D"], a["scale"], a["tau"], a["counts"], a["ws"],
+                                         a["wsb"], None)
     assert call(D=64, os_=512) == ERR_UNSUPPORTED
     assert call(v8=None) == ERR_INVALID
     assert call(v8=U) == ERR_MISALIGNED
     assert call(os_=512) == ERR_INVALID
     assert call(ws=None) == ERR_WORKSPACE
+    assert call(tau=-1.0) == ERR_INVALID
+    assert call(tau=float("nan")) == ERR_INVALID
+    assert call(tau=8.0, counts=A + 4) == ERR_MISALIGNED
     assert call(T=0, q8=None) == 0
 
 

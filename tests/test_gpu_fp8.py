@@ -180,15 +180,17 @@ def test_joint_sequence_58048_sampled():
 
 # ---------------------------------------------------------------- Q, K, V and P in FP8
 
-def _full_fp8_gpu(x, scale):
+def _full_fp8_gpu(x, scale, tau=math.inf):
     torch = torch_cuda()
     q8, k8, deq_qk = _quantise_gpu(x)
     v8, deq_v = pqk.quantize_e4m3(to_dev_bf16(x["v"]))
     deq = torch.cat([deq_qk, deq_v]).contiguous()
-    o, lse = pqk.varlen_attn_fwd_fp8(q8, k8, v8, deq, to_dev(x["cu_seqlens"]), softmax_scale=scale, want_lse=True)
+    c = torch.zeros(2, dtype=torch.int64, device="cuda")
+    o, lse = pqk.varlen_attn_fwd_fp8(q8, k8, v8, deq, to_dev(x["cu_seqlens"]), softmax_scale=scale, want_lse=True,
+                                     skip_threshold_log2=tau, skip_counts=c)
     torch.cuda.synchronize()
     assert pqk.get_device_status() == 0
-    return o, lse, v8, deq
+    return o, lse, v8, deq, tuple(int(a) for a in c.cpu())
 
 
 # The whole-FP8 kernel is an online softmax over K/V tiles of 128 keys whose
@@ -208,11 +210,34 @@ def _e4m3_quantum(p):
     return np.exp2(e - 3)
 
 
-def _row_terms(qd, kd, scale, lo, hi, t, h):
-    """For row t, head h over keys [lo, hi): the probabilities p_j against
-    the row's exact maximum, and c_j = 2^(M - m_j), where m_j is the kernel's
-    running maximum when key j's tile is visited (c_j >= 1)."""
+def _kept_keys(qd, kd, scale, lo, hi, t, h, tau):
+    """Keys of row t's request kept by the block-skipping rule (32-row query
+    blocks x 128-key blocks counted from the request's first token, decided
+    in float64 on the dequantised scores); all of them for tau = inf."""
+    L = hi - lo
+    if math.isinf(tau):
+        return np.ones(L, bool)
+    qr, kb = SKIP_BLOCK
+    r0 = lo + (t - lo) // qr * qr
+    r1 = min(hi, r0 + qr)
+    u = scale * (qd[r0:r1, h] @ kd[lo:hi, h].T) / math.log(2.0)
+    nkb = (L + kb - 1) // kb
+    pad = np.full((r1 - r0, nkb * kb), -np.inf)
+    pad[:, :L] = u
+    tmax = pad.reshape(r1 - r0, nkb, kb).max(axis=2)
+    prev = np.maximum.accumulate(tmax, axis=1)
+    drop = np.zeros(nkb, bool)
+    drop[1:] = np.all(tmax[:, 1:] < prev[:, :-1] - tau, axis=0)
+    return np.repeat(~drop, kb)[:L]
+
+
+def _row_terms(qd, kd, scale, lo, hi, t, h, keep):
+    """For row t, head h over the kept keys of [lo, hi): the probabilities p_j
+    against the maximum over those keys, and c_j = 2^(M - m_j), where m_j is
+    the kernel's running maximum when key j's tile is visited (c_j >= 1;
+    dropped tiles do not move it). p is 0 at dropped keys."""
     u = scale * (kd[lo:hi, h] @ qd[t, h]) / math.log(2.0)
+    u = np.where(keep, u, -np.inf)
     M = u.max()
     m_at = np.empty_like(u)
     m = -np.inf
@@ -224,7 +249,7 @@ def _row_terms(qd, kd, scale, lo, hi, t, h):
     return np.exp2(u - M), np.exp2(M - m_at)
 
 
-def _check_full_fp8(x, scale, what, rows=None, peaked=False):
+def _check_full_fp8(x, scale, what, rows=None, peaked=False, tau=math.inf):
     """Element-wise against the oracle, twice.
 
     (1) The definition (oracle.varlen_attn_fp8: each probability p_j <= 1
@@ -242,14 +267,25 @@ def _check_full_fp8(x, scale, what, rows=None, peaked=False):
     inputs the unit-scale bound) plus, per row, one e4m3 step of each key
     whose probability lies within 2^-10 (relative) of an e4m3 rounding
     midpoint: the kernel rounds fp32 probabilities and the oracle float64
-    ones, so only those keys can round differently."""
-    o, lse, v8, deq = _full_fp8_gpu(x, scale)
+    ones, so only those keys can round differently.
+
+    With a finite tau (block skipping) both sides drop the same key blocks
+    (the callers check that no decision lies near the threshold), the sums
+    run over the kept keys, and the skip counts must be equal."""
+    o, lse, v8, deq, counts = _full_fp8_gpu(x, scale, tau)
     T, H, D = x["q"].shape
     sel = np.arange(T) if rows is None else rows
-    rd, rld, rdeq = oracle.varlen_attn_fp8(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, rows=rows)
+    kw = {} if math.isinf(tau) else {"tau": tau, "skip_block": SKIP_BLOCK, "skip_tile_rows": SKIP_TILE_ROWS}
+    c_def, c_sch = [], []
+    rd, rld, rdeq = oracle.varlen_attn_fp8(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, rows=rows,
+                                           counts_out=c_def, **kw)
     rs, rls, _ = oracle.varlen_attn_fp8_online(x["q"], x["k"], x["v"], x["cu_seqlens"], scale, kblock=KERNEL_KBLOCK,
-                                               threshold=KERNEL_THRESHOLD, rows=rows)
+                                               threshold=KERNEL_THRESHOLD, rows=rows, counts_out=c_sch, **kw)
     assert np.array_equal(deq.cpu().numpy(), rdeq)
+    if math.isinf(tau):
+        assert counts == (0, 0)
+    elif rows is None:
+        assert c_def == c_sch == [counts], f"{what}: skip counts {counts} vs oracle {c_def}"
     g = bf16_to_f64(o)[sel]
     assert rel_l2(g, rs) <= ATTN_REL_L2, f"{what}: rel-L2 {rel_l2(g, rs):.3e} against the kernel's schedule"
     qd, kd, vd = (_decode(c) * dq[None, :, None]
@@ -259,18 +295,19 @@ def _check_full_fp8(x, scale, what, rows=None, peaked=False):
         i = int(np.searchsorted(cu, t, side="right") - 1)
         lo, hi = int(cu[i]), int(cu[i + 1])
         for h in range(H):
-            p, c = _row_terms(qd, kd, scale, lo, hi, t, h)
+            keep = _kept_keys(qd, kd, scale, lo, hi, t, h, tau)
+            p, c = _row_terms(qd, kd, scale, lo, hi, t, h, keep)
             l = p.sum()
             av = np.abs(vd[lo:hi, h])
             # (1) the definition
-            bound = ATTN_MAX_ABS + (np.maximum(2.0 ** -3 * p, 2.0 ** -9)[:, None] * av).sum(0) / l
+            bound = ATTN_MAX_ABS + (np.where(keep, np.maximum(2.0 ** -3 * p, 2.0 ** -9), 0.0)[:, None] * av).sum(0) / l
             err = np.abs(g[n, h] - rd[n, h])
             assert np.all(err <= bound), f"{what}: row {t} head {h}: {err.max():.3e} over the definition's bound"
             # (2) the schedule: keys near a rounding midpoint, in the frame the kernel rounds in
             ps = p * c
-            qn = _e4m3_quantum(ps)
+            qn = _e4m3_quantum(np.where(keep, ps, 1.0))
             frac = ps / qn - np.floor(ps / qn)
-            near = np.abs(frac - 0.5) * qn <= 2.0 ** -10 * ps
+            near = keep & (np.abs(frac - 0.5) * qn <= 2.0 ** -10 * ps)
             slack = (near[:, None] * (qn / c)[:, None] * av).sum(0) / l
             err = np.abs(g[n, h] - rs[n, h])
             tol = ELEM_UNIT_MAX * np.maximum(1.0, np.abs(rs[n, h])) if peaked else ATTN_MAX_ABS
@@ -317,5 +354,40 @@ def test_full_fp8_attention_is_deterministic():
     w = wl.custom([1000, 2000], 4, 128, seed=46)
     x = wl.attention_inputs(w)
     a = [_full_fp8_gpu(x, 0.1) for _ in range(3)]
-    for o, lse, _, _ in a[1:]:
+    for o, lse, _, _, _ in a[1:]:
         assert torch.equal(o.view(torch.int16), a[0][0].view(torch.int16)) and torch.equal(lse, a[0][1])
+
+
+@pytest.mark.parametrize("lens, seed", [([700, 1300, 129], 47), ([640, 0, 257, 1], 48)])
+@pytest.mark.parametrize("tau", [4.0, 8.0])
+def test_full_fp8_with_block_skipping_matches_oracle_and_counts(lens, seed, tau):
+    # SAGE FP8 with Skip-Softmax together: decisions taken on the FP8 scores
+    # (margins checked on the dequantised Q, K in float64), then every element
+    # against both oracles and the skip counts exactly
+    import torch
+    from tests.test_gpu_attention_skip import MARGIN, decision_margins
+    torch_cuda()
+    w = wl.custom(lens, 2, 128, seed=seed)
+    x = wl.block_scaled_attention_inputs(w)
+    scale = 1.0 / math.sqrt(128)
+    H = w.H
+    (q8r, dqr), (k8r, dkr) = oracle.quantize_e4m3(x["q"]), oracle.quantize_e4m3(x["k"])
+    xd = {"q": _decode(q8r) * dqr[None, :, None], "k": _decode(k8r) * dkr[None, :, None],
+          "cu_seqlens": x["cu_seqlens"]}
+    assert decision_margins(xd, tau, scale) >= MARGIN
+    _check_full_fp8(x, scale, f"full fp8 + skip tau {tau} {lens}", peaked=True, tau=tau)
+    _, _, _, _, counts = _full_fp8_gpu(x, scale, tau)
+    assert counts[0] > 0
+
+
+def test_full_fp8_skipping_with_infinite_threshold_is_bitwise_the_plain_kernel():
+    torch = torch_cuda()
+    w = wl.custom([1000, 37, 640], 2, 128, seed=49)
+    x = wl.attention_inputs(w)
+    a = _full_fp8_gpu(x, 0.1)
+    q8, k8, deq_qk = _quantise_gpu(x)
+    v8, deq_v = pqk.quantize_e4m3(to_dev_bf16(x["v"]))
+    o, lse = pqk.varlen_attn_fwd_fp8(q8, k8, v8, torch.cat([deq_qk, deq_v]).contiguous(), to_dev(x["cu_seqlens"]),
+                                     softmax_scale=0.1, want_lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o.view(torch.int16), a[0].view(torch.int16)) and torch.equal(lse, a[1])
