@@ -93,16 +93,20 @@ typedef enum { PQK_NORM_RMS = 0, PQK_NORM_LAYER = 1, PQK_NORM_NONE = 2 } pqk_nor
  *
  * q_in, k_in    device bf16 [T, H, D], q_stride_t / k_stride_t elements
  *               between consecutive tokens (>= H*D; a fused QKV row works).
- * q_out, k_out  device bf16, same layout and strides as the inputs; may
- *               equal q_in / k_in (in place).
+ * q_out, k_out  device bf16 [T, H, D] with their own token strides
+ *               q_out_stride_t / k_out_stride_t (>= H*D, multiples of 8): a
+ *               slot of a wider buffer works, such as the send buffer of a
+ *               sequence-parallel exchange; equal to q_in / k_in with equal
+ *               strides for in-place use (no other overlap allowed).
  * q_weight, k_weight  device bf16 [D], shared by all heads.
  * pos           device int32 [T], RoPE position id of every token.
  * D             64 or 128. T >= 0 (T == 0 enqueues nothing). eps > 0.
  */
 PQK_API int pqk_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out,
-                     int64_t q_stride_t, int64_t k_stride_t, const void* q_weight,
-                     const void* k_weight, const int32_t* pos, int64_t T, int H, int D,
-                     float eps, float rope_base, int rope_style, void* stream);
+                     int64_t q_stride_t, int64_t k_stride_t, int64_t q_out_stride_t,
+                     int64_t k_out_stride_t, const void* q_weight, const void* k_weight,
+                     const int32_t* pos, int64_t T, int H, int D, float eps, float rope_base,
+                     int rope_style, void* stream);
 
 /*
  * pqk_qk_norm_rope_3axis -- pqk_qk_norm_rope with a (t, h, w) position per

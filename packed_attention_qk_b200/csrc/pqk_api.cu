@@ -102,22 +102,28 @@ void pqk_set_wait_timeout_ns(int64_t ns) {
 }
 
 int pqk_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride_t,
-                     int64_t k_stride_t, const void* q_weight, const void* k_weight, const int32_t* pos, int64_t T,
-                     int H, int D, float eps, float rope_base, int rope_style, void* stream) {
+                     int64_t k_stride_t, int64_t q_out_stride_t, int64_t k_out_stride_t, const void* q_weight,
+                     const void* k_weight, const int32_t* pos, int64_t T, int H, int D, float eps, float rope_base,
+                     int rope_style, void* stream) {
   if (T < 0 || H <= 0 || !(eps > 0.f) || !(rope_base > 0.f)) return PQK_ERR_INVALID_ARG;
   if (rope_style != PQK_ROPE_INTERLEAVED && rope_style != PQK_ROPE_HALF) return PQK_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return PQK_ERR_UNSUPPORTED;
-  if (q_stride_t < static_cast<int64_t>(H) * D || k_stride_t < static_cast<int64_t>(H) * D)
+  const int64_t row = static_cast<int64_t>(H) * D;
+  if (q_stride_t < row || k_stride_t < row || q_out_stride_t < row || k_out_stride_t < row)
     return PQK_ERR_INVALID_ARG;
   if (T == 0) return PQK_OK;
   if (!q_in || !k_in || !q_out || !k_out || !q_weight || !k_weight || !pos) return PQK_ERR_INVALID_ARG;
+  // in place needs the same layout on both sides
+  if ((q_out == q_in && q_out_stride_t != q_stride_t) || (k_out == k_in && k_out_stride_t != k_stride_t))
+    return PQK_ERR_INVALID_ARG;
   if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(q_out) || !aligned16(k_out) || !aligned16(q_weight) ||
-      !aligned16(k_weight) || (q_stride_t % 8) || (k_stride_t % 8))
+      !aligned16(k_weight) || (q_stride_t % 8) || (k_stride_t % 8) || (q_out_stride_t % 8) ||
+      (k_out_stride_t % 8))
     return PQK_ERR_MISALIGNED;
   DeviceInfo* d = nullptr;
   if (int rc = check_device(&d)) return rc;
-  return pqk::launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_stride_t, k_stride_t, q_weight, k_weight, pos,
-                                  nullptr, false, T, H, D, eps, rope_base, rope_style,
+  return pqk::launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_stride_t, k_stride_t, q_out_stride_t, k_out_stride_t,
+                                  q_weight, k_weight, pos, nullptr, false, T, H, D, eps, rope_base, rope_style,
                                   static_cast<cudaStream_t>(stream), d->num_sms)
              ? PQK_ERR_CUDA
              : PQK_OK;
@@ -141,8 +147,8 @@ int pqk_qk_norm_rope_3axis(const void* q_in, const void* k_in, void* q_out, void
   DeviceInfo* d = nullptr;
   if (int rc = check_device(&d)) return rc;
   const int sections[3] = {sec_t, sec_h, sec_w};
-  return pqk::launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_stride_t, k_stride_t, q_weight, k_weight, pos3,
-                                  sections, false, T, H, D, eps, rope_base, rope_style,
+  return pqk::launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_stride_t, k_stride_t, q_stride_t, k_stride_t, q_weight,
+                                  k_weight, pos3, sections, false, T, H, D, eps, rope_base, rope_style,
                                   static_cast<cudaStream_t>(stream), d->num_sms)
              ? PQK_ERR_CUDA
              : PQK_OK;
@@ -163,8 +169,8 @@ int pqk_qk_fullc_norm_rope(const void* q_in, const void* k_in, void* q_out, void
     return PQK_ERR_MISALIGNED;
   DeviceInfo* d = nullptr;
   if (int rc = check_device(&d)) return rc;
-  return pqk::launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_stride_t, k_stride_t, q_weight, k_weight, pos,
-                                  nullptr, true, T, H, D, eps, rope_base, rope_style,
+  return pqk::launch_qk_norm_rope(q_in, k_in, q_out, k_out, q_stride_t, k_stride_t, q_stride_t, k_stride_t, q_weight,
+                                  k_weight, pos, nullptr, true, T, H, D, eps, rope_base, rope_style,
                                   static_cast<cudaStream_t>(stream), d->num_sms)
              ? PQK_ERR_CUDA
              : PQK_OK;

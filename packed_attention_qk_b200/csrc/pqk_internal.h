@@ -12,12 +12,14 @@
 
 namespace pqk {
 
-// sections == nullptr: one position per token; else pos is [T, 3] and
+// Strides in elements between tokens, separately for the inputs and the
+// outputs. sections == nullptr: one position per token; else pos is [T, 3] and
 // sections[0..2] are the pairs per (t, h, w) axis. full_width: the norm runs
 // over all H*D elements of a token with weights of H*D entries (one-axis
 // positions only).
 int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride,
-                        int64_t k_stride, const void* wq, const void* wk, const int32_t* pos, const int* sections,
+                        int64_t k_stride, int64_t q_out_stride, int64_t k_out_stride, const void* wq,
+                        const void* wk, const int32_t* pos, const int* sections,
                         bool full_width, int64_t T, int H, int D, float eps, float rope_base, int style,
                         cudaStream_t stream, int num_sms);
 

@@ -43,8 +43,10 @@ struct QkParams {
   const __nv_bfloat16* k_in;
   __nv_bfloat16* q_out;
   __nv_bfloat16* k_out;
-  int64_t q_stride;
+  int64_t q_stride;      // elements between tokens of q_in
   int64_t k_stride;
+  int64_t q_out_stride;  // elements between tokens of q_out
+  int64_t k_out_stride;
   const __nv_bfloat16* wq;
   const __nv_bfloat16* wk;
   const int32_t* pos;  // [T] ids, or [T, 3] (t, h, w) ids for the three-axis variant
@@ -86,7 +88,7 @@ __device__ __forceinline__ void rope_sincos(int32_t pos, double theta, float& c,
   __sincosf(r, &s, &c);  // |r| <= pi: absolute error ~4e-7
 }
 
-template <int D, bool kThreeAxis, bool kFullWidth>
+template <int D, bool kThreeAxis, bool kFullWidth, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParams p) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerStep = 32 / kLanesPerRow;
@@ -116,13 +118,13 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
   const uint4 wq_raw = kFullWidth ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(p.wq + chunk * 8);
   const uint4 wk_raw = kFullWidth ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(p.wk + chunk * 8);
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-  const int64_t n_tasks = p.T * p.n_split;
+  const int64_t n_tasks = kSplit ? p.T * p.n_split : p.T;
   for (int64_t task = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + threadIdx.x / 32; task < n_tasks;
        task += warps_total) {
-    const int64_t t = p.n_split == 1 ? task : task / p.n_split;
+    const int64_t t = kSplit ? task / p.n_split : task;
     // this task's rows [r_lo, rows) of the token's 2H (Q heads, then K heads)
-    const int r_lo = p.n_split == 1 ? 0 : static_cast<int>(task % p.n_split) * p.rows_per_task;
-    const int rows = min(2 * p.H, r_lo + p.rows_per_task);
+    const int r_lo = kSplit ? static_cast<int>(task % p.n_split) * p.rows_per_task : 0;
+    const int rows = kSplit ? min(2 * p.H, r_lo + p.rows_per_task) : 2 * p.H;
     int32_t pos3[3];
     if constexpr (kThreeAxis) {
       pos3[0] = p.pos[3 * t];
@@ -131,15 +133,19 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
     } else {
       pos3[0] = p.pos[t];
     }
+    // a slot's position by selection, not by indexing pos3 (which would
+    // place pos3 in local memory)
+    auto slot_pos = [&](int i) {
+      if constexpr (kThreeAxis) return axis[i] == 0 ? pos3[0] : (axis[i] == 1 ? pos3[1] : pos3[2]);
+      return pos3[0];
+    };
     float cs[8], sn[8];
     if (interleaved) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        rope_sincos(kThreeAxis ? pos3[axis[i]] : pos3[0], theta[j0 + i], cs[i], sn[i]);
+      for (int i = 0; i < 4; ++i) rope_sincos(slot_pos(i), theta[j0 + i], cs[i], sn[i]);
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        rope_sincos(kThreeAxis ? pos3[axis[i]] : pos3[0], theta[j0 + i], cs[i], sn[i]);
+      for (int i = 0; i < 8; ++i) rope_sincos(slot_pos(i), theta[j0 + i], cs[i], sn[i]);
     }
     // full width: the RMS of every Q (and K) element of the token, from a
     // first pass over its rows and a reduction over the whole warp
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
         }
         if (live[u]) {
           const int h = is_q ? r : r - p.H;
-          __nv_bfloat16* dst = is_q ? p.q_out + t * p.q_stride : p.k_out + t * p.k_stride;
+          __nv_bfloat16* dst = is_q ? p.q_out + t * p.q_out_stride : p.k_out + t * p.k_out_stride;
           *reinterpret_cast<uint4*>(dst + h * D + chunk * 8) = pack8(o);
         }
       }
@@ -248,7 +254,8 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
 }  // namespace
 
 int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride,
-                        int64_t k_stride, const void* wq, const void* wk, const int32_t* pos, const int* sections,
+                        int64_t k_stride, int64_t q_out_stride, int64_t k_out_stride, const void* wq,
+                        const void* wk, const int32_t* pos, const int* sections,
                         bool full_width, int64_t T, int H, int D, float eps, float rope_base, int style,
                         cudaStream_t stream, int num_sms) {
   QkParams p;
@@ -258,6 +265,8 @@ int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k
   p.k_out = static_cast<__nv_bfloat16*>(k_out);
   p.q_stride = q_stride;
   p.k_stride = k_stride;
+  p.q_out_stride = q_out_stride;
+  p.k_out_stride = k_out_stride;
   p.wq = static_cast<const __nv_bfloat16*>(wq);
   p.wk = static_cast<const __nv_bfloat16*>(wk);
   p.pos = pos;
@@ -290,20 +299,25 @@ int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k
   const int64_t want = (tasks + warps_per_block - 1) / warps_per_block;
   const int grid = static_cast<int>(want < cap ? want : cap);
   const bool three = sections != nullptr;
+  const bool split = p.n_split > 1;
   if (D == 128) {
     if (full_width)
-      qk_norm_rope_kernel<128, false, true><<<grid, kThreads, 0, stream>>>(p);
+      qk_norm_rope_kernel<128, false, true, false><<<grid, kThreads, 0, stream>>>(p);
     else if (three)
-      qk_norm_rope_kernel<128, true, false><<<grid, kThreads, 0, stream>>>(p);
+      split ? qk_norm_rope_kernel<128, true, false, true><<<grid, kThreads, 0, stream>>>(p)
+            : qk_norm_rope_kernel<128, true, false, false><<<grid, kThreads, 0, stream>>>(p);
     else
-      qk_norm_rope_kernel<128, false, false><<<grid, kThreads, 0, stream>>>(p);
+      split ? qk_norm_rope_kernel<128, false, false, true><<<grid, kThreads, 0, stream>>>(p)
+            : qk_norm_rope_kernel<128, false, false, false><<<grid, kThreads, 0, stream>>>(p);
   } else {
     if (full_width)
-      qk_norm_rope_kernel<64, false, true><<<grid, kThreads, 0, stream>>>(p);
+      qk_norm_rope_kernel<64, false, true, false><<<grid, kThreads, 0, stream>>>(p);
     else if (three)
-      qk_norm_rope_kernel<64, true, false><<<grid, kThreads, 0, stream>>>(p);
+      split ? qk_norm_rope_kernel<64, true, false, true><<<grid, kThreads, 0, stream>>>(p)
+            : qk_norm_rope_kernel<64, true, false, false><<<grid, kThreads, 0, stream>>>(p);
     else
-      qk_norm_rope_kernel<64, false, false><<<grid, kThreads, 0, stream>>>(p);
+      split ? qk_norm_rope_kernel<64, false, false, true><<<grid, kThreads, 0, stream>>>(p)
+            : qk_norm_rope_kernel<64, false, false, false><<<grid, kThreads, 0, stream>>>(p);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

@@ -50,7 +50,7 @@ def lib(path: str | None = None) -> C.CDLL:
         raise RuntimeError(f"libpqk.so not found at {p}: build it with `python -m packed_attention_qk_b200.build`")
     L = C.CDLL(p)
     vp, i64, i32, f32, sz = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
-    L.pqk_qk_norm_rope.argtypes = [vp, vp, vp, vp, i64, i64, vp, vp, vp, i64, i32, i32, f32, f32, i32, vp]
+    L.pqk_qk_norm_rope.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, i64, i32, i32, f32, f32, i32, vp]
     L.pqk_qk_norm_rope.restype = i32
     L.pqk_qk_norm_rope_3axis.argtypes = [vp, vp, vp, vp, i64, i64, vp, vp, vp, i32, i32, i32, i64, i32, i32, f32, f32,
                                          i32, vp]
@@ -135,15 +135,15 @@ def _token_stride(t, ndim: int) -> int:
 def qk_norm_rope(q, k, w_q, w_k, pos, *, eps: float = 1e-6, rope_base: float = 10000.0,
                  style: int = ROPE_INTERLEAVED, q_out=None, k_out=None, stream=None):
     """Fused Q/K RMSNorm + RoPE. q, k: bf16 [T, H, D] (token dim may be
-    strided); outputs default to in place."""
+    strided); q_out, k_out: [T, H, D] views with their own token strides
+    (default: in place)."""
     q_out = q if q_out is None else q_out
     k_out = k if k_out is None else k_out
     T, H, D = q.shape
-    qs, ks = _token_stride(q, 3), _token_stride(k, 3)
-    assert _token_stride(q_out, 3) == qs and _token_stride(k_out, 3) == ks
+    assert tuple(q_out.shape) == (T, H, D) and tuple(k_out.shape) == (T, H, D)
     _check("pqk_qk_norm_rope", lib().pqk_qk_norm_rope(
-        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), qs, ks, _ptr(w_q), _ptr(w_k), _ptr(pos), T, H, D, eps,
-        rope_base, style, _stream(stream)))
+        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _token_stride(q, 3), _token_stride(k, 3), _token_stride(q_out, 3),
+        _token_stride(k_out, 3), _ptr(w_q), _ptr(w_k), _ptr(pos), T, H, D, eps, rope_base, style, _stream(stream)))
     return q_out, k_out
 
 

@@ -69,8 +69,16 @@ def qk(L, **kw):
     a = dict(q_in=A, k_in=A, q_out=A, k_out=A, qs=1024, ks=1024, wq=A, wk=A, pos=A, T=16, H=8, D=128, eps=1e-6,
              base=10000.0, style=0)
     a.update(kw)
-    return L.pqk_qk_norm_rope(a["q_in"], a["k_in"], a["q_out"], a["k_out"], a["qs"], a["ks"], a["wq"], a["wk"],
-                              a["pos"], a["T"], a["H"], a["D"], a["eps"], a["base"], a["style"], None)
+    qos, kos = a.get("qos", a["qs"]), a.get("kos", a["ks"])
+    return L.pqk_qk_norm_rope(a["q_in"], a["k_in"], a["q_out"], a["k_out"], a["qs"], a["ks"], qos, kos, a["wq"],
+                              a["wk"], a["pos"], a["T"], a["H"], a["D"], a["eps"], a["base"], a["style"], None)
+
+
+def test_qk_norm_rope_output_strides(L):
+    assert qk(L, qos=1000) == ERR_INVALID             # output stride below H*D
+    assert qk(L, qos=1028, q_out=A + 4096) == ERR_MISALIGNED
+    assert qk(L, kos=2048) == ERR_INVALID             # in place (k_out == k_in) needs the same stride
+    assert qk(L, T=0, qos=3072, kos=3072, q_out=A + 8192, k_out=A + 16384) == 0
 
 
 def test_qk_norm_rope_host_errors(L):

@@ -27,7 +27,8 @@ int main(void) {
   if (pqk_varlen_attn_workspace_size(0) != 0) ++fails;
   if (pqk_varlen_attn_workspace_size(4096) < pqk_varlen_attn_workspace_size(1)) ++fails;
   /* argument errors are host-side and need no GPU */
-  if (pqk_qk_norm_rope(a, a, a, a, 1024, 1024, a, a, a, 16, 8, 96, 1e-6f, 1e4f, 0, NULL) != PQK_ERR_UNSUPPORTED)
+  if (pqk_qk_norm_rope(a, a, a, a, 1024, 1024, 1024, 1024, a, a, a, 16, 8, 96, 1e-6f, 1e4f, 0, NULL) !=
+      PQK_ERR_UNSUPPORTED)
     ++fails;
   if (pqk_varlen_attn_fwd(a, a, a, a, NULL, 1024, 1024, 1024, 1024, a, 0, 512, 8, 128, 0.1f, a, 4096, NULL) !=
       PQK_ERR_INVALID_ARG)

@@ -48,6 +48,30 @@ def test_qk_norm_rope_out_of_place_ragged(style):
     prologue_case(w, style, in_place=False)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_qk_norm_rope_into_wider_output_rows_with_guard_bands(D):
+    # outputs with their own token strides: Q and K written into two slots of
+    # a wider row (as into a sequence-parallel send buffer), inputs
+    # contiguous; everything outside the two slots keeps its canary value
+    torch = torch_cuda()
+    w = wl.custom([300, 0, 17, 129], H=6, D=D, seed=43)
+    x = wl.prologue_inputs(w)
+    T, H = w.T, w.H
+    q, k = to_dev_bf16(x["q"]), to_dev_bf16(x["k"])
+    wq, wk, pos = to_dev_bf16(x["w_q"]), to_dev_bf16(x["w_k"]), to_dev(x["pos"])
+    width = 3 * H * D + 64
+    buf = torch.full((T + 2, width), 7.0, dtype=torch.bfloat16, device="cuda")
+    qo = buf[1:1 + T, 32:32 + H * D].view(T, H, D)
+    ko = buf[1:1 + T, 32 + H * D:32 + 2 * H * D].view(T, H, D)
+    pqk.qk_norm_rope(q, k, wq, wk, pos, eps=w.eps, rope_base=w.rope_base, q_out=qo, k_out=ko)
+    torch.cuda.synchronize()
+    for name, out, wname in (("q", qo, "w_q"), ("k", ko, "w_k")):
+        ref = oracle.qk_norm_rope(x[name], x[wname], x["pos"], w.eps, w.rope_base)
+        assert_elementwise(bf16_to_f64(out), ref, f"{name} into a wider row")
+    guard = torch.cat([buf[0], buf[T + 1], buf[1:1 + T, :32].flatten(), buf[1:1 + T, 32 + 2 * H * D:].flatten()])
+    assert bool((guard == 7.0).all())
+
+
 def test_qk_norm_rope_58048_tokens_sampled():
     w = wl.config(3)
     prologue_case(w, pqk.ROPE_INTERLEAVED, rows=wl.sample_rows(w, 512))

@@ -42,28 +42,54 @@ def _oracle_attn(q, k, v, cu, scale):
     return torch.from_numpy(o)
 
 
-def _rank_main(rank, world, port, H, D, out):
+def _oracle_prologue(w_q, w_k, pos):
+    """The oracle's RMSNorm + RoPE of one head group, written into the send
+    buffer's slots (views with their own token strides)."""
+    def run(qg, kg, q_out, k_out):
+        q_out.copy_(torch.from_numpy(oracle.qk_norm_rope(qg.numpy(), w_q, pos, 1e-6, 10000.0)))
+        k_out.copy_(torch.from_numpy(oracle.qk_norm_rope(kg.numpy(), w_k, pos, 1e-6, 10000.0)))
+    return run
+
+
+def _rank_main(rank, world, port, H, D, out, with_prologue=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         (q, k, v), cu = _inputs(H, D)
-        Tl = q.shape[0] // world
+        T = q.shape[0]
+        Tl = T // world
         sl = slice(rank * Tl, (rank + 1) * Tl)
+        prologue = None
+        if with_prologue:
+            g = np.random.default_rng(11)
+            w_q, w_k = g.uniform(0.5, 1.5, D), g.uniform(0.5, 1.5, D)
+            pos = np.concatenate([np.arange(L) for L in LENS]).astype(np.int32)
+            prologue = _oracle_prologue(w_q, w_k, pos[sl])
+            qn = oracle.qk_norm_rope(q, w_q, pos, 1e-6, 10000.0)
+            kn = oracle.qk_norm_rope(k, w_k, pos, 1e-6, 10000.0)
         o = ulysses.ulysses_attention(torch.from_numpy(q[sl]), torch.from_numpy(k[sl]), torch.from_numpy(v[sl]),
-                                      torch.from_numpy(cu), softmax_scale=0.2, attn=_oracle_attn)
-        ref, _ = oracle.varlen_attn(q, k, v, cu, 0.2)
+                                      torch.from_numpy(cu), softmax_scale=0.2, attn=_oracle_attn, prologue=prologue,
+                                      total_tokens=T)
+        if with_prologue:
+            ref, _ = oracle.varlen_attn(qn, kn, v, cu, 0.2)
+        else:
+            ref, _ = oracle.varlen_attn(q, k, v, cu, 0.2)
         out.put((rank, bool(np.array_equal(o.numpy(), ref[sl])), tuple(o.shape)))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world, H", [(2, 4), (4, 4), (4, 8)])
-def test_shards_equal_the_whole_sequence_attention(world, H):
+@pytest.mark.parametrize("world, H, with_prologue", [(2, 4, False), (4, 4, False), (4, 8, False), (2, 4, True),
+                                                    (4, 8, True)])
+def test_shards_equal_the_whole_sequence_attention(world, H, with_prologue):
+    # with_prologue: the Q/K norm + RoPE of every head group is written
+    # straight into the send buffer and must equal the whole-sequence
+    # prologue followed by the whole-sequence attention
     D = 8
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, H, D, out)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, H, D, out, with_prologue)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
