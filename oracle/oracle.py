@@ -72,9 +72,11 @@ def load(path: str):
                                                C.c_int, C.c_int, i32p, C.c_int64, f64p]
     L.oracle_linear_swiglu.argtypes = [vp, C.c_int64, vp, C.c_int, C.c_int64, C.c_int, C.c_int, i32p, C.c_int64,
                                        f64p]
+    L.oracle_qk_norm_rope_e4m3.argtypes = [vp, C.c_int, C.c_int64, vp, C.c_int, i32p, C.c_int64, C.c_int, C.c_int,
+                                           C.c_double, C.c_double, C.c_int, i32p, C.c_int64, u8p, f32p]
     L.oracle_e4m3_codes.argtypes = [f32p, C.c_int64, u8p]
     L.oracle_e4m3_codes.restype = None
-    for f in (L.oracle_qk_norm_rope, L.oracle_qk_norm_rope_3axis, L.oracle_qk_fullc_norm_rope, L.oracle_varlen_attn,
+    for f in (L.oracle_qk_norm_rope, L.oracle_qk_norm_rope_e4m3, L.oracle_qk_norm_rope_3axis, L.oracle_qk_fullc_norm_rope, L.oracle_varlen_attn,
               L.oracle_varlen_attn_skip, L.oracle_quantize_e4m3, L.oracle_varlen_attn_fp8qk, L.oracle_varlen_attn_fp8,
               L.oracle_varlen_attn_fp8_online, L.oracle_modulate_swiglu, L.oracle_linear_gated_residual, L.oracle_linear_swiglu):
         f.restype = C.c_int
@@ -135,6 +137,27 @@ def qk_norm_rope(x: np.ndarray, w: np.ndarray, pos: np.ndarray, eps: float, base
     if rc:
         raise ValueError("oracle_qk_norm_rope: invalid arguments")
     return y
+
+
+def qk_norm_rope_e4m3(x: np.ndarray, w: np.ndarray, pos: np.ndarray, eps: float, base: float,
+                      style: int = ROPE_INTERLEAVED, rows=None):
+    """RMSNorm + RoPE, then e4m3 codes with the per-tensor scale of the bound
+    sqrt(D) * max|w| (oracle_qk_norm_rope_e4m3). Returns (codes uint8
+    [nrows, H, D], deq float32)."""
+    T, H, D = x.shape
+    stride_t = x.strides[0] // x.itemsize
+    assert x.strides[2] == x.itemsize and x.strides[1] == D * x.itemsize
+    w = np.ascontiguousarray(w)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    r, n = _rows(rows)
+    codes = np.empty((n if r is not None else T, H, D), np.uint8)
+    deq = np.empty(1, np.float32)
+    rc = lib().oracle_qk_norm_rope_e4m3(_ptr(x), _kind(x), stride_t, _ptr(w), _kind(w), _ptr(pos, C.c_int32), T, H, D,
+                                        eps, base, style, _ptr(r, C.c_int32), n, _ptr(codes, C.c_uint8),
+                                        _ptr(deq, C.c_float))
+    if rc:
+        raise ValueError("oracle_qk_norm_rope_e4m3: invalid arguments")
+    return codes, deq[0]
 
 
 def qk_norm_rope_3axis(x: np.ndarray, w: np.ndarray, pos3: np.ndarray, sections, eps: float, base: float,

@@ -15,6 +15,10 @@
  *   oracle_qk_norm_rope_3axis -- the same with a (t, h, w) position per
  *                             token for video latents (a reading: the pages
  *                             give no RoPE variant; see the function).
+ *   oracle_qk_norm_rope_e4m3 -- the same followed by e4m3 codes with a
+ *                             per-tensor scale from the normalised rows'
+ *                             bound (SAGE FP8 folded into the prologue; a
+ *                             reading).
  *   oracle_qk_fullc_norm_rope -- the same with the norm over all heads of
  *                             a token (weight of H*D entries), a reading of
  *                             "Q/K normalisation" the pages leave open.
@@ -367,6 +371,41 @@ static void skip_block_flags(const void* q, const void* k, int in_kind, int64_t 
                              int64_t r0, int64_t r1, int h, int D, double scale, double tau, int kblock,
                              unsigned char* keep);
 static int64_t skip_tile_count(const unsigned char* keep, int H, int64_t nqb, int64_t nkb, int64_t per_tile);
+
+/*
+ * RMSNorm + RoPE as oracle_qk_norm_rope, then e4m3 codes with one scale per
+ * tensor taken from a bound rather than from the data (a reading of SAGE's
+ * FP8 quantisation folded into the Q/K prologue, first page, bullet on
+ * TRTLLM_ATTN SAGE and Skip-Softmax): a normalised row has
+ * sum_d (x_d / rms)^2 <= D, so every element of it, and of its rotation
+ * (which preserves each pair's norm), is at most sqrt(D) * max_d |w_d| in
+ * magnitude. In float arithmetic, amax = sqrtf(D) * max_d |w_d|,
+ * inv = 448 / amax and deq = amax / 448 (both 1 when amax = 0); every element
+ * y (the float64 result) gets code e4m3((float)(y * inv)). codes:
+ * [nrows, H, D]; deq_out: that one factor.
+ */
+int oracle_qk_norm_rope_e4m3(const void* x, int x_kind, int64_t stride_t, const void* w, int w_kind,
+                             const int32_t* pos, int64_t T, int H, int D, double eps, double base, int style,
+                             const int32_t* rows, int64_t nrows, uint8_t* codes, float* deq_out) {
+  if (D <= 0 || H <= 0 || T < 0) return -1;
+  const int64_t nr = rows ? nrows : T;
+  const int64_t n = nr * (int64_t)H * D;
+  double* y = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  int rc = oracle_qk_norm_rope(x, x_kind, stride_t, w, w_kind, pos, T, H, D, eps, base, style, rows, nrows, y);
+  if (!rc) {
+    float maxw = 0.0f;
+    for (int d = 0; d < D; ++d) {
+      const float a = (float)fabs(load(w, w_kind, d));
+      if (a > maxw) maxw = a;
+    }
+    const float amax = sqrtf((float)D) * maxw;
+    const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;
+    *deq_out = amax > 0.0f ? amax / 448.0f : 1.0f;
+    for (int64_t e = 0; e < n; ++e) codes[e] = e4m3_code((float)(y[e] * (double)inv));
+  }
+  free(y);
+  return rc;
+}
 
 /*
  * Attention with Q and K quantised to e4m3 per head (oracle_quantize_e4m3)

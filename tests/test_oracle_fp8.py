@@ -443,3 +443,53 @@ def test_fp8_skipping_sampled_rows_equal_full_evaluation():
     o2, l2, _ = oracle.varlen_attn_fp8(q, k, v, cu, scale, tau=10.0, skip_block=(16, 64), skip_tile_rows=64,
                                        rows=rows)
     assert np.array_equal(o2, o[rows]) and np.array_equal(l2, lse[rows])
+
+
+# ----------------------------------------------- Q/K prologue with e4m3 output (bound scale)
+
+def test_fp8_prologue_scale_is_the_normalised_rows_bound():
+    # deq = sqrt(D) * max |w| / 448 in float arithmetic, whatever the data
+    g = np.random.default_rng(20)
+    for D in (64, 128):
+        w = g.uniform(0.5, 1.5, D)
+        w[3] = -1.75  # the largest magnitude is negative
+        x = g.standard_normal((50, 2, D))
+        _, deq = oracle.qk_norm_rope_e4m3(x, w, np.arange(50, dtype=np.int32), 1e-6, 10000.0)
+        amax = np.float32(np.sqrt(np.float32(D))) * np.float32(1.75)
+        assert deq == np.float32(amax / np.float32(448.0))
+        _, deq2 = oracle.qk_norm_rope_e4m3(x * 100.0, w, np.arange(50, dtype=np.int32), 1e-6, 10000.0)
+        assert deq2 == deq
+
+
+def test_fp8_prologue_one_hot_row_reaches_the_bound():
+    # x = (a, 0, ..., 0) at position 0: the normalised row is sqrt(D) at d = 0,
+    # times w_0 = max |w|, i.e. exactly the bound: code +-448 (0x7E / 0xFE),
+    # every other element 0
+    D = 128
+    w = np.full(D, 0.75)
+    w[0] = 1.25
+    x = np.zeros((2, 1, D))
+    x[0, 0, 0] = 1000.0
+    x[1, 0, 0] = -1000.0
+    codes, _ = oracle.qk_norm_rope_e4m3(x, w, np.zeros(2, np.int32), 1e-12, 10000.0)
+    assert codes[0, 0, 0] == 0x7E and codes[1, 0, 0] == 0xFE
+    assert np.all(codes[:, 0, 1:] == 0)
+
+
+def test_fp8_prologue_codes_are_within_an_e4m3_step_of_the_rotated_rows():
+    g = np.random.default_rng(21)
+    T, H, D = 300, 3, 128
+    x = g.standard_normal((T, H, D))
+    x[7] *= 40.0
+    w = g.uniform(0.5, 1.5, D)
+    pos = g.integers(0, 60000, T).astype(np.int32)
+    for style in (oracle.ROPE_INTERLEAVED, oracle.ROPE_HALF):
+        codes, deq = oracle.qk_norm_rope_e4m3(x, w, pos, 1e-6, 10000.0, style)
+        y = oracle.qk_norm_rope(x, w, pos, 1e-6, 10000.0, style)
+        back = _decode(codes) * float(deq)
+        assert np.all(np.abs(y) <= 448.0 * float(deq) * (1 + 1e-6))  # the bound holds
+        assert np.all(np.abs(back - y) <= np.maximum(2.0 ** -4 * np.abs(y), 2.0 ** -10 * float(deq)) * (1 + 1e-6))
+        # sampled rows = full evaluation
+        rows = np.array([0, 7, 150, 299], np.int32)
+        c2, d2 = oracle.qk_norm_rope_e4m3(x, w, pos, 1e-6, 10000.0, style, rows=rows)
+        assert np.array_equal(c2, codes[rows]) and d2 == deq

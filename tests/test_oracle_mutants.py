@@ -76,6 +76,9 @@ MUTANTS = {
                                    "\n      const double pq = pj;"),
     "fp8_online_denominator_quantised": ("\n      den += pj;\n", "\n      den += pq;\n"),
     "fp8_online_numerator_not_rescaled": ("      for (int d = 0; d < D; ++d) num[d] *= alpha;\n", ""),
+    "fp8_prologue_scale_without_sqrt_d": ("const float amax = sqrtf((float)D) * maxw;", "const float amax = maxw;"),
+    "fp8_prologue_signed_weight_max": ("const float a = (float)fabs(load(w, w_kind, d));",
+                                       "const float a = (float)load(w, w_kind, d);"),
     "fp8_skip_dropped_keys_summed": ("    if (keep && !keep[j / kblock]) continue;\n    const double pj", "    const double pj"),
     "fp8_online_dropped_keys_summed": ("      if (keep && !keep[j / skip_kblock]) continue;\n", ""),
     "linear_w_transposed": ("load(w, in_kind, (int64_t)n * K + k)", "load(w, in_kind, (int64_t)k * N + n)"),
