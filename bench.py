@@ -21,7 +21,8 @@ three-axis RoPE, back-to-back and full-width norm timings; the block-
 skipping attention on the local-attention stand-in (``--skip-tau``, plain
 vs skipping vs FP8 Q K^T and the whole attention in FP8, each with and
 without skipping); the FP8 Q K^T attention
-on the step's inputs (``--no-fp8`` leaves it out); the block's three linear
+on the step's inputs, and the Q/K prologue with e4m3 output against the
+prologue followed by the separate quantisation (``--no-fp8`` leaves them out); the block's three linear
 layers with the gated residual or SwiGLU in the GEMM epilogue, on the step's
 own activations, against cuBLAS plus torch epilogues (``linear_epilogue``;
 ``--no-linear`` leaves it out); the two HBM-bound kernels on the 40-head
@@ -687,7 +688,22 @@ def run_ours(args, w):
         full_ms = ev3[0].elapsed_time(ev3[1]) / 3
         if pqk.get_device_status() != 0:
             raise RuntimeError("device status set during the FP8 timing")
+        # the Q/K prologue with e4m3 output (the quantisation folded in, bound
+        # scale): replaces qk_norm_rope + the separate quantisation pass
+        pqk.qk_norm_rope_e4m3(d["q"], d["k"], d["w_q"], d["w_k"], d["pos"], eps=w.eps, rope_base=w.rope_base,
+                              q8=q8, k8=k8)
+        ev3[0].record()
+        for _ in range(reps3):
+            pqk.qk_norm_rope_e4m3(d["q"], d["k"], d["w_q"], d["w_k"], d["pos"], eps=w.eps, rope_base=w.rope_base,
+                                  q8=q8, k8=k8)
+        ev3[1].record()
+        torch.cuda.synchronize()
+        fused_us = ev3[0].elapsed_time(ev3[1]) / reps3 * 1e3
+        fused_bytes = w.T * (6 * w.H * w.D + 4)
         fp8 = {"quantize_us": quant_us, "attn_ms": fp8_ms, "attn_tflops": flops / (fp8_ms * 1e-3) / 1e12,
+               "prologue_e4m3_us": fused_us, "prologue_e4m3_gbs": fused_bytes / (fused_us * 1e-6) / 1e9,
+               "prologue_e4m3_frac_hbm": fused_bytes / (fused_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+               "separate_prologue_and_quantize_us": rope1_b2b_us + quant_us,
                "speedup_vs_bf16": att_ms / fp8_ms,
                "quantize_gbs": (4 * w.T * w.H * w.D + 2 * w.T * w.H * w.D) / (quant_us * 1e-6) / 1e9,
                "full_fp8_attn_ms": full_ms, "full_fp8_speedup_vs_bf16": att_ms / full_ms}

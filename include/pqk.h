@@ -109,6 +109,29 @@ PQK_API int pqk_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, vo
                      int rope_style, void* stream);
 
 /*
+ * pqk_qk_norm_rope_e4m3 -- pqk_qk_norm_rope with its outputs as FP8 e4m3
+ * codes, the SAGE FP8 quantisation of Q and K (first page, bullet on
+ * TRTLLM_ATTN SAGE and Skip-Softmax) folded into the prologue, so that no
+ * separate quantisation pass reads Q and K again. A reading: one scale per
+ * tensor from a bound instead of the data. A normalised row has
+ * sum_d (x_d / rms)^2 <= D, so every element of it, rotated or not, is at
+ * most sqrt(D) * max_d |w_X[d]| in magnitude; with amax that bound (in
+ * float), the codes are e4m3(y * 448 / amax) (nearest even) and the
+ * dequantisation factor of every head of X is amax / 448 (1 if amax = 0).
+ *
+ * q_in, k_in, q_weight, k_weight, pos, T, H, D, eps, rope_base, rope_style:
+ *               as pqk_qk_norm_rope.
+ * q8, k8        device e4m3 codes [T, H, D] bytes, contiguous, 16-byte
+ *               aligned (the layout pqk_varlen_attn_fwd_fp8qk / _fp8 read).
+ * deq           device fp32 [2H]: Q's then K's per-head dequantisation
+ *               factors (all heads of a tensor equal), as those entries take.
+ */
+PQK_API int pqk_qk_norm_rope_e4m3(const void* q_in, const void* k_in, void* q8, void* k8, int64_t q_stride_t,
+                          int64_t k_stride_t, const void* q_weight, const void* k_weight,
+                          const int32_t* pos, int64_t T, int H, int D, float eps, float rope_base,
+                          int rope_style, float* deq, void* stream);
+
+/*
  * pqk_qk_norm_rope_3axis -- pqk_qk_norm_rope with a (t, h, w) position per
  * token for video latents. The pages give no RoPE variant; the reading
  * taken: every pair j keeps theta_j = rope_base^(-2j/D) and takes its angle
@@ -361,6 +384,10 @@ PQK_API int pqk_varlen_attn_fwd_noalloc(const void* q, const void* k, const void
  * act           device bf16 [T, F] contiguous; may equal gate when
  *               gu_stride_t == F.
  * C, F          multiples of 8; C <= 16384. B >= 1, T >= 0, eps > 0.
+ * A token's x' and h are written in the last pass over its row, each chunk
+ * after that chunk's last read of x, and each act chunk after the read of
+ * its gate chunk, so the aliases above are safe (x_out and h must not
+ * alias each other).
  */
 PQK_API int pqk_modulate_swiglu(const void* x, const void* branch, void* x_out, void* h,
                         const float* shift, const float* scale, const float* gate_res,

@@ -129,6 +129,30 @@ int pqk_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_ou
              : PQK_OK;
 }
 
+int pqk_qk_norm_rope_e4m3(const void* q_in, const void* k_in, void* q8, void* k8, int64_t q_stride_t,
+                          int64_t k_stride_t, const void* q_weight, const void* k_weight, const int32_t* pos,
+                          int64_t T, int H, int D, float eps, float rope_base, int rope_style, float* deq,
+                          void* stream) {
+  if (T < 0 || H <= 0 || !(eps > 0.f) || !(rope_base > 0.f)) return PQK_ERR_INVALID_ARG;
+  if (rope_style != PQK_ROPE_INTERLEAVED && rope_style != PQK_ROPE_HALF) return PQK_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return PQK_ERR_UNSUPPORTED;
+  const int64_t row = static_cast<int64_t>(H) * D;
+  if (q_stride_t < row || k_stride_t < row) return PQK_ERR_INVALID_ARG;
+  if (T == 0) return PQK_OK;
+  if (!q_in || !k_in || !q8 || !k8 || !q_weight || !k_weight || !pos || !deq) return PQK_ERR_INVALID_ARG;
+  if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(q8) || !aligned16(k8) || !aligned16(q_weight) ||
+      !aligned16(k_weight) || (reinterpret_cast<uintptr_t>(deq) % 4) || (q_stride_t % 8) || (k_stride_t % 8))
+    return PQK_ERR_MISALIGNED;
+  DeviceInfo* d = nullptr;
+  if (int rc = check_device(&d)) return rc;
+  // the byte outputs are addressed as [T, H, D]; their "stride" is unused
+  return pqk::launch_qk_norm_rope(q_in, k_in, q8, k8, q_stride_t, k_stride_t, row, row, q_weight, k_weight, pos,
+                                  nullptr, false, T, H, D, eps, rope_base, rope_style,
+                                  static_cast<cudaStream_t>(stream), d->num_sms, deq)
+             ? PQK_ERR_CUDA
+             : PQK_OK;
+}
+
 int pqk_qk_norm_rope_3axis(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride_t,
                            int64_t k_stride_t, const void* q_weight, const void* k_weight, const int32_t* pos3,
                            int sec_t, int sec_h, int sec_w, int64_t T, int H, int D, float eps, float rope_base,

@@ -16,12 +16,14 @@ namespace pqk {
 // outputs. sections == nullptr: one position per token; else pos is [T, 3] and
 // sections[0..2] are the pairs per (t, h, w) axis. full_width: the norm runs
 // over all H*D elements of a token with weights of H*D entries (one-axis
-// positions only).
+// positions only). e4m3_deq non-null: the outputs are e4m3 codes ([T, H, D]
+// bytes, contiguous) at the per-tensor bound scale, whose [2H]
+// dequantisation factors go to e4m3_deq (one-axis, per-head norm only).
 int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t q_stride,
                         int64_t k_stride, int64_t q_out_stride, int64_t k_out_stride, const void* wq,
                         const void* wk, const int32_t* pos, const int* sections,
                         bool full_width, int64_t T, int H, int D, float eps, float rope_base, int style,
-                        cudaStream_t stream, int num_sms);
+                        cudaStream_t stream, int num_sms, float* e4m3_deq = nullptr);
 
 int launch_modulate_swiglu(const void* x, const void* branch, void* x_out, void* h, const float* shift,
                            const float* scale, const float* gate_res, const int32_t* cu_seqlens, int B, int64_t T,

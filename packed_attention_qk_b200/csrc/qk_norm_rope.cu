@@ -19,6 +19,9 @@
 // K) with one weight per element: a first pass of the warp over the token's
 // rows sums the squares (full-warp reduction), the second pass re-reads the
 // rows (now in cache), normalises, rotates and stores.
+// The e4m3-output variant (SAGE FP8 folded into the prologue) writes codes
+// [T, H, D] bytes at one scale per tensor, the bound sqrt(D) max|w| of a
+// normalised row mapping to 448, and the [2H] dequantisation factors.
 // Few tokens: with about one token per resident warp the slowest warps take
 // two tokens while most take one, and the launch ends at the tail. The
 // launcher then splits each token's 2*H rows into n_split tasks of
@@ -58,6 +61,7 @@ struct QkParams {
   int style;
   int n_split;        // tasks per token (1: the whole token)
   int rows_per_task;  // rows of the token's 2H a task covers (2H when n_split is 1)
+  float* deq;         // e4m3 output: [2H] dequantisation factors (Q's heads, then K's)
 };
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
@@ -88,7 +92,7 @@ __device__ __forceinline__ void rope_sincos(int32_t pos, double theta, float& c,
   __sincosf(r, &s, &c);  // |r| <= pi: absolute error ~4e-7
 }
 
-template <int D, bool kThreeAxis, bool kFullWidth, bool kSplit>
+template <int D, bool kThreeAxis, bool kFullWidth, bool kSplit, bool kE4m3Out = false>
 __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParams p) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerStep = 32 / kLanesPerRow;
@@ -117,6 +121,30 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
   // per-head weights ([D], shared by all heads) stay in registers
   const uint4 wq_raw = kFullWidth ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(p.wq + chunk * 8);
   const uint4 wk_raw = kFullWidth ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(p.wk + chunk * 8);
+  // e4m3 output: a normalised row has sum (x/rms)^2 <= D, so every element of
+  // it, rotated or not, is at most sqrt(D) max|w| in magnitude; that bound
+  // maps to 448 (one scale per tensor, no pass over the data)
+  float inv_q8 = 1.0f, inv_k8 = 1.0f;
+  if constexpr (kE4m3Out) {
+    float wv[8], mq = 0.f, mk = 0.f;
+    unpack8(wq_raw, wv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mq = fmaxf(mq, fabsf(wv[i]));
+    unpack8(wk_raw, wv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mk = fmaxf(mk, fabsf(wv[i]));
+#pragma unroll
+    for (int off = kHalfLanes; off >= 1; off >>= 1) {
+      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, off));
+      mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, off));
+    }
+    const float aq = sqrtf(static_cast<float>(D)) * mq, ak = sqrtf(static_cast<float>(D)) * mk;
+    inv_q8 = aq > 0.0f ? 448.0f / aq : 1.0f;
+    inv_k8 = ak > 0.0f ? 448.0f / ak : 1.0f;
+    if (blockIdx.x == 0)
+      for (int h = threadIdx.x; h < 2 * p.H; h += kThreads)
+        p.deq[h] = h < p.H ? (aq > 0.0f ? aq / 448.0f : 1.0f) : (ak > 0.0f ? ak / 448.0f : 1.0f);
+  }
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
   const int64_t n_tasks = kSplit ? p.T * p.n_split : p.T;
   for (int64_t task = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + threadIdx.x / 32; task < n_tasks;
@@ -243,8 +271,18 @@ __global__ void __launch_bounds__(kThreads, 3) qk_norm_rope_kernel(const QkParam
         }
         if (live[u]) {
           const int h = is_q ? r : r - p.H;
-          __nv_bfloat16* dst = is_q ? p.q_out + t * p.q_out_stride : p.k_out + t * p.k_out_stride;
-          *reinterpret_cast<uint4*>(dst + h * D + chunk * 8) = pack8(o);
+          if constexpr (kE4m3Out) {
+            // codes [T, H, D] bytes: 8 per lane
+            const float inv = is_q ? inv_q8 : inv_k8;
+            uint2 c;
+            c.x = pack_e4m3x2(o[0] * inv, o[1] * inv) | (pack_e4m3x2(o[2] * inv, o[3] * inv) << 16);
+            c.y = pack_e4m3x2(o[4] * inv, o[5] * inv) | (pack_e4m3x2(o[6] * inv, o[7] * inv) << 16);
+            uint8_t* dst8 = reinterpret_cast<uint8_t*>(is_q ? p.q_out : p.k_out) + (t * p.H + h) * D + chunk * 8;
+            *reinterpret_cast<uint2*>(dst8) = c;
+          } else {
+            __nv_bfloat16* dst = is_q ? p.q_out + t * p.q_out_stride : p.k_out + t * p.k_out_stride;
+            *reinterpret_cast<uint4*>(dst + h * D + chunk * 8) = pack8(o);
+          }
         }
       }
     }
@@ -257,7 +295,7 @@ int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k
                         int64_t k_stride, int64_t q_out_stride, int64_t k_out_stride, const void* wq,
                         const void* wk, const int32_t* pos, const int* sections,
                         bool full_width, int64_t T, int H, int D, float eps, float rope_base, int style,
-                        cudaStream_t stream, int num_sms) {
+                        cudaStream_t stream, int num_sms, float* e4m3_deq) {
   QkParams p;
   p.q_in = static_cast<const __nv_bfloat16*>(q_in);
   p.k_in = static_cast<const __nv_bfloat16*>(k_in);
@@ -267,6 +305,7 @@ int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k
   p.k_stride = k_stride;
   p.q_out_stride = q_out_stride;
   p.k_out_stride = k_out_stride;
+  p.deq = e4m3_deq;
   p.wq = static_cast<const __nv_bfloat16*>(wq);
   p.wk = static_cast<const __nv_bfloat16*>(wk);
   p.pos = pos;
@@ -300,6 +339,17 @@ int launch_qk_norm_rope(const void* q_in, const void* k_in, void* q_out, void* k
   const int grid = static_cast<int>(want < cap ? want : cap);
   const bool three = sections != nullptr;
   const bool split = p.n_split > 1;
+  if (e4m3_deq != nullptr) {
+    // one-axis positions, per-head norm only
+    if (three || full_width) return -1;
+    if (D == 128)
+      split ? qk_norm_rope_kernel<128, false, false, true, true><<<grid, kThreads, 0, stream>>>(p)
+            : qk_norm_rope_kernel<128, false, false, false, true><<<grid, kThreads, 0, stream>>>(p);
+    else
+      split ? qk_norm_rope_kernel<64, false, false, true, true><<<grid, kThreads, 0, stream>>>(p)
+            : qk_norm_rope_kernel<64, false, false, false, true><<<grid, kThreads, 0, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  }
   if (D == 128) {
     if (full_width)
       qk_norm_rope_kernel<128, false, true, false><<<grid, kThreads, 0, stream>>>(p);

@@ -22,7 +22,7 @@ ROPE_INTERLEAVED, ROPE_HALF = 0, 1
 NORM_RMS, NORM_LAYER, NORM_NONE = 0, 1, 2
 
 # every symbol include/pqk.h declares
-EXPORTS = ("pqk_qk_norm_rope", "pqk_qk_norm_rope_3axis", "pqk_qk_fullc_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd",
+EXPORTS = ("pqk_qk_norm_rope", "pqk_qk_norm_rope_e4m3", "pqk_qk_norm_rope_3axis", "pqk_qk_fullc_norm_rope", "pqk_varlen_attn_workspace_size", "pqk_varlen_attn_fwd",
            "pqk_varlen_attn_fwd_skip", "pqk_quantize_qk_e4m3", "pqk_varlen_attn_fwd_fp8qk", "pqk_quantize_e4m3",
            "pqk_varlen_attn_fwd_fp8",
            "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu", "pqk_linear_gated_residual", "pqk_linear_swiglu",
@@ -52,6 +52,8 @@ def lib(path: str | None = None) -> C.CDLL:
     vp, i64, i32, f32, sz = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
     L.pqk_qk_norm_rope.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, vp, vp, vp, i64, i32, i32, f32, f32, i32, vp]
     L.pqk_qk_norm_rope.restype = i32
+    L.pqk_qk_norm_rope_e4m3.argtypes = [vp, vp, vp, vp, i64, i64, vp, vp, vp, i64, i32, i32, f32, f32, i32, vp, vp]
+    L.pqk_qk_norm_rope_e4m3.restype = i32
     L.pqk_qk_norm_rope_3axis.argtypes = [vp, vp, vp, vp, i64, i64, vp, vp, vp, i32, i32, i32, i64, i32, i32, f32, f32,
                                          i32, vp]
     L.pqk_qk_norm_rope_3axis.restype = i32
@@ -145,6 +147,25 @@ def qk_norm_rope(q, k, w_q, w_k, pos, *, eps: float = 1e-6, rope_base: float = 1
         _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _token_stride(q, 3), _token_stride(k, 3), _token_stride(q_out, 3),
         _token_stride(k_out, 3), _ptr(w_q), _ptr(w_k), _ptr(pos), T, H, D, eps, rope_base, style, _stream(stream)))
     return q_out, k_out
+
+
+def qk_norm_rope_e4m3(q, k, w_q, w_k, pos, *, eps: float = 1e-6, rope_base: float = 10000.0,
+                      style: int = ROPE_INTERLEAVED, q8=None, k8=None, deq=None, stream=None):
+    """Fused Q/K RMSNorm + RoPE with e4m3 output at the per-tensor bound
+    scale sqrt(D) max|w| -> 448. Returns (q8, k8 uint8 [T, H, D], deq fp32 [2H])."""
+    import torch
+    T, H, D = q.shape
+    if q8 is None:
+        q8 = torch.empty((T, H, D), dtype=torch.uint8, device=q.device)
+    if k8 is None:
+        k8 = torch.empty((T, H, D), dtype=torch.uint8, device=q.device)
+    if deq is None:
+        deq = torch.empty(2 * H, dtype=torch.float32, device=q.device)
+    assert q8.is_contiguous() and k8.is_contiguous() and deq.numel() >= 2 * H
+    _check("pqk_qk_norm_rope_e4m3", lib().pqk_qk_norm_rope_e4m3(
+        _ptr(q), _ptr(k), _ptr(q8), _ptr(k8), _token_stride(q, 3), _token_stride(k, 3), _ptr(w_q), _ptr(w_k),
+        _ptr(pos), T, H, D, eps, rope_base, style, _ptr(deq), _stream(stream)))
+    return q8, k8, deq
 
 
 def qk_norm_rope_3axis(q, k, w_q, w_k, pos3, sections, *, eps: float = 1e-6, rope_base: float = 10000.0,

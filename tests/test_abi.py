@@ -81,6 +81,20 @@ def test_qk_norm_rope_output_strides(L):
     assert qk(L, T=0, qos=3072, kos=3072, q_out=A + 8192, k_out=A + 16384) == 0
 
 
+def test_qk_norm_rope_e4m3_host_errors(L):
+    def call(**kw):
+        a = dict(q=A, k=A, q8=A, k8=A, qs=1024, ks=1024, wq=A, wk=A, pos=A, T=16, H=8, D=128, deq=A)
+        a.update(kw)
+        return L.pqk_qk_norm_rope_e4m3(a["q"], a["k"], a["q8"], a["k8"], a["qs"], a["ks"], a["wq"], a["wk"], a["pos"],
+                                       a["T"], a["H"], a["D"], 1e-6, 10000.0, 0, a["deq"], None)
+    assert call(D=96) == ERR_UNSUPPORTED
+    assert call(qs=1000) == ERR_INVALID
+    assert call(deq=None) == ERR_INVALID
+    assert call(q8=A + 8) == ERR_MISALIGNED
+    assert call(deq=A + 2) == ERR_MISALIGNED
+    assert call(T=0, q=None) == 0
+
+
 def test_qk_norm_rope_host_errors(L):
     assert qk(L, D=96) == ERR_UNSUPPORTED
     assert qk(L, D=256) == ERR_UNSUPPORTED

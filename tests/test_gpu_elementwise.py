@@ -286,13 +286,18 @@ def test_modulate_swiglu_in_place_outputs():
     gu[:, :w.F] = to_dev_bf16(e["gate"])
     gu[:, w.F:] = to_dev_bf16(e["up"])
     gate, up = gu[:, :w.F], gu[:, w.F:]
-    # x' back into x, h into a separate buffer, act into a contiguous copy of gate
-    act = gate.contiguous()
-    pqk.modulate_swiglu(x, to_dev(e["shift"]), to_dev(e["scale"]), to_dev(e["cu_seqlens"]),
-                        gate_res=to_dev(e["gate_res"]), branch=to_dev_bf16(e["branch"]), gate=act, up=up.contiguous(),
-                        x_out=x, act=act)
-    torch.cuda.synchronize()
-    rxo, rh, ract = oracle.modulate_swiglu(e["x"], e["shift"], e["scale"], e["gate_res"], e["cu_seqlens"],
-                                           branch=e["branch"], gate=e["gate"], up=e["up"])
-    assert_elementwise(bf16_to_f64(x), rxo, "x in place")
-    assert_elementwise(bf16_to_f64(act), ract, "act in place")
+    # x' back into x, h into a separate buffer, act into a contiguous copy of
+    # gate; h must come from x' (formed once from the original x), for both
+    # norms that read the row more than once
+    for norm_type in (pqk.NORM_RMS, pqk.NORM_LAYER):
+        x = to_dev_bf16(e["x"])
+        act = gate.contiguous()
+        _, h, _ = pqk.modulate_swiglu(x, to_dev(e["shift"]), to_dev(e["scale"]), to_dev(e["cu_seqlens"]),
+                                      gate_res=to_dev(e["gate_res"]), branch=to_dev_bf16(e["branch"]), gate=act,
+                                      up=up.contiguous(), x_out=x, act=act, norm_type=norm_type)
+        torch.cuda.synchronize()
+        rxo, rh, ract = oracle.modulate_swiglu(e["x"], e["shift"], e["scale"], e["gate_res"], e["cu_seqlens"],
+                                               branch=e["branch"], gate=e["gate"], up=e["up"], norm_type=norm_type)
+        assert_elementwise(bf16_to_f64(x), rxo, "x in place")
+        assert_elementwise(bf16_to_f64(h), rh, "h with x' written over x")
+        assert_elementwise(bf16_to_f64(act), ract, "act in place")

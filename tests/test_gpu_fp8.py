@@ -391,3 +391,105 @@ def test_full_fp8_skipping_with_infinite_threshold_is_bitwise_the_plain_kernel()
                                      softmax_scale=0.1, want_lse=True)
     torch.cuda.synchronize()
     assert torch.equal(o.view(torch.int16), a[0].view(torch.int16)) and torch.equal(lse, a[1])
+
+
+# ---------------------------------------------------------------- FP8 output of the Q/K prologue
+
+def _prologue_fp32_error(x, w_, pos, eps, base, rows, inv):
+    """Absolute bound on the kernel's fp32 error in y * inv for every element:
+    y = a cos(phi) - b sin(phi) (or a sin + b cos) with a, b the pair's
+    normalised, weighted values. The sum of D squares in fp32 is off by at
+    most D * 2^-24 relative, the reciprocal square root by 2 ulp, so a and b
+    carry at most 2^-17 relative error for D <= 128; the fp32 sine and cosine
+    of the reduced angle (|phi| <= pi) are off by at most 2^-21.41 absolute
+    (CUDA's stated bound for __sincosf there); a handful of fp32 roundings
+    add 2^-20 of the result. So |error| <= inv * ((|a| + |b|) * 2^-17 + |y| * 2^-20)."""
+    zero = np.zeros_like(pos)
+    a = np.abs(oracle.qk_norm_rope(x, w_, zero, eps, base, rows=rows))  # phi = 0: the unrotated values
+    T, H, D = a.shape
+    pair = a.reshape(T, H, D // 2, 2)[..., ::-1].reshape(T, H, D)  # interleaved pairs (2j, 2j+1)
+    y = np.abs(oracle.qk_norm_rope(x, w_, pos, eps, base, rows=rows))
+    return inv * ((a + pair) * 2.0 ** -17 + y * 2.0 ** -20), y * inv
+
+
+def _check_prologue_e4m3(x, w, rows=None, stride_pad=0, what=""):
+    """Codes and scales of pqk_qk_norm_rope_e4m3 against the oracle. The
+    scales are equal bit for bit (the same float arithmetic on both sides).
+    The kernel rounds fp32 values and the oracle float64 ones, so a code may
+    differ only where the oracle's value lies within the kernel's fp32 error
+    bound (_prologue_fp32_error) of an e4m3 rounding boundary, and then it
+    must be the other neighbour of that boundary."""
+    torch = torch_cuda()
+    T, H, D = x["q"].shape
+    if stride_pad:
+        buf = torch.zeros((T, 2 * H * D + stride_pad), dtype=torch.bfloat16, device="cuda")
+        buf[:, :H * D] = to_dev_bf16(x["q"]).view(T, H * D)
+        buf[:, H * D + stride_pad:] = to_dev_bf16(x["k"]).view(T, H * D)
+        q, k = buf[:, :H * D].view(T, H, D), buf[:, H * D + stride_pad:].view(T, H, D)
+    else:
+        q, k = to_dev_bf16(x["q"]), to_dev_bf16(x["k"])
+    q8, k8, deq = pqk.qk_norm_rope_e4m3(q, k, to_dev_bf16(x["w_q"]), to_dev_bf16(x["w_k"]), to_dev(x["pos"]),
+                                         eps=w.eps, rope_base=w.rope_base)
+    torch.cuda.synchronize()
+    assert pqk.get_device_status() == 0
+    d = deq.cpu().numpy()
+    sel = np.arange(T) if rows is None else rows
+    ties = total = 0
+    for i, (name, codes) in enumerate((("q", q8), ("k", k8))):
+        rc, rdeq = oracle.qk_norm_rope_e4m3(x[name], x["w_" + name], x["pos"], w.eps, w.rope_base, rows=rows)
+        assert np.all(d[i * H:(i + 1) * H] == rdeq), f"{what}: {name} scale"
+        g = codes.cpu().numpy()[sel]
+        mism = g != rc
+        if mism.any():
+            inv = 1.0 / float(rdeq)
+            err, scaled = _prologue_fp32_error(x[name], x["w_" + name], x["pos"], w.eps, w.rope_base, rows, inv)
+            y = oracle.qk_norm_rope(x[name], x["w_" + name], x["pos"], w.eps, w.rope_base, rows=rows)
+            v = y[mism] * inv
+            gv = _decode(g[mism])
+            step = _e4m3_quantum(np.abs(v))
+            bad = np.abs(gv - v) > step * 0.5 + err[mism]
+            assert not bad.any(), (f"{what}: {name} code off by more than a rounding boundary plus the fp32 bound: "
+                                   f"{gv[bad][:4]} vs {v[bad][:4]} (bound {err[mism][bad][:4]})")
+        ties += int(mism.sum())
+        total += g.size
+    assert ties <= max(8, total // 200), f"{what}: {ties} of {total} codes differ"
+    return q8, k8, deq
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_prologue_e4m3_configs(cfg):
+    w = wl.config(cfg)
+    _check_prologue_e4m3(wl.prologue_inputs(w), w, what=f"configuration {cfg}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_prologue_e4m3_ragged_and_strided(D):
+    w = wl.custom([300, 0, 17, 129], H=6, D=D, seed=51)
+    _check_prologue_e4m3(wl.prologue_inputs(w), w, stride_pad=64, what=f"ragged strided D{D}")
+
+
+def test_prologue_e4m3_58048_tokens_sampled():
+    w = wl.config(3)
+    _check_prologue_e4m3(wl.prologue_inputs(w), w, rows=wl.sample_rows(w, 256), what="58,048 tokens")
+
+
+def test_prologue_e4m3_feeds_the_fp8_attention():
+    # the fused prologue's codes in the FP8 Q K^T attention = the plain
+    # attention on their dequantised values
+    torch = torch_cuda()
+    w = wl.custom([700, 1300], H=4, D=128, seed=52)
+    x = wl.prologue_inputs(w)
+    v = wl.attention_inputs(w)["v"]
+    q8, k8, deq = _check_prologue_e4m3(x, w, what="feeds the attention")
+    scale = 1.0 / math.sqrt(128)
+    o, lse = pqk.varlen_attn_fwd_fp8qk(q8, k8, to_dev_bf16(v), deq, to_dev(w.cu_seqlens()), softmax_scale=scale,
+                                       want_lse=True)
+    torch.cuda.synchronize()
+    assert pqk.get_device_status() == 0
+    H = w.H
+    dq = deq.cpu().numpy().astype(np.float64)
+    qd = _decode(q8.cpu().numpy()) * dq[None, :H, None]
+    kd = _decode(k8.cpu().numpy()) * dq[None, H:, None]
+    ro, rl = oracle.varlen_attn(qd, kd, wl.bf16_bits_to_f64(v), w.cu_seqlens(), scale)
+    assert_attention(bf16_to_f64(o), ro, "fused prologue -> FP8 attention")
+    assert max_abs(lse.cpu().numpy().astype(np.float64).T, rl) <= LSE_MAX_ABS

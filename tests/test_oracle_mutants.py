@@ -63,8 +63,10 @@ MUTANTS = {
                                        "kd[i] = e4m3_value(kc[i]) * (double)dq[h];"),
     "fp8_amax_of_first_token": ("    for (int64_t t = 0; t < T; ++t)\n      for (int d = 0; d < D; ++d) {\n        const float v = (float)fabs(",
                                 "    for (int64_t t = 0; t < 1; ++t)\n      for (int d = 0; d < D; ++d) {\n        const float v = (float)fabs("),
-    "fp8_range_240": ("const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;",
-                      "const float inv = amax > 0.0f ? 240.0f / amax : 1.0f;"),
+    "fp8_range_240": ("const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;\n    deq[h]",
+                      "const float inv = amax > 0.0f ? 240.0f / amax : 1.0f;\n    deq[h]"),
+    "fp8_prologue_range_240": ("const float inv = amax > 0.0f ? 448.0f / amax : 1.0f;\n    *deq_out",
+                               "const float inv = amax > 0.0f ? 240.0f / amax : 1.0f;\n    *deq_out"),
     "fp8_p_not_quantised": ("\n    const double pq = e4m3_value(e4m3_code((float)pj));", "\n    const double pq = pj;"),
     "fp8_denominator_quantised": ("\n    den += pj;\n", "\n    den += pq;\n"),
     "fp8_reference_first_key": ("    s[j] = scale * dot;\n    if (s[j] > m) m = s[j];",
