@@ -84,6 +84,8 @@ def parse():
                     help="leave out the linear layers with the fused epilogues (gated residual, SwiGLU)")
     ap.add_argument("--no-bw-sweep", action="store_true",
                     help="leave out the HBM-bound kernels on the 40-head sweep shapes at 4,096 and 58,048 tokens")
+    ap.add_argument("--no-pairs", action="store_true",
+                    help="leave out the step's attention timed again on CTA pairs (pqk_set_attn_cta_pairs)")
     ap.add_argument("--graph", action="store_true",
                     help="also time the block call captured once in a CUDA graph and replayed (graph_ms_per_step)")
     ap.add_argument("--skip-tau", type=float, default=8.0,
@@ -572,6 +574,41 @@ def run_ours(args, w):
     fullc_us = ev3[0].elapsed_time(ev3[1]) / reps3 * 1e3
     fullc_gbs = (w.prologue_bytes() + 2 * w.H * w.D * 2) / (fullc_us * 1e-6) / 1e9
 
+    # the step's attention on CTA pairs against the default one-SM kernel,
+    # alternated, ten launches each, with the SM clock sampled meanwhile
+    pairs = None
+    if not args.no_pairs and w.D == 128:
+        po = torch.empty_like(o["o"])
+        run_attn = lambda: pqk.varlen_attn_fwd(o["qn"], o["kn"], d["v"], d["cu"], o=po, workspace=o["ws"])
+        pt = {"one_sm": [], "pairs": []}
+        pclk = {"one_sm": [], "pairs": []}
+        try:
+            for rnd in range(2):
+                for name, on in (("one_sm", False), ("pairs", True)):
+                    pqk.set_attn_cta_pairs(on)
+                    run_attn()
+                    torch.cuda.synchronize()
+                    with ClockSampler(local, enabled=not args.no_clocks) as cs:
+                        ev3[0].record()
+                        for _ in range(10):
+                            run_attn()
+                        ev3[1].record()
+                        torch.cuda.synchronize()
+                    pt[name].append(ev3[0].elapsed_time(ev3[1]) / 10)
+                    summ = cs.summary()
+                    if summ and summ.get("sm_mhz"):
+                        pclk[name].append(summ["sm_mhz"])
+        finally:
+            pqk.set_attn_cta_pairs(False)
+        if pqk.get_device_status() != 0:
+            raise RuntimeError("device status set during the CTA-pair timing")
+        one_ms, pair_ms = min(pt["one_sm"]), min(pt["pairs"])
+        pairs = {"one_sm_ms": one_ms, "pairs_ms": pair_ms, "pairs_tflops": flops / (pair_ms * 1e-3) / 1e12,
+                 "speedup": one_ms / pair_ms,
+                 "one_sm_sm_mhz": statistics.median(pclk["one_sm"]) if pclk["one_sm"] else None,
+                 "pairs_sm_mhz": statistics.median(pclk["pairs"]) if pclk["pairs"] else None}
+        del po
+
     # block skipping (Skip-Softmax) on the local-attention stand-in: Q and K
     # from sinusoids of the (t, h, w) ids plus noise, so that attention weight
     # sits on nearby tokens as in video; plain and skipping kernels on the
@@ -816,6 +853,7 @@ def run_ours(args, w):
                     "qk_norm_rope_back_to_back_us": rope1_b2b_us,
                     "qk_fullc_norm_rope_us": fullc_us, "qk_fullc_norm_rope_gbs": fullc_gbs,
                     "qk_fullc_norm_rope_frac_hbm": fullc_gbs / pk["hbm_gbs"],
+                    "varlen_attn_cta_pairs": pairs,
                     "varlen_attn_skip": skip, "varlen_attn_fp8qk": fp8, "linear_epilogue": lin,
                     "bandwidth_sweep_40_heads": bw},
         "cpu_baseline": cpu,

@@ -468,6 +468,19 @@ PQK_API int pqk_get_device_status(void* stream);
 PQK_API void pqk_set_wait_timeout_ns(int64_t ns);
 
 /*
+ * pqk_set_attn_cta_pairs -- nonzero: pqk_varlen_attn_fwd (and the
+ * no-allocation entry) with bf16 operands and D = 128 runs on CTA pairs:
+ * two SMs share each 512-row work tile, one thread issues the pair's
+ * products with tcgen05 cta_group::2 (M = 256) and each SM streams half of
+ * every K and V tile. The results are bit-identical to the default one-SM
+ * kernel. On B200 it needs about 6 % fewer SM cycles per tile, but under the
+ * 1 kW power cap it runs at a correspondingly lower clock, so the two take
+ * the same time in a long run; hence off by default. Process-wide; affects
+ * calls enqueued afterwards (and graphs captured afterwards).
+ */
+PQK_API void pqk_set_attn_cta_pairs(int enable);
+
+/*
  * pqk_selftest_wait_timeout -- diagnostic: enqueues one thread block that
  * waits, with the bounded wait used by the attention pipeline, on a
  * barrier that nothing completes. The wait runs out after timeout_ns and

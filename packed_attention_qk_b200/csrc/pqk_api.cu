@@ -29,6 +29,7 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 
 std::atomic<long long> g_timeout_ns{1000000000LL};
+std::atomic<int> g_attn_cta_pairs{0};
 
 // Caches the properties of the current device; returns nullptr on failure.
 DeviceInfo* current_device() {
@@ -95,6 +96,8 @@ const char* pqk_status_string(int status) {
 }
 
 const char* pqk_version(void) { return "0.1.0"; }
+
+void pqk_set_attn_cta_pairs(int enable) { g_attn_cta_pairs.store(enable != 0 ? 1 : 0); }
 
 void pqk_set_wait_timeout_ns(int64_t ns) {
   constexpr int64_t kDefault = 1000000000LL, kMin = 1000LL, kMax = 10000000000LL;
@@ -223,7 +226,8 @@ int pqk_varlen_attn_fwd(const void* q, const void* k, const void* v, void* o, fl
   if (int rc = check_device(&d)) return rc;
   const int rc = pqk::launch_varlen_attn(q, k, v, o, lse, q_stride_t, k_stride_t, v_stride_t, o_stride_t,
                                          cu_seqlens, B, T, H, D, softmax_scale, workspace, d->status,
-                                         g_timeout_ns.load(), static_cast<cudaStream_t>(stream), d->num_sms);
+                                         g_timeout_ns.load(), static_cast<cudaStream_t>(stream), d->num_sms, false,
+                                         0.0f, nullptr, nullptr, false, g_attn_cta_pairs.load() != 0);
   return rc == 0 ? PQK_OK : (rc == -2 ? PQK_ERR_INVALID_ARG : PQK_ERR_CUDA);
 }
 

@@ -40,14 +40,16 @@ size_t attn_schedule_bytes(int B);
 // with Q, K given as e4m3 bytes ([T, H, D], strides in bytes) and deq their
 // [2H] per-head dequantisation factors (D = 128; skipping may be combined
 // with it). fp8_pv: V is e4m3 bytes too and P is rounded to e4m3 for P V
-// (deq then [3H], V's last; skipping may be combined with it too). Returns 0, or
-// -1 when a CUDA call failed, -2 when the tensor maps could not be encoded.
+// (deq then [3H], V's last; skipping may be combined with it too). cta_pairs:
+// the bf16, head_dim 128 attention without skipping runs on CTA pairs
+// (tcgen05 cta_group::2). Returns 0, or -1 when a CUDA call failed, -2 when
+// the tensor maps could not be encoded.
 int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, float* lse, int64_t q_stride,
                        int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
                        int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
                        long long timeout_ns, cudaStream_t stream, int num_sms, bool skip = false,
                        float skip_tau = 0.0f, unsigned long long* skip_counts = nullptr,
-                       const float* deq = nullptr, bool fp8_pv = false);
+                       const float* deq = nullptr, bool fp8_pv = false, bool cta_pairs = false);
 
 // Per-head absmax e4m3 quantisation of Q and K ([T, H, D] bf16, strides in
 // elements) into q8, k8 ([T, H, D] bytes, contiguous). scales: [4H] floats,

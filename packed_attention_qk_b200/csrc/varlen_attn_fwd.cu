@@ -51,6 +51,24 @@
 // for that), both bounded by kDrainTimeoutNs rather than the caller's
 // timeout; only then is the tensor memory freed and the block exits.
 //
+// CTA pairs (kPair; bf16, head_dim 128, no block skipping): two CTAs of a
+// cluster share one work tile of 512 query rows, 256 per CTA as above, and
+// one thread of the first CTA (the leader) issues every MMA of the pair with
+// tcgen05 cta_group::2, M = 256: S_i = Q_i K^T over both CTAs' 128-row Q_i
+// with each CTA holding 64 of K_j's 128 keys, and O_i += P_i V_j with P_i in
+// each CTA's tensor memory and each CTA holding 64 of V_j's columns. Each SM
+// thus streams half of every K/V tile (16 KB stages, ten of them) and reads
+// 96 instead of 128 bytes of operands from shared memory per cycle of a
+// Q K^T product, whose one-CTA form is bound by that bandwidth. The leader
+// claims the tiles, posts the bytes of both CTAs' copies on its own
+// barriers before it hands each tile and stage to the second CTA's
+// producer, and commits "S ready" and "O done" to both CTAs' barriers; the
+// second CTA's softmax warps report "P ready" with one remote arrive per
+// warp. On a timeout both CTAs' abort flags are raised; after a cluster
+// barrier the leader drains the copies and MMAs of the pair and a second
+// cluster barrier keeps the second CTA, whose copies signal the leader's
+// barriers, resident until then.
+//
 // Two compile-time variants of the same pipeline:
 //   kSkip  block skipping ("Skip-Softmax", first page, bullet on TRTLLM_ATTN
 //          SAGE and Skip-Softmax): a softmax warp whose 32 rows all have the
@@ -78,7 +96,8 @@ namespace {
 
 constexpr int kBM = 128;          // query rows per Q tile
 constexpr int kBN = 128;          // keys per K/V tile
-constexpr int kRowsPerWork = 2 * kBM;
+constexpr int kRowsPerWork = 2 * kBM;      // one CTA: two 128-row query tiles
+constexpr int kRowsPerPairWork = 4 * kBM;  // a CTA pair: two tiles in each CTA
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -102,14 +121,17 @@ constexpr int kSlabBytes = 128 * 128;      // 128 rows x 64 bf16 (one 128-byte s
 // softmax warps: at most three slots are live.
 constexpr int kWorkSlots = 4;
 
-template <int D>
+template <int D, bool kPair = false>
 struct Layout {
   static constexpr int kSlabs = D / 64;
-  static constexpr int kTileBytes = kSlabs * kSlabBytes;
-  static constexpr int kStages = D == 128 ? 5 : 10;
+  static constexpr int kTileBytes = kSlabs * kSlabBytes;  // a Q tile; a whole K or V tile
+  // a K/V stage: a whole tile, or on a CTA pair this CTA's half (64 keys of
+  // K; 64 of V's columns for all 128 keys)
+  static constexpr int kStageBytes = kPair ? kTileBytes / 2 : kTileBytes;
+  static constexpr int kStages = (kPair || D != 128) ? 10 : 5;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kStageBytes;
   // barriers: kv_full[S], kv_empty[S], q_full, q_empty, s_full[2], p_full[2], o_done[2], drain,
   // work_full[kWorkSlots]
   static constexpr int kNumBars = 2 * kStages + 9 + kWorkSlots;
@@ -129,7 +151,7 @@ struct Layout {
 
 // Schedule in the workspace (int32): [0] number of work tiles, [1] number of
 // requests B, [2] the claim counter (reset to 0 by the schedule kernel on
-// every call), [3] unused, then for the requests in schedule order r =
+// every call), [3] query rows per work tile, then for the requests in schedule order r =
 // 0..B-1: tile_start[B+1] (prefix of tiles), seg_start[B], seg_len[B].
 constexpr int kSchedHeader = 4;
 __host__ __device__ constexpr size_t sched_words(int B) {
@@ -172,10 +194,11 @@ __device__ __forceinline__ Work decode_work(const int32_t* sched, int H, int w) 
   Work wk;
   wk.seg_start = seg_start[lo];
   wk.seg_len = seg_len[lo];
-  const int nqb = (wk.seg_len + kRowsPerWork - 1) / kRowsPerWork;
+  const int rows_per_work = sched[3];
+  const int nqb = (wk.seg_len + rows_per_work - 1) / rows_per_work;
   const int local = w - tile_start[lo];
   wk.head = local / nqb;
-  wk.q0 = wk.seg_start + (local % nqb) * kRowsPerWork;
+  wk.q0 = wk.seg_start + (local % nqb) * rows_per_work;
   wk.n_kv = (wk.seg_len + kBN - 1) / kBN;
   (void)H;
   return wk;
@@ -208,6 +231,10 @@ __device__ __noinline__ void drain_mmas(uint32_t bar_drain) {
   tc_commit(bar_drain);
   mbar_drain_wait(bar_drain, 0);
 }
+__device__ __noinline__ void drain_mmas_pair(uint32_t bar_drain) {
+  tc_commit_pair(bar_drain);
+  mbar_drain_wait(bar_drain, 0);
+}
 
 // ------------------------------------------------------------ schedule
 
@@ -217,7 +244,8 @@ constexpr int kSortLimit = 8192;  // requests ordered longest first up to this B
 constexpr int kSchedSmem = kSortLimit * 8;
 
 __global__ void __launch_bounds__(kSchedThreads) build_schedule_kernel(const int32_t* cu, int B, int64_t T, int H,
-                                                                        int32_t* sched, int* status) {
+                                                                        int rows_per_work, int32_t* sched,
+                                                                        int* status) {
   extern __shared__ uint64_t sort_keys[];
   __shared__ int bad;
   __shared__ int32_t carry;
@@ -237,6 +265,7 @@ __global__ void __launch_bounds__(kSchedThreads) build_schedule_kernel(const int
       sched[0] = 0;
       sched[1] = B;
       sched[2] = 0;
+      sched[3] = rows_per_work;
       atomicCAS(status, 0, kStatusBadSeqlens);
     }
     return;
@@ -285,7 +314,7 @@ __global__ void __launch_bounds__(kSchedThreads) build_schedule_kernel(const int
   __shared__ int32_t warp_sums[kSchedThreads / 32];
   for (int base = 0; base < B; base += kSchedThreads) {
     const int i = base + threadIdx.x;
-    const int32_t n = i < B ? ((seg_len[i] + kRowsPerWork - 1) / kRowsPerWork) * H : 0;
+    const int32_t n = i < B ? ((seg_len[i] + rows_per_work - 1) / rows_per_work) * H : 0;
     int32_t incl = n;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -306,6 +335,7 @@ __global__ void __launch_bounds__(kSchedThreads) build_schedule_kernel(const int
     sched[0] = carry;
     sched[1] = B;
     sched[2] = 0;  // claim counter
+    sched[3] = rows_per_work;
   }
 }
 
@@ -411,13 +441,14 @@ __device__ __forceinline__ float exp_tile_store(const float (&s)[128], float sca
   return (l0 + l1) + (l2 + l3);
 }
 
-template <int D, bool kSkip, bool kFp8, bool kFp8Pv>
+template <int D, bool kSkip, bool kFp8, bool kFp8Pv, bool kPair = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using L = Layout<D>;
+  using L = Layout<D, kPair>;
   static_assert(!kFp8 || D == 128, "FP8 Q K^T: one 128-byte swizzle row per token");
   static_assert(!kFp8Pv || kFp8, "FP8 P V comes with FP8 Q K^T");
+  static_assert(!kPair || (D == 128 && !kSkip && !kFp8), "CTA pairs: bf16, head_dim 128, no block skipping");
   // FP8 Q K^T: the MMA thread waits for the next V stage (loaded long ago)
   // while it waits for P1 anyway, and probes the next K stage there without
   // blocking (its copy may still be in flight), instead of waiting for both
@@ -433,6 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pair: rank 0 (the leader) issues every MMA of the pair and owns the
+  // barriers of the K/V and Q copies; each CTA keeps its own 256 query rows
+  const uint32_t rank = kPair ? ctarank() : 0u;
+  const bool leader = rank == 0;
   const uint32_t q_smem = base + L::kQOff;
   const uint32_t kv_smem = base + L::kKVOff;
   const uint32_t bar0 = base + L::kBarOff;
@@ -449,6 +484,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlotOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbortOff);
   volatile uint8_t* votes = smem + L::kVoteOff;
+  // a wait that ran out stops this CTA's roles and, on a pair, the other CTA's
+  auto abort_all = [&]() {
+    raise_abort(abort_flag, p.status);
+    if constexpr (kPair) st_remote_u32(in_cta(base + L::kAbortOff, rank ^ 1u), 1u);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -459,7 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(p_full(i), kBM);
+      // one arrival per softmax thread, or on a pair one per softmax warp of either CTA
+      mbar_init(p_full(i), kPair ? 8 : kBM);
       mbar_init(o_done(i), 1);
     }
     mbar_init(drain, 1);
@@ -468,8 +509,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(base + L::kTmemSlotOff, 512);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(base + L::kTmemSlotOff, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(base + L::kTmemSlotOff, 512);
+      tmem_relinquish();
+    }
   }
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tensor_map(&tm_q);
@@ -477,7 +523,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensor_map(&tm_v);
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (kPair) {
+    __syncwarp();
+    cluster_sync_all();  // both CTAs' barriers are initialised before any remote arrive
+  } else {
+    __syncthreads();
+  }
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const int n_work = p.sched[0];
@@ -490,6 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // block aborts first.
   auto next_work = [&](int wt, int& w) {
     if (!mbar_wait(work_full(wt % kWorkSlots), (wt / kWorkSlots) & 1, abort_flag, p.timeout_ns)) return false;
+    // on a pair's second CTA the slot was written by the leader's producer
+    if (kPair && !leader) asm volatile("fence.acq_rel.cluster;" ::: "memory");
     w = work_slot[wt % kWorkSlots];
     return true;
   };
@@ -500,6 +553,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t load_idx = 0;
       uint32_t q_loads = 0;
       bool ok = true;
+      if constexpr (kPair) {
+        // The leader claims each work tile, posts the bytes of both CTAs'
+        // copies on its own barriers and only then hands the tile, and each
+        // K/V stage, to the second CTA's producer (so that no copy completes
+        // before the count it belongs to). Both CTAs copy their own two Q
+        // tiles, their 64 of each K tile's keys and their 64 of each V
+        // tile's columns; every copy completes on the leader's barrier.
+        const uint32_t q_bar = in_cta(q_full, 0);
+        for (int wt = 0; ok; ++wt) {
+          int w;
+          if (leader) {
+            if (wt > 0 && !(ok = mbar_wait(q_empty, (wt - 1) & 1, abort_flag, p.timeout_ns))) break;
+            const int claimed = atomicAdd(claim_counter, 1);
+            w = claimed < n_work ? claimed : -1;
+            if (w >= 0) {
+              mbar_arrive_expect_tx(q_full, 4 * kQKBytes);
+              ++q_loads;
+            }
+            work_slot[wt % kWorkSlots] = w;
+            mbar_arrive(work_full(wt % kWorkSlots));
+            st_remote_u32(in_cta(base + L::kWorkOff + 4u * (wt % kWorkSlots), 1), static_cast<uint32_t>(w));
+            arrive_remote_release(in_cta(work_full(wt % kWorkSlots), 1));
+          } else if (!(ok = next_work(wt, w))) {
+            break;
+          }
+          if (w < 0) break;
+          const Work wk = decode_work(p.sched, p.H, w);
+          const int qrow = wk.q0 + static_cast<int>(rank) * kRowsPerWork;
+          for (int i = 0; i < 2; ++i)
+            for (int sl = 0; sl < L::kSlabs; ++sl)
+              tma_load_3d_pair(q_smem + i * L::kTileBytes + sl * kSlabBytes, &tm_q, q_bar, sl * 64, wk.head,
+                               qrow + i * kBM);
+          for (int j = 0; j < wk.n_kv && ok; ++j) {
+            const int key0 = wk.seg_start + j * kBN;
+            for (int kv = 0; kv < 2; ++kv) {
+              const int s = load_idx % L::kStages;
+              const uint32_t round = load_idx / L::kStages;
+              if (leader) {
+                if (round > 0 && !(ok = mbar_wait(kv_empty(s), (round - 1) & 1, abort_flag, p.timeout_ns))) break;
+                mbar_arrive_expect_tx(kv_full(s), 2 * L::kStageBytes);
+                arrive_remote(in_cta(kv_empty(s), 1));
+              } else if (!(ok = mbar_wait(kv_empty(s), round & 1, abort_flag, p.timeout_ns))) {
+                break;
+              }
+              const uint32_t dst = kv_smem + s * L::kStageBytes;
+              const uint32_t bar = in_cta(kv_full(s), 0);
+              if (kv == 0) {
+                for (int sl = 0; sl < L::kSlabs; ++sl)
+                  tma_load_3d_pair(dst + sl * (kSlabBytes / 2), &tm_k, bar, sl * 64, wk.head,
+                                   key0 + static_cast<int>(rank) * (kBN / 2));
+              } else {
+                tma_load_3d_pair(dst, &tm_v, bar, static_cast<int>(rank) * 64, wk.head, key0);
+              }
+              ++load_idx;
+            }
+          }
+        }
+      } else {
       for (int wt = 0; ok; ++wt) {
         // the Q tiles of the previous work tile are no longer needed: claim the next one
         if (wt > 0 && !(ok = mbar_wait(q_empty, (wt - 1) & 1, abort_flag, p.timeout_ns))) break;
@@ -528,28 +639,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             if ((kFp8 && kv == 0) || (kFp8Pv && kv == 1)) {
               // one 128-byte e4m3 row per token: a single 16 KB box
               mbar_arrive_expect_tx(kv_full(s), kQKBytes);
-              tma_load_3d(kv_smem + s * L::kTileBytes, kv == 0 ? &tm_k : &tm_v, kv_full(s), 0, wk.head,
+              tma_load_3d(kv_smem + s * L::kStageBytes, kv == 0 ? &tm_k : &tm_v, kv_full(s), 0, wk.head,
                           wk.seg_start + j * kBN);
             } else {
               mbar_arrive_expect_tx(kv_full(s), L::kTileBytes);
               const CUtensorMap* tm = kv == 0 ? &tm_k : &tm_v;
               for (int sl = 0; sl < L::kSlabs; ++sl)
-                tma_load_3d(kv_smem + s * L::kTileBytes + sl * kSlabBytes, tm, kv_full(s), sl * 64, wk.head,
+                tma_load_3d(kv_smem + s * L::kStageBytes + sl * kSlabBytes, tm, kv_full(s), sl * 64, wk.head,
                             wk.seg_start + j * kBN);
             }
             ++load_idx;
           }
         }
       }
-      if (!ok) raise_abort(abort_flag, p.status);
+      }
+      if (!ok) abort_all();
       loads_done[0] = load_idx;
       loads_done[1] = q_loads;
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdescQK = kFp8 ? idesc_e4m3_f32(kBM, kBN) : idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
+    // ------------------------------------------------ MMA issuer (the leader's, on a pair)
+    if (lane == 0 && leader) {
+      // a pair's products have M = 256: each CTA's 128 rows of Q_i, S_i, P_i, O_i
+      constexpr int kM = kPair ? 2 * kBM : kBM;
+      constexpr uint32_t kIdescQK = kFp8 ? idesc_e4m3_f32(kBM, kBN) : idesc_bf16_f32(kM, kBN, false);
+      constexpr uint32_t kIdescPV = idesc_bf16_f32(kM, D, true);
+      // completions: of this CTA's copies' consumers (stages, Q), or seen by
+      // both CTAs' softmax warps (S ready, O done)
+      auto commit_own = [&](uint32_t bar) {
+        if constexpr (kPair) tc_commit_pair(bar); else tc_commit(bar);
+      };
+      auto commit_all = [&](uint32_t bar) {
+        if constexpr (kPair) tc_commit_pair_both(bar); else tc_commit(bar);
+      };
       constexpr uint32_t kIdescPV8 = idesc_e4m3_f32(kBM, D, true);
       uint32_t cons_idx = 0;
       uint32_t p_phase = 0;
@@ -564,13 +686,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // with 64-wide column slabs kSlabBytes apart); one high word for all.
       constexpr uint32_t kDescHi = smem_desc_hi_sw128(1024);
       constexpr uint32_t kTileWords = L::kTileBytes >> 4;
+      constexpr uint32_t kStageWords = L::kStageBytes >> 4;
+      // a K stage's two 64-column slabs (on a pair 64 keys each)
+      constexpr uint32_t kKSlabBytes = kPair ? kSlabBytes / 2 : kSlabBytes;
       const uint32_t q_lo = smem_desc_lo(q_smem, 16);
       const uint32_t k_lo = smem_desc_lo(kv_smem, 16);
       const uint32_t v_lo = smem_desc_lo(kv_smem, kSlabBytes);
       // S_i = Q_i K^T over D/16 K-steps of 16 (32 bytes inside the 128-byte row)
       auto issue_qk = [&](int i, int stage) {
         const uint32_t a0 = q_lo + i * kTileWords;
-        const uint32_t b0 = k_lo + stage * kTileWords;
+        const uint32_t b0 = k_lo + stage * kStageWords;
         if constexpr (kFp8) {
           // e4m3: K = 32 per instruction, 32 bytes inside the one 128-byte row
 #pragma unroll
@@ -580,16 +705,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = ((k / 4) * kSlabBytes + (k % 4) * 32) >> 4;
-            mma_bf16_ss_w(tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1), a0 + off, b0 + off, kDescHi, kIdescQK,
-                          k > 0 ? 1u : 0u);
+            const uint32_t off_a = ((k / 4) * kSlabBytes + (k % 4) * 32) >> 4;
+            const uint32_t off_b = ((k / 4) * kKSlabBytes + (k % 4) * 32) >> 4;
+            if constexpr (kPair)
+              mma_bf16_ss_pair(tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1), a0 + off_a, b0 + off_b, kDescHi, kIdescQK,
+                               k > 0 ? 1u : 0u);
+            else
+              mma_bf16_ss_w(tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1), a0 + off_a, b0 + off_b, kDescHi, kIdescQK,
+                            k > 0 ? 1u : 0u);
           }
         }
       };
       // O_i (+)= P_i V over kBN/16 K-steps; V is MN-major: 64-wide column
       // slabs kSlabBytes apart, 8-row groups 1024 bytes apart
       auto issue_pv = [&](int i, int stage, bool accumulate) {
-        const uint32_t b0 = v_lo + stage * kTileWords;
+        const uint32_t b0 = v_lo + stage * kStageWords;
         const uint32_t p_col = tmem + (i == 0 ? L::kTmemS0 : L::kTmemS1);
         if constexpr (kFp8Pv) {
           // e4m3 P (four keys per column, 8 columns per K = 32 step) and V as
@@ -601,8 +731,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int k = 0; k < kBN / 16; ++k) {
-            mma_bf16_ts_w(tmem + (i == 0 ? L::kTmemO0 : L::kTmemO1), p_col + 8 * k, b0 + ((k * 2048) >> 4),
-                          kDescHi, kIdescPV, (accumulate || k > 0) ? 1u : 0u);
+            if constexpr (kPair)
+              mma_bf16_ts_pair(tmem + (i == 0 ? L::kTmemO0 : L::kTmemO1), p_col + 8 * k, b0 + ((k * 2048) >> 4),
+                               kDescHi, kIdescPV, (accumulate || k > 0) ? 1u : 0u);
+            else
+              mma_bf16_ts_w(tmem + (i == 0 ? L::kTmemO0 : L::kTmemO1), p_col + 8 * k, b0 + ((k * 2048) >> 4),
+                            kDescHi, kIdescPV, (accumulate || k > 0) ? 1u : 0u);
           }
         }
       };
@@ -619,11 +753,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait_stage(k_stage_idx))) break;
         tc_fence_after_sync();
         issue_qk(0, k_stage_idx % L::kStages);
-        tc_commit(s_full(0));
+        commit_all(s_full(0));
         issue_qk(1, k_stage_idx % L::kStages);
-        tc_commit(s_full(1));
-        tc_commit(kv_empty(k_stage_idx % L::kStages));
-        if (wk.n_kv == 1) tc_commit(q_empty);
+        commit_all(s_full(1));
+        commit_own(kv_empty(k_stage_idx % L::kStages));
+        if (wk.n_kv == 1) commit_own(q_empty);
         ++cons_idx;
         // stages of iteration j: V_j and K_{j+1}
         uint32_t v_idx = cons_idx++;
@@ -642,10 +776,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             issue_pv(0, v_idx % L::kStages, j > 0);
           }
-          if (!more) tc_commit(o_done(0));
+          if (!more) commit_all(o_done(0));
           if (more) {
             issue_qk(0, nk_idx % L::kStages);
-            tc_commit(s_full(0));
+            commit_all(s_full(0));
           }
           uint32_t next_v = 0, next_nk = 0;
           if (more) {
@@ -666,13 +800,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             issue_pv(1, v_idx % L::kStages, j > 0);
           }
-          if (!more) tc_commit(o_done(1));
-          tc_commit(kv_empty(v_idx % L::kStages));
+          if (!more) commit_all(o_done(1));
+          commit_own(kv_empty(v_idx % L::kStages));
           if (more) {
             issue_qk(1, nk_idx % L::kStages);
-            tc_commit(s_full(1));
-            tc_commit(kv_empty(nk_idx % L::kStages));
-            if (j + 2 == wk.n_kv) tc_commit(q_empty);
+            commit_all(s_full(1));
+            commit_own(kv_empty(nk_idx % L::kStages));
+            if (j + 2 == wk.n_kv) commit_own(q_empty);
           }
           p_phase ^= 1u;
           v_idx = next_v;
@@ -680,7 +814,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (kSkip && p.skip_counts != nullptr && pv_skips != 0) atomicAdd(&p.skip_counts[1], pv_skips);
-      if (!ok) raise_abort(abort_flag, p.status);
+      if (!ok) abort_all();
     }
   } else {
     // ------------------------------------------------ softmax groups
@@ -698,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, next_work(wt, w));
       if (!ok || w < 0) break;
       const Work wk = decode_work(p.sched, p.H, w);
-      const int row = wk.q0 + grp * kBM + r;
+      const int row = wk.q0 + static_cast<int>(rank) * kRowsPerWork + grp * kBM + r;
       // log2-domain score factor; FP8 scores carry the two heads' dequantisation factors
       const float sl2 = kFp8 ? p.scale_log2 * p.deq[wk.head] * p.deq[p.H + wk.head] : p.scale_log2;
       float m = -INFINITY, l = 0.f;
@@ -770,7 +904,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l += exp_tile_store<kFp8Pv>(s, sl2, -m, t_s);
         tc_fence_before_sync();
-        mbar_arrive(p_full(grp));
+        if constexpr (kPair) {
+          // one arrival per warp at the leader's barrier. P and the rescaled
+          // O are in this CTA's tensor memory, their stores complete
+          // (tcgen05.wait::st) and fenced before this point, so a plain
+          // remote arrive hands them over; a cluster-scope release here,
+          // on every tile's critical path, cost 15 % of the kernel's time
+          __syncwarp();
+          if (lane == 0) {
+            if (leader) mbar_arrive(p_full(grp));
+            else arrive_remote(in_cta(p_full(grp), 0));
+          }
+        } else {
+          mbar_arrive(p_full(grp));
+        }
       }
       if (!ok) break;
       // epilogue: normalise O_i and write the valid rows
@@ -802,23 +949,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before_sync();
     }
     if (kSkip && p.skip_counts != nullptr && lane == 0 && warp_skips != 0) atomicAdd(&p.skip_counts[0], warp_skips);
-    if (!ok) raise_abort(abort_flag, p.status);
+    if (!ok) abort_all();
   }
 
   tc_fence_before_sync();
-  __syncthreads();
-  // Every role has stopped, so the abort flag is final. On an abort, copies
-  // and MMAs may still be in flight into this block's shared and tensor
-  // memory: wait for all of them before the memory is freed.
+  auto block_sync = [&]() {
+    if constexpr (kPair) {
+      __syncwarp();
+      cluster_sync_all();
+    } else {
+      __syncthreads();
+    }
+  };
+  block_sync();
+  // Every role (of both CTAs, on a pair) has stopped, so the abort flag is
+  // final. On an abort, copies and MMAs may still be in flight into the
+  // block's shared and tensor memory: wait for all of them before the memory
+  // is freed. On a pair every copy completes on a leader's barrier, which
+  // completes only once both CTAs' halves have landed; the second CTA waits
+  // at the cluster barrier meanwhile.
   if (*abort_flag) {
-    if (warp == kProducerWarp && lane == 0)
+    if (leader && warp == kProducerWarp && lane == 0)
       drain_copies(kv_full(0), q_full, L::kStages, loads_done[0], loads_done[1]);
-    else if (warp == kMmaWarp && lane == 0)
-      drain_mmas(drain);
-    __syncthreads();
+    else if (leader && warp == kMmaWarp && lane == 0)
+      kPair ? drain_mmas_pair(drain) : drain_mmas(drain);
+    block_sync();
   }
   tc_fence_after_sync();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  if (warp == kMmaWarp) {
+    if constexpr (kPair) tmem_dealloc_pair(tmem, 512); else tmem_dealloc(tmem, 512);
+  }
 }
 
 // ------------------------------------------------------------ self-test
@@ -859,13 +1019,13 @@ EncodeTiledFn encode_fn() {
 }
 
 // [T, H, D] bf16 with `stride` elements between tokens, read as boxes of
-// 64 columns x 1 head x 128 tokens, 128-byte swizzled; rows past T read as 0.
-bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t T, int H, int D, int64_t stride) {
+// 64 columns x 1 head x box_rows tokens, 128-byte swizzled; rows past T read as 0.
+bool make_qkv_map(CUtensorMap* map, const void* ptr, int64_t T, int H, int D, int64_t stride, int box_rows = kBM) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(stride) * 2};
-  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kBM)};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -899,6 +1059,49 @@ bool set_schedule_smem_attr() {
   return true;
 }
 
+// Per device: the shared-memory attribute of the pair kernel is set and the
+// number of CTA pairs that can be resident at once is queried on the first
+// call (which must precede any stream capture), so that the persistent grid
+// never leaves a pair waiting for a second wave.
+int resident_attn_pairs(cudaLaunchConfig_t* cfg) {
+  static int pairs[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (pairs[dev] == 0) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<128, false, false, false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<128, true>::kAlloc) != cudaSuccess)
+      return -1;
+    int n = 0;
+    cfg->gridDim = dim3(2, 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&n, attn_fwd_kernel<128, false, false, false, true>, cfg) != cudaSuccess ||
+        n < 1)
+      return -1;
+    pairs[dev] = n;
+  }
+  return pairs[dev];
+}
+
+int launch_attn_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
+                     int64_t max_work, cudaStream_t stream) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Layout<128, true>::kAlloc;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int max_pairs = resident_attn_pairs(&cfg);
+  if (max_pairs < 1) return -1;
+  cfg.gridDim = dim3(2 * static_cast<unsigned>(max_work < max_pairs ? max_work : max_pairs), 1, 1);
+  if (cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, false, false, false, true>, tq, tk, tv, p) != cudaSuccess)
+    return -1;
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
 template <int D, bool kSkip, bool kFp8, bool kFp8Pv>
 bool set_smem_attr() {
   static int done[64] = {0};
@@ -921,19 +1124,25 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
                        int64_t k_stride, int64_t v_stride, int64_t o_stride, const int32_t* cu_seqlens, int B,
                        int64_t T, int H, int D, float softmax_scale, void* workspace, int* status,
                        long long timeout_ns, cudaStream_t stream, int num_sms, bool skip, float skip_tau,
-                       unsigned long long* skip_counts, const float* deq, bool fp8_pv) {
+                       unsigned long long* skip_counts, const float* deq, bool fp8_pv, bool cta_pairs) {
   CUtensorMap tq, tk, tv;
   const bool maps_ok = deq != nullptr
                            ? make_e4m3_map(&tq, q, T, H, D, q_stride) && make_e4m3_map(&tk, k, T, H, D, k_stride)
                            : make_qkv_map(&tq, q, T, H, D, q_stride) && make_qkv_map(&tk, k, T, H, D, k_stride);
   const bool v_ok = fp8_pv ? make_e4m3_map(&tv, v, T, H, D, v_stride) : make_qkv_map(&tv, v, T, H, D, v_stride);
   if (!maps_ok || !v_ok) return -2;
+  // bf16, head_dim 128, no block skipping: on CTA pairs when asked, whose K
+  // copies are 64-key halves
+  const bool pair = cta_pairs && deq == nullptr && !skip && D == 128;
+  if (pair && !make_qkv_map(&tk, k, T, H, D, k_stride, kBN / 2)) return -2;
+  const int rows_per_work = pair ? kRowsPerPairWork : kRowsPerWork;
   int32_t* sched = static_cast<int32_t*>(workspace);
   int sort_n = 1;
   while (sort_n < B) sort_n <<= 1;
   const size_t sched_smem = B <= kSortLimit ? static_cast<size_t>(sort_n) * 8 : 0;
   if (sched_smem > 48 * 1024 && !set_schedule_smem_attr()) return -1;
-  build_schedule_kernel<<<1, kSchedThreads, sched_smem, stream>>>(cu_seqlens, B, T, H, sched, status);
+  build_schedule_kernel<<<1, kSchedThreads, sched_smem, stream>>>(cu_seqlens, B, T, H, rows_per_work, sched,
+                                                                  status);
   if (cudaGetLastError() != cudaSuccess) return -1;
   AttnParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -949,8 +1158,9 @@ int launch_varlen_attn(const void* q, const void* k, const void* v, void* o, flo
   p.skip_counts = skip_counts;
   p.deq = deq;
   // upper bound of work tiles: every request adds at most one partial block
-  const int64_t max_work = static_cast<int64_t>(H) * ((T + kRowsPerWork - 1) / kRowsPerWork + B);
+  const int64_t max_work = static_cast<int64_t>(H) * ((T + rows_per_work - 1) / rows_per_work + B);
   const int grid = static_cast<int>(max_work < num_sms ? max_work : num_sms);
+  if (pair) return launch_attn_pair(tq, tk, tv, p, max_work, stream);
   if (fp8_pv && !skip) {
     if (D != 128 || deq == nullptr) return -1;
     if (!set_smem_attr<128, false, true, true>()) return -1;

@@ -26,7 +26,8 @@ EXPORTS = ("pqk_qk_norm_rope", "pqk_qk_norm_rope_e4m3", "pqk_qk_norm_rope_3axis"
            "pqk_varlen_attn_fwd_skip", "pqk_quantize_qk_e4m3", "pqk_varlen_attn_fwd_fp8qk", "pqk_quantize_e4m3",
            "pqk_varlen_attn_fwd_fp8",
            "pqk_varlen_attn_fwd_noalloc", "pqk_modulate_swiglu", "pqk_linear_gated_residual", "pqk_linear_swiglu",
-           "pqk_get_device_status", "pqk_set_wait_timeout_ns", "pqk_selftest_wait_timeout", "pqk_status_string",
+           "pqk_get_device_status", "pqk_set_wait_timeout_ns", "pqk_set_attn_cta_pairs", "pqk_selftest_wait_timeout",
+           "pqk_status_string",
            "pqk_version")
 
 
@@ -91,6 +92,8 @@ def lib(path: str | None = None) -> C.CDLL:
     L.pqk_get_device_status.restype = i32
     L.pqk_set_wait_timeout_ns.argtypes = [i64]
     L.pqk_set_wait_timeout_ns.restype = None
+    L.pqk_set_attn_cta_pairs.argtypes = [C.c_int]
+    L.pqk_set_attn_cta_pairs.restype = None
     L.pqk_selftest_wait_timeout.argtypes = [i64, vp]
     L.pqk_selftest_wait_timeout.restype = i32
     L.pqk_status_string.argtypes = [i32]
@@ -420,6 +423,11 @@ def get_device_status(stream=None) -> int:
 
 def set_wait_timeout_ns(ns: int) -> None:
     lib().pqk_set_wait_timeout_ns(int(ns))
+
+
+def set_attn_cta_pairs(enable: bool) -> None:
+    """The bf16, head_dim 128 attention on CTA pairs (bit-identical results)."""
+    lib().pqk_set_attn_cta_pairs(1 if enable else 0)
 
 
 def selftest_wait_timeout(timeout_ns: int, stream=None) -> None:
