@@ -473,10 +473,12 @@ PQK_API void pqk_set_wait_timeout_ns(int64_t ns);
  * two SMs share each 512-row work tile, one thread issues the pair's
  * products with tcgen05 cta_group::2 (M = 256) and each SM streams half of
  * every K and V tile. The results are bit-identical to the default one-SM
- * kernel. On B200 it needs about 6 % fewer SM cycles per tile, but under the
- * 1 kW power cap it runs at a correspondingly lower clock, so the two take
- * the same time in a long run; hence off by default. Process-wide; affects
- * calls enqueued afterwards (and graphs captured afterwards).
+ * kernel. On B200 it halves the L2-to-SM traffic and cuts the tensor cores'
+ * shared-memory reads by a third, but the cross-CTA hand-offs lengthen each
+ * tile's critical chain: in the 58,048-token step the two take the same
+ * time, and a 16,384-token launch takes 5 % more cycles; hence off by
+ * default. Process-wide; affects calls enqueued afterwards (and graphs
+ * captured afterwards).
  */
 PQK_API void pqk_set_attn_cta_pairs(int enable);
 
