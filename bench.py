@@ -826,7 +826,10 @@ def run_ours(args, w):
         tf, secs, nrows, cores = cpu_baseline_sample(w, 96)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                "sample": f"attention of {nrows} seeded query rows x {w.H} heads over all keys of their request "
-                         f"(float64 oracle, {secs:.1f} s)"}
+                         f"(float64 oracle, {secs:.1f} s)",
+               "per_row_ms": secs / nrows * 1e3,
+               "extrapolated_full_call_s": w.attn_flops() / (tf * 1e12),
+               "extrapolation": "the whole attention at the sample's rate (not measured)"}
 
     traffic = attn_traffic()
     peak = pk["bf16_tflops_sustained"]
