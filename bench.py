@@ -393,6 +393,29 @@ def cpu_baseline_sample(w, rows_per_request, seed_rows=None):
     return flops / dt / 1e12, dt, int(len(rows)), oracle.num_threads()
 
 
+def cpu_elementwise_sample(w, n_tokens=16384):
+    """Times the oracle's Q/K norm + RoPE and its modulation + SwiGLU on a
+    seeded sample of the step's tokens (the step's shapes, residual branch
+    on). Returns ({qk_norm_rope_gbs, modulate_swiglu_gbs}, seconds, tokens)."""
+    from oracle import oracle
+    from packed_attention_qk_b200 import workloads as wl
+    p = wl.prologue_inputs(w)
+    e = wl.epilogue_inputs(w, with_branch=True)
+    rows = np.sort(np.random.default_rng(w.seed + 2000).choice(w.T, size=min(n_tokens, w.T), replace=False))
+    rows = rows.astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.qk_norm_rope(p["q"], p["w_q"], p["pos"], w.eps, w.rope_base, rows=rows)
+    oracle.qk_norm_rope(p["k"], p["w_k"], p["pos"], w.eps, w.rope_base, rows=rows)
+    t1 = time.perf_counter()
+    oracle.modulate_swiglu(e["x"], e["shift"], e["scale"], e["gate_res"], e["cu_seqlens"], eps=w.eps,
+                           branch=e["branch"], gate=e["gate"], up=e["up"], rows=rows)
+    t2 = time.perf_counter()
+    n = len(rows)
+    pro = w.prologue_bytes() / w.T * n / (t1 - t0) / 1e9
+    epi = w.epilogue_bytes(with_branch=True) / w.T * n / (t2 - t1) / 1e9
+    return {"qk_norm_rope_gbs": pro, "modulate_swiglu_gbs": epi}, t2 - t0, n
+
+
 # ------------------------------------------------------------------ arms
 
 def run_reference(args, w):
@@ -830,6 +853,11 @@ def run_ours(args, w):
                "per_row_ms": secs / nrows * 1e3,
                "extrapolated_full_call_s": w.attn_flops() / (tf * 1e12),
                "extrapolation": "the whole attention at the sample's rate (not measured)"}
+        el, el_secs, el_n = cpu_elementwise_sample(w)
+        cpu["elementwise"] = {**el, "unit": "GB/s", "kind": "oracle",
+                              "sample": f"Q/K norm + RoPE and modulation + SwiGLU (residual branch on) of {el_n} "
+                                        f"seeded tokens of the step, counted as their algorithmic bytes "
+                                        f"(float64 oracle, {el_secs:.1f} s)"}
 
     traffic = attn_traffic()
     peak = pk["bf16_tflops_sustained"]
