@@ -377,13 +377,21 @@ def time_bandwidth_sweep(w_step, dev, pk, pk_kind, tokens=(4096, 58048), reps=10
 
 # ------------------------------------------------------------------ CPU oracle
 
-def cpu_baseline_sample(w, rows_per_request, seed_rows=None):
+def cpu_baseline_sample(w, rows_per_request, seed_rows=None, threads=None):
     """Times the oracle's attention on a seeded sample of query rows (all
-    heads, full keys). Returns (TFLOP/s, seconds, rows, threads)."""
+    heads, full keys), on `threads` OpenMP threads (all of them by default).
+    Returns (TFLOP/s, seconds, rows, threads)."""
     from oracle import oracle
     from packed_attention_qk_b200 import workloads as wl
     x = wl.attention_inputs(w)
     rows = wl.sample_rows(w, rows_per_request)
+    if threads is not None:
+        all_threads = oracle.num_threads()
+        oracle.set_num_threads(threads)
+        try:
+            return cpu_baseline_sample(w, rows_per_request, seed_rows)
+        finally:
+            oracle.set_num_threads(all_threads)
     cu = w.cu_seqlens()
     seg = np.searchsorted(cu, rows, side="right") - 1
     flops = float(sum(4.0 * w.H * w.D * (cu[s + 1] - cu[s]) for s in seg))
@@ -853,6 +861,10 @@ def run_ours(args, w):
                "per_row_ms": secs / nrows * 1e3,
                "extrapolated_full_call_s": w.attn_flops() / (tf * 1e12),
                "extrapolation": "the whole attention at the sample's rate (not measured)"}
+        tf1, secs1, nrows1, _ = cpu_baseline_sample(w, 4, threads=1)
+        cpu["single_thread"] = {"value": tf1, "unit": "TFLOP/s", "cores": 1,
+                                "sample": f"attention of {nrows1} seeded query rows x {w.H} heads "
+                                          f"(float64 oracle, {secs1:.1f} s)"}
         el, el_secs, el_n = cpu_elementwise_sample(w)
         cpu["elementwise"] = {**el, "unit": "GB/s", "kind": "oracle",
                               "sample": f"Q/K norm + RoPE and modulation + SwiGLU (residual branch on) of {el_n} "

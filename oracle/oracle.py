@@ -81,6 +81,8 @@ def load(path: str):
               L.oracle_varlen_attn_fp8_online, L.oracle_modulate_swiglu, L.oracle_linear_gated_residual, L.oracle_linear_swiglu):
         f.restype = C.c_int
     L.oracle_num_threads.restype = C.c_int
+    L.oracle_set_num_threads.argtypes = [C.c_int]
+    L.oracle_set_num_threads.restype = None
     return L
 
 
@@ -95,6 +97,11 @@ def lib():
 
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of later oracle calls (timing only; results do not depend on it)."""
+    lib().oracle_set_num_threads(int(n))
 
 
 def _kind(a: np.ndarray) -> int:

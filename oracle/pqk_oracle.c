@@ -968,6 +968,16 @@ int oracle_linear_swiglu(const void* a, int64_t a_stride, const void* w1, int in
   return bad ? -1 : 0;
 }
 
+/* Sets the number of OpenMP threads later parallel regions use (n >= 1);
+ * for timing the oracle on one core beside its all-core figure. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* Number of OpenMP threads a parallel region of this library uses. */
 int oracle_num_threads(void) {
   int n = 1;
