@@ -123,3 +123,19 @@ def test_pairs_pipeline_timeout_is_reported_drained_and_recovered():
     ro, rl = oracle.varlen_attn(x["q"], x["k"], x["v"], x["cu_seqlens"], 1.0 / math.sqrt(D), rows=rows)
     assert_attention(bf16_to_f64(o2)[rows], ro, "CTA pairs after a timed-out call")
     assert max_abs(lse2.cpu().numpy().astype(np.float64).T[rows], rl) <= LSE_MAX_ABS
+
+
+def test_pairs_no_alloc_entry_bitwise():
+    # the no-allocation entry keeps its schedule (512-row work tiles on pairs)
+    # in the library's own array: same results as the one-SM workspace entry
+    torch = torch_cuda()
+    w = wl.custom([1000, 17, 0, 2049], 8, 128, seed=85)
+    x = wl.attention_inputs(w)
+    q, k, v = (to_dev_bf16(x[n]) for n in ("q", "k", "v"))
+    cu = to_dev(x["cu_seqlens"])
+    o1, l1 = pqk.varlen_attn_fwd(q, k, v, cu, want_lse=True)
+    with cta_pairs():
+        o2, l2 = pqk.varlen_attn_fwd_noalloc(q, k, v, cu, want_lse=True)
+        torch.cuda.synchronize()
+        assert pqk.get_device_status() == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
